@@ -1,0 +1,184 @@
+"""Plain fp64 CPU oracle for the fused linear + cross-entropy (FLCE) head.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the package's smoke check and
+the benchmark's CPU-baseline leg may import this module; the product path never
+does, and this module imports nothing from the product.
+
+What it computes is the unfused definition written out in fp64.  The pages say
+the fused head returns the same loss as the plain "linear layer, then
+cross-entropy" pipeline, only without keeping the logit tensor:
+
+* "Liger-Kernel: Triton kernels that replace HF training ops", section "What
+  actually gets replaced": FusedLinearCrossEntropy takes the hidden states and
+  the LM-head weight and returns the loss directly, a drop-in replacement with
+  the same call signature.
+* "Liger Kernel explained", section on the cross-entropy head: the loss and its
+  gradient are computed in chunks over the vocabulary, so the full logit tensor
+  is never resident; a naive head materialises it once for the forward softmax
+  and once more for the gradient.
+* "Complete Guide to Liger Kernel", section LigerFusedLinearCrossEntropyLoss:
+  ``loss = fused_loss_fn(hidden_states, weight, labels)`` with ``weight`` of
+  shape ``(vocab_size, hidden_size)``.
+
+The oracle therefore *does* materialise the logits (that is the plain
+definition) and follows these steps, with ``n`` the number of non-ignored rows:
+
+1. ``valid_i = (y_i != ignore_index)``; a valid ``y_i`` outside ``[0, V)`` is an
+   error.
+2. ``z_ij = x_i . w_j``; ``lse_i = m_i + log(sum_j exp(z_ij - m_i))`` with
+   ``m_i = max_j z_ij``; ``l_i = lse_i - z_{i, y_i}``.
+3. ``loss = (sum over valid i of l_i) / n``  (token mean, the PyTorch
+   ``reduction='mean'`` convention a drop-in replacement implies).
+4. ``G_ij = valid_i * (exp(z_ij - lse_i) - [j == y_i]) / n``  (d loss / d z).
+5. ``dX = G W``  and  ``dW = G^T X``.
+
+Readings where the pages are silent: the mean runs over non-ignored rows; with
+no valid row the loss, dX and dW are all zero (PyTorch would give NaN); there is
+no bias, label smoothing, soft-cap or z-loss term.
+
+Inputs are converted exactly to fp64 (bf16 -> fp64 is exact).  A matrix product
+(numpy/BLAS in fp64) serves as a step; nothing is blocked, fused or reordered
+beyond what the definition states, except that the functions meant for full-size
+workloads evaluate the per-row definition for a block of rows at a time so that
+the fp64 logits of a block, not of the whole batch, are in memory.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+IGNORE_INDEX = -100
+
+
+class TargetOutOfRange(ValueError):
+    """A non-ignored target lies outside [0, V)."""
+
+
+def _f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):  # a torch tensor; bf16 -> fp32 -> fp64 is exact
+        a = a.detach().to("cpu")
+        if str(a.dtype) in ("torch.bfloat16", "torch.float16"):
+            a = a.float()
+        a = a.numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def _i64(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").numpy()
+    return np.asarray(a, dtype=np.int64)
+
+
+def valid_mask(y: np.ndarray, V: int, ignore_index: int = IGNORE_INDEX) -> np.ndarray:
+    """Step 1: which rows count, and the range check on the ones that do."""
+    y = _i64(y)
+    valid = y != ignore_index
+    bad = valid & ((y < 0) | (y >= V))
+    if bad.any():
+        raise TargetOutOfRange(f"target {int(y[bad][0])} outside [0, {V})")
+    return valid
+
+
+def log_sum_exp(Z: np.ndarray) -> np.ndarray:
+    """Step 2: lse_i = m_i + log(sum_j exp(z_ij - m_i)), m_i = max_j z_ij."""
+    m = Z.max(axis=1)
+    return m + np.log(np.exp(Z - m[:, None]).sum(axis=1))
+
+
+def flce_reference(X, W, y, ignore_index: int = IGNORE_INDEX):
+    """The whole definition on full matrices: returns (loss, dX, dW, lse, n).
+
+    For shapes whose N x V fp64 logits fit in host memory.
+    """
+    X = _f64(X)
+    W = _f64(W)
+    y = _i64(y)
+    N, _ = X.shape
+    V = W.shape[0]
+    valid = valid_mask(y, V, ignore_index)
+    n = int(valid.sum())
+    rows = np.arange(N)
+    yv = np.where(valid, y, 0)
+
+    Z = X @ W.T                                   # z_ij = x_i . w_j
+    lse = log_sum_exp(Z)
+    row_loss = np.where(valid, lse - Z[rows, yv], 0.0)
+    loss = float(row_loss.sum() / n) if n else 0.0
+
+    G = np.exp(Z - lse[:, None])                  # softmax
+    G[rows, yv] -= 1.0                            # minus the one-hot target
+    G *= valid[:, None]                           # ignored rows give nothing
+    G *= (1.0 / n) if n else 0.0                  # token mean
+    dX = G @ W
+    dW = G.T @ X
+    return loss, dX, dW, lse, n
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads: the same per-row definition, evaluated on chosen rows.
+# ---------------------------------------------------------------------------
+
+def row_lse(X, W, rows=None, block: int = 256, W64=None) -> np.ndarray:
+    """lse_i (step 2) for the given rows (all rows when ``rows`` is None).
+
+    Rows are independent, so each block of rows is the definition applied to
+    those rows; only memory is bounded by the blocking.
+    """
+    X = _f64(X)
+    if rows is not None:
+        X = X[np.asarray(rows, dtype=np.int64)]
+    W64 = _f64(W) if W64 is None else W64
+    out = np.empty(X.shape[0], dtype=np.float64)
+    for b in range(0, X.shape[0], block):
+        out[b:b + block] = log_sum_exp(X[b:b + block] @ W64.T)
+    return out
+
+
+def full_loss(X, W, y, ignore_index: int = IGNORE_INDEX, block: int = 256, W64=None):
+    """Step 3 over all rows without the N x V matrix: returns (loss, lse, n)."""
+    W64 = _f64(W) if W64 is None else W64
+    X64 = _f64(X)
+    y = _i64(y)
+    V = W64.shape[0]
+    valid = valid_mask(y, V, ignore_index)
+    n = int(valid.sum())
+    lse = row_lse(X64, W64, None, block, W64)
+    yv = np.where(valid, y, 0)
+    zy = np.einsum("ih,ih->i", X64, W64[yv])      # z_{i, y_i}
+    row_loss = np.where(valid, lse - zy, 0.0)
+    loss = float(row_loss.sum() / n) if n else 0.0
+    return loss, lse, n
+
+
+def dx_rows(X, W, y, rows, lse_rows, n: int, ignore_index: int = IGNORE_INDEX, W64=None):
+    """Steps 4-5 for the chosen token rows: dX_i = sum_j G_ij w_j."""
+    W64 = _f64(W) if W64 is None else W64
+    rows = np.asarray(rows, dtype=np.int64)
+    Xr = _f64(X)[rows]
+    yr = _i64(y)[rows]
+    V = W64.shape[0]
+    valid = valid_mask(yr, V, ignore_index)
+    Z = Xr @ W64.T
+    G = np.exp(Z - np.asarray(lse_rows, dtype=np.float64)[:, None])
+    G[np.arange(len(rows)), np.where(valid, yr, 0)] -= 1.0
+    G *= valid[:, None]
+    G *= (1.0 / n) if n else 0.0
+    return G @ W64
+
+
+def dw_rows(X, W, y, vocab_rows, lse, n: int, ignore_index: int = IGNORE_INDEX, W64=None, X64=None):
+    """Steps 4-5 for the chosen vocab entries: dW_j = sum_i G_ij x_i.
+
+    Needs lse_i for every token row (from :func:`full_loss`).
+    """
+    W64 = _f64(W) if W64 is None else W64
+    X64 = _f64(X) if X64 is None else X64
+    y = _i64(y)
+    J = np.asarray(vocab_rows, dtype=np.int64)
+    V = W64.shape[0]
+    valid = valid_mask(y, V, ignore_index)
+    Z = X64 @ W64[J].T                            # z_ij for all i, chosen j
+    G = np.exp(Z - np.asarray(lse, dtype=np.float64)[:, None])
+    G -= (y[:, None] == J[None, :])               # one-hot at the target
+    G *= valid[:, None]
+    G *= (1.0 / n) if n else 0.0
+    return G.T @ X64

@@ -1,0 +1,250 @@
+"""Checks that pin the fp64 oracle to facts outside itself.
+
+Each ``pin_*`` takes the oracle module and raises ``AssertionError`` when the
+module disagrees with a closed form, a textbook special case, a library routine
+used as a brute force (torch fp64 cross-entropy plus autograd), central finite
+differences or an invariant of the method.  ``test_oracle.py`` runs them on the
+oracle; ``test_oracle_mutants.py`` runs them on copies of the oracle with one
+planted mistake each and requires that some pin fails.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+IGN = -100
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _case(seed, N, H, V, n_ign=1, scale_x=1.0, scale_w=0.3):
+    r = _rng(seed)
+    X = r.standard_normal((N, H)) * scale_x
+    W = r.standard_normal((V, H)) * scale_w
+    y = r.integers(0, V, size=N)
+    if n_ign:
+        y[r.permutation(N)[:n_ign]] = IGN
+    return X, W, y
+
+
+def _close(a, b, rtol, atol=0.0, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    lim = atol + rtol * (np.max(np.abs(b)) if b.size else 0.0)
+    assert err <= lim, f"{what}: max err {err:.3e} > {lim:.3e}"
+
+
+def pin_zero_weight(orc):
+    """W = 0: every logit is 0, softmax is uniform 1/V.
+
+    loss = ln V exactly; dX = 0; dW_j = (1/n) sum_valid (1/V - [y_i = j]) x_i.
+    """
+    N, H, V = 7, 5, 11
+    X, _, y = _case(1, N, H, V, n_ign=2)
+    W = np.zeros((V, H))
+    loss, dX, dW, _, n = orc.flce_reference(X, W, y)
+    assert n == N - 2
+    assert abs(loss - math.log(V)) <= 1e-15 * math.log(V), loss
+    assert np.all(dX == 0.0)
+    want = np.zeros((V, H))
+    for i in range(N):
+        if y[i] == IGN:
+            continue
+        for j in range(V):
+            want[j] += ((1.0 / V) - (1.0 if y[i] == j else 0.0)) * X[i] / n
+    _close(dW, want, 1e-13, what="dW at W=0")
+
+
+def pin_zero_input(orc):
+    """X = 0: loss = ln V, dW = 0, dX_i = valid_i (mean_j w_j - w_{y_i}) / n."""
+    N, H, V = 6, 4, 9
+    _, W, y = _case(2, N, H, V, n_ign=1)
+    X = np.zeros((N, H))
+    loss, dX, dW, _, n = orc.flce_reference(X, W, y)
+    assert abs(loss - math.log(V)) <= 1e-15 * math.log(V)
+    assert np.all(dW == 0.0)
+    wbar = W.mean(axis=0)
+    for i in range(N):
+        want = np.zeros(H) if y[i] == IGN else (wbar - W[y[i]]) / n
+        _close(dX[i], want, 1e-13, atol=1e-16, what=f"dX row {i} at X=0")
+
+
+def pin_two_class(orc):
+    """V = 2 is logistic regression: l_i = softplus(z_other - z_target),
+    dX_i = sigmoid(z_other - z_target) (w_other - w_target) / n."""
+    N, H = 9, 6
+    X, W, y = _case(3, N, H, 2, n_ign=2, scale_w=0.8)
+    loss, dX, dW, _, n = orc.flce_reference(X, W, y)
+    tot = 0.0
+    for i in range(N):
+        if y[i] == IGN:
+            assert np.all(dX[i] == 0.0)
+            continue
+        t, o = int(y[i]), 1 - int(y[i])
+        d = float(X[i] @ W[o] - X[i] @ W[t])
+        tot += max(d, 0.0) + math.log1p(math.exp(-abs(d)))
+        sig = 1.0 / (1.0 + math.exp(-d))
+        _close(dX[i], sig * (W[o] - W[t]) / n, 1e-12, atol=1e-15, what=f"dX row {i}, V=2")
+    assert abs(loss - tot / n) <= 1e-13 * abs(tot / n), (loss, tot / n)
+
+
+def pin_large_logits(orc):
+    """Logits of magnitude ~1e3 overflow a naive exp; the max-shifted lse must
+    stay finite and equal softplus(d) = d + log1p(exp(-d)) for V = 2."""
+    X = np.array([[30.0, -20.0], [-25.0, 40.0]])
+    W = np.array([[20.0, 10.0], [-15.0, 12.0]])
+    y = np.array([0, 0])
+    loss, dX, dW, lse, n = orc.flce_reference(X, W, y)
+    tot = 0.0
+    for i in range(2):
+        d = float(X[i] @ W[1] - X[i] @ W[0])
+        tot += max(d, 0.0) + math.log1p(math.exp(-abs(d)))
+    assert np.isfinite(loss) and np.all(np.isfinite(dX)) and np.all(np.isfinite(dW))
+    assert abs(loss - tot / 2) <= 1e-13 * abs(tot / 2), (loss, tot / 2)
+
+
+def pin_torch_autograd(orc):
+    """Brute force through another library: torch fp64 logits, torch's own
+    cross_entropy(ignore_index=-100, mean) and autograd for both gradients."""
+    for seed, (N, H, V, ig) in enumerate([(5, 3, 7, 1), (16, 12, 33, 4), (3, 8, 2, 0), (40, 24, 130, 7)]):
+        X, W, y = _case(10 + seed, N, H, V, n_ign=ig)
+        loss, dX, dW, _, _ = orc.flce_reference(X, W, y)
+        tX = torch.tensor(X, dtype=torch.float64, requires_grad=True)
+        tW = torch.tensor(W, dtype=torch.float64, requires_grad=True)
+        ty = torch.tensor(y, dtype=torch.int64)
+        tl = torch.nn.functional.cross_entropy(tX @ tW.T, ty, ignore_index=IGN, reduction="mean")
+        tl.backward()
+        assert abs(loss - tl.item()) <= 1e-12 * abs(tl.item()), (loss, tl.item())
+        _close(dX, tX.grad.numpy(), 1e-11, what="dX vs autograd")
+        _close(dW, tW.grad.numpy(), 1e-11, what="dW vs autograd")
+
+
+def pin_finite_difference(orc):
+    """Central differences of the loss against every entry of X and W."""
+    N, H, V = 4, 8, 16
+    X, W, y = _case(20, N, H, V, n_ign=1)
+    _, dX, dW, _, _ = orc.flce_reference(X, W, y)
+    h = 1e-5
+
+    def L(Xa, Wa):
+        return orc.flce_reference(Xa, Wa, y)[0]
+
+    for (A, dA, is_x) in ((X, dX, True), (W, dW, False)):
+        fd = np.zeros_like(A)
+        for idx in np.ndindex(A.shape):
+            Ap, Am = A.copy(), A.copy()
+            Ap[idx] += h
+            Am[idx] -= h
+            lp = L(Ap, W) if is_x else L(X, Ap)
+            lm = L(Am, W) if is_x else L(X, Am)
+            fd[idx] = (lp - lm) / (2 * h)
+        _close(dA, fd, 1e-6, atol=1e-9, what="finite differences")
+
+
+def pin_rows_of_g_sum_to_zero(orc):
+    """sum_j (softmax - onehot)_ij = 0 for every row, hence sum_j dW_j = 0."""
+    X, W, y = _case(30, 12, 10, 50, n_ign=3)
+    _, dX, dW, _, _ = orc.flce_reference(X, W, y)
+    s = dW.sum(axis=0)
+    assert np.max(np.abs(s)) <= 1e-13 * np.max(np.abs(dW)) * 50, s
+
+
+def pin_shift_invariance(orc):
+    """w_j -> w_j + c for every j adds x_i.c to a whole row of logits, which
+    leaves softmax, loss and dX unchanged."""
+    X, W, y = _case(40, 10, 6, 20, n_ign=2)
+    c = _rng(41).standard_normal(6)
+    l0, dX0, _, _, _ = orc.flce_reference(X, W, y)
+    l1, dX1, _, _, _ = orc.flce_reference(X, W + c[None, :], y)
+    assert abs(l0 - l1) <= 1e-12 * abs(l0)
+    _close(dX1, dX0, 1e-11, atol=1e-15, what="dX under shift")
+
+
+def pin_ignored_rows(orc):
+    """Ignored rows give exactly zero dX, and changing their hidden state moves
+    neither the loss nor dW."""
+    X, W, y = _case(50, 10, 6, 20, n_ign=4)
+    l0, dX0, dW0, _, _ = orc.flce_reference(X, W, y)
+    ign = y == IGN
+    assert np.all(dX0[ign] == 0.0)
+    X2 = X.copy()
+    X2[ign] += 5.0
+    l1, _, dW1, _, _ = orc.flce_reference(X2, W, y)
+    assert abs(l0 - l1) <= 1e-15 * abs(l0)
+    _close(dW1, dW0, 1e-14, what="dW after moving ignored rows")
+
+
+def pin_no_valid_rows(orc):
+    """Reading for n_valid = 0: loss 0 and zero gradients."""
+    X, W, _ = _case(60, 5, 4, 9, n_ign=0)
+    y = np.full(5, IGN)
+    loss, dX, dW, _, n = orc.flce_reference(X, W, y)
+    assert n == 0 and loss == 0.0 and np.all(dX == 0) and np.all(dW == 0)
+
+
+def pin_target_range(orc):
+    X, W, _ = _case(61, 3, 4, 9, n_ign=0)
+    for bad in (-1, 9, 1000):
+        try:
+            orc.flce_reference(X, W, np.array([0, bad, 2]))
+        except orc.TargetOutOfRange:
+            continue
+        except Exception as e:  # crashed instead of reporting the bad target
+            raise AssertionError(f"target {bad}: {type(e).__name__} instead of TargetOutOfRange")
+        raise AssertionError(f"target {bad} accepted")
+
+
+def pin_permutations(orc):
+    """Relabelling the vocabulary permutes dW's rows; reordering tokens
+    permutes dX's rows; neither changes the loss."""
+    X, W, y = _case(70, 11, 7, 23, n_ign=2)
+    l0, dX0, dW0, _, _ = orc.flce_reference(X, W, y)
+    p = _rng(71).permutation(23)        # new vocab index k holds old entry p[k]
+    inv = np.argsort(p)
+    y2 = np.where(y == IGN, IGN, inv[np.where(y == IGN, 0, y)])
+    l1, dX1, dW1, _, _ = orc.flce_reference(X, W[p], y2)
+    assert abs(l0 - l1) <= 1e-13 * abs(l0)
+    _close(dX1, dX0, 1e-12, atol=1e-16, what="dX under vocab relabel")
+    _close(dW1, dW0[p], 1e-12, atol=1e-16, what="dW under vocab relabel")
+    q = _rng(72).permutation(11)
+    l2, dX2, dW2, _, _ = orc.flce_reference(X[q], W, y[q])
+    assert abs(l0 - l2) <= 1e-13 * abs(l0)
+    _close(dX2, dX0[q], 1e-12, atol=1e-16, what="dX under token reorder")
+    _close(dW2, dW0, 1e-12, atol=1e-16, what="dW under token reorder")
+
+
+def pin_equal_logits(orc):
+    """All w_j equal: every row is uniform, lse_i = z_i + ln V."""
+    X, _, y = _case(80, 6, 5, 13, n_ign=1)
+    w = _rng(81).standard_normal(5)
+    W = np.tile(w, (13, 1))
+    _, _, _, lse, _ = orc.flce_reference(X, W, y)
+    _close(lse, X @ w + math.log(13), 1e-14, what="lse with equal rows")
+
+
+def pin_row_functions(orc):
+    """The row-subset functions used at full size give what the whole-matrix
+    definition gives on a case where both run."""
+    X, W, y = _case(90, 300, 16, 700, n_ign=30)
+    loss, dX, dW, lse, n = orc.flce_reference(X, W, y)
+    l2, lse2, n2 = orc.full_loss(X, W, y, block=64)
+    assert n2 == n and abs(l2 - loss) <= 1e-13 * abs(loss)
+    _close(lse2, lse, 1e-14, what="row lse")
+    rows = np.array([0, 5, 77, 299])
+    _close(orc.dx_rows(X, W, y, rows, lse[rows], n), dX[rows], 1e-12, atol=1e-18, what="dx_rows")
+    J = np.array([0, 1, 350, 699])
+    _close(orc.dw_rows(X, W, y, J, lse, n), dW[J], 1e-12, atol=1e-18, what="dw_rows")
+    _close(orc.row_lse(X, W, rows), lse[rows], 1e-14, what="row_lse subset")
+
+
+ALL_PINS = [
+    pin_zero_weight, pin_zero_input, pin_two_class, pin_large_logits,
+    pin_torch_autograd, pin_finite_difference, pin_rows_of_g_sum_to_zero,
+    pin_shift_invariance, pin_ignored_rows, pin_no_valid_rows, pin_target_range,
+    pin_permutations, pin_equal_logits, pin_row_functions,
+]

@@ -1,0 +1,54 @@
+"""Plants one plausible mistake at a time in a copy of the oracle and checks that
+the pins catch it.  The mistakes are edits of the oracle's own source text, made
+on the CPU; the real module is never touched."""
+import importlib.util
+import inspect
+import types
+
+import pytest
+
+import oracle_pins
+from oracle import flce_oracle
+
+# (description, original text, mutated text); each original must occur in the source.
+MUTATIONS = [
+    ("one-hot added instead of subtracted", "G[rows, yv] -= 1.0", "G[rows, yv] += 1.0"),
+    ("ignored rows not masked in G", "G *= valid[:, None]                           # ignored rows",
+     "G *= 1.0                                      # ignored rows"),
+    ("mean over all rows, not valid rows", "G *= (1.0 / n) if n else 0.0                  # token mean",
+     "G *= (1.0 / N) if n else 0.0                  # token mean"),
+    ("softmax not normalised", "G = np.exp(Z - lse[:, None])                  # softmax",
+     "G = np.exp(Z)                                 # softmax"),
+    ("max dropped from log-sum-exp", "return m + np.log(np.exp(Z - m[:, None]).sum(axis=1))",
+     "return np.log(np.exp(Z - m[:, None]).sum(axis=1))"),
+    ("target logit added to the row loss", "row_loss = np.where(valid, lse - Z[rows, yv], 0.0)",
+     "row_loss = np.where(valid, lse + Z[rows, yv], 0.0)"),
+    ("dW from X transposed against G", "dW = G.T @ X", "dW = (X.T @ G).T * 0 + G.T @ (X * 0.5)"),
+    ("dX against the wrong operand", "dX = G @ W", "dX = G @ (W - W.mean(axis=0)) * 0.5"),
+    ("full-size loss drops the target logit", "row_loss = np.where(valid, lse - zy, 0.0)",
+     "row_loss = np.where(valid, lse, 0.0)"),
+    ("full-size dW one-hot sign", "G -= (y[:, None] == J[None, :])", "G += (y[:, None] == J[None, :])"),
+    ("full-size dX ignores the valid mask", "    G *= valid[:, None]\n    G *= (1.0 / n) if n else 0.0\n    return G @ W64",
+     "    G *= (1.0 / n) if n else 0.0\n    return G @ W64"),
+    ("target range not checked", "bad = valid & ((y < 0) | (y >= V))", "bad = valid & (y < -10**9)"),
+]
+
+
+def _mutant(orig, new):
+    src = inspect.getsource(flce_oracle)
+    assert src.count(orig) == 1, f"mutation anchor not unique/present: {orig!r}"
+    mod = types.ModuleType("flce_oracle_mutant")
+    exec(compile(src.replace(orig, new), "<mutant>", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("desc,orig,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutant(desc, orig, new):
+    mod = _mutant(orig, new)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(mod)
+        except Exception as e:  # AssertionError, or a crash the mistake causes
+            caught.append(f"{pin.__name__}: {type(e).__name__}")
+    assert caught, f"no pin caught the planted mistake: {desc}"
