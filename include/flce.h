@@ -1,0 +1,145 @@
+/*
+ * flce.h -- C ABI of the fused linear + cross-entropy (FLCE) head for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operation.  Given hidden states X[N,H] and an LM-head weight W[V,H] (one
+ * row per vocabulary entry) and integer targets y[N], the head returns the
+ * token-mean cross-entropy of the logits z = X W^T against y, and the
+ * gradients of that loss with respect to X and W, without ever holding the
+ * N x V logit tensor in device memory:
+ *
+ *   valid_i = (y_i != ignore_index),       n = sum_i valid_i
+ *   lse_i   = log sum_j exp(z_ij)
+ *   loss    = (1/n) sum_{valid i} (lse_i - z_{i,y_i})
+ *   G_ij    = valid_i (exp(z_ij - lse_i) - [j == y_i]) / n
+ *   dX      = G W,      dW = G^T X
+ *
+ * Sources: "Liger-Kernel: Triton kernels that replace HF training ops",
+ * section "What actually gets replaced" (FusedLinearCrossEntropy consumes the
+ * hidden states and the LM-head weight and produces the loss directly, the
+ * (batch, sequence, vocab) tensor is never allocated, same call signature as
+ * the unfused modules); "Liger Kernel explained", section on the
+ * cross-entropy head (loss and gradient computed in chunks over the
+ * vocabulary, intermediates recomputed instead of stored); "Complete Guide to
+ * Liger Kernel", section LigerFusedLinearCrossEntropyLoss (the call takes
+ * hidden states, a (vocab_size, hidden_size) weight and labels).  The pages
+ * never state the ignore value or the mean's denominator; this library reads
+ * them as PyTorch's: targets equal to ignore_index (normally -100) are
+ * skipped and the mean runs over the n non-ignored rows.  With n = 0 the
+ * loss, dX and dW are all zero.
+ *
+ * Layouts.  Every matrix is row-major and contiguous.  X, W, dX and dW hold
+ * bf16 values (passed as uint16_t bit patterns); y holds int32 targets; the
+ * loss is an fp32 scalar.  H must be a multiple of 8 (16-byte rows for the
+ * tensor-memory-access engine); X, W, dX and dW must be 16-byte aligned and
+ * the workspace 256-byte aligned.
+ *
+ * Ownership.  All device pointers belong to the caller.  The library never
+ * allocates device memory: scratch space is the caller's `workspace`, at least
+ * flce_workspace_size(N, H, V) bytes, whose size depends on N and H only.  dX
+ * and dW are overwritten, not accumulated into.  The library keeps only
+ * read-only host caches (device properties, a driver entry point).
+ *
+ * Errors.  Argument errors are found on the host and returned before anything
+ * is launched.  Errors found on the device (a valid target outside [0, V), a
+ * bounded wait inside a kernel that ran out) are written to a device status
+ * word; the synchronous entry points read it back and return it.  Nothing
+ * traps or asserts on the device.
+ */
+#ifndef FLCE_H_
+#define FLCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FLCE_OK = 0,
+  FLCE_ERR_INVALID_ARGUMENT = 1,    /* NULL pointer, non-positive size, size too large */
+  FLCE_ERR_UNSUPPORTED = 2,         /* H % 8 != 0, misaligned pointer, device is not sm_100 */
+  FLCE_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < flce_workspace_size(N, H, V) */
+  FLCE_ERR_TARGET_OUT_OF_RANGE = 4, /* some y_i != ignore_index lies outside [0, V) */
+  FLCE_ERR_TIMEOUT = 5,             /* a bounded wait inside a kernel gave up */
+  FLCE_ERR_CUDA = 6                 /* a CUDA runtime call failed */
+} flce_status_t;
+
+/* Human-readable name of a status code (static storage). */
+const char* flce_status_string(int status);
+
+/* Bytes of device workspace one call needs.  Depends on N and H only (V is
+ * accepted for symmetry and ignored): the logits are processed one vocabulary
+ * chunk of fixed width at a time.  Returns 0 for invalid sizes. */
+size_t flce_workspace_size(int64_t N, int64_t H, int64_t V);
+
+/* Synchronous forward + backward.
+ *   X  [N,H] bf16, device      W  [V,H] bf16, device      y [N] int32, device
+ *   loss: HOST float*, receives the token-mean loss
+ *   dX [N,H] bf16, device (out)   dW [V,H] bf16, device (out)
+ *   workspace: device, >= flce_workspace_size(N, H, V) bytes, 256-B aligned
+ *   stream: the CUDA stream to run on (0 = legacy default stream)
+ * Blocks the calling host thread until the stream has finished the call, then
+ * returns FLCE_OK or the first error seen, including device-side errors. */
+flce_status_t flce_forward_backward(const uint16_t* X, const uint16_t* W, const int32_t* y,
+                                    int64_t N, int64_t H, int64_t V, int32_t ignore_index,
+                                    float* loss, uint16_t* dX, uint16_t* dW, void* workspace,
+                                    cudaStream_t stream);
+
+/* Asynchronous twin: enqueues the whole computation on `stream` and returns.
+ *   d_loss:   DEVICE float*, receives the loss when the stream gets there
+ *   d_status: DEVICE int32_t*, receives 0 or a device-side flce_status_t
+ *   workspace_bytes: size of `workspace`, checked against flce_workspace_size
+ * Host-side argument errors are returned immediately; device-side errors only
+ * appear in *d_status. */
+flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, const int32_t* y,
+                                          int64_t N, int64_t H, int64_t V, int32_t ignore_index,
+                                          float* d_loss, int32_t* d_status, uint16_t* dX,
+                                          uint16_t* dW, void* workspace, size_t workspace_bytes,
+                                          cudaStream_t stream);
+
+/* End-to-end entry for callers whose data sits in HOST memory.
+ *   h_X, h_W, h_y: host inputs (pinned memory gives full copy bandwidth)
+ *   h_loss, h_dX, h_dW: host outputs
+ *   d_X, d_W, d_y, d_dX, d_dW, workspace: caller-owned device buffers of the
+ *   same shapes (workspace >= flce_workspace_size bytes)
+ * Copies the inputs to the device, runs the computation, copies loss, dX and
+ * dW back, and waits for the stream.  No allocation happens inside. */
+flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_W,
+                                         const int32_t* h_y, int64_t N, int64_t H, int64_t V,
+                                         int32_t ignore_index, float* h_loss, uint16_t* h_dX,
+                                         uint16_t* h_dW, uint16_t* d_X, uint16_t* d_W,
+                                         int32_t* d_y, uint16_t* d_dX, uint16_t* d_dW,
+                                         void* workspace, size_t workspace_bytes,
+                                         cudaStream_t stream);
+
+/* How a call of these sizes is split into launches (host-only query). */
+typedef struct {
+  int64_t workspace_bytes; /* same as flce_workspace_size */
+  int32_t vocab_chunk;     /* vocabulary entries per pass-2 chunk */
+  int32_t num_chunks;      /* pass-2 chunks */
+  int32_t lse_splits;      /* vocabulary splits of the pass-1 log-sum-exp */
+  int32_t launches;        /* kernels launched by one call */
+  int32_t num_sms;         /* SMs the persistent kernels are sized for */
+} flce_plan_t;
+flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out);
+
+/* Per-kernel timing.  While enabled, every launch of the library is bracketed
+ * by CUDA events on its stream.  flce_profile_read waits for those events and
+ * returns, per kernel kind, the number of launches and their summed device
+ * time in milliseconds, then clears the record.  kinds: 0 pass-1 GEMM +
+ * online log-sum-exp, 1 combine, 2 pass-2 logits recompute + G, 3 dW
+ * contraction, 4 dX contraction. */
+#define FLCE_NUM_KERNEL_KINDS 5
+const char* flce_kernel_name(int kind);
+flce_status_t flce_profile_enable(int on);
+flce_status_t flce_profile_read(int32_t* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLCE_H_ */

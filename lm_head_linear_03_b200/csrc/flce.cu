@@ -1,0 +1,515 @@
+// Host side of the FLCE library: argument checks, workspace carving, TMA
+// descriptors, the launch plan and the C ABI declared in include/flce.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "flce.h"
+#include "flce_kernels.cuh"
+
+namespace {
+
+using namespace flce;
+
+// Vocabulary entries per pass-2 chunk.  The G chunk buffer is N x VC bf16, so
+// the workspace stays independent of V.
+constexpr int VC = 2048;
+constexpr int MAX_SPLITS = 64;
+constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per bounded wait
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t ctrl, lse2, zy, part_m, part_l, blk_loss, blk_cnt, G, lo, total;
+};
+
+// ctrl block: [0] status, [4] ticket, [8] n_valid, [12] inv_n, [16] loss
+struct Ctrl {
+  int32_t status;
+  uint32_t ticket;
+  int32_t n_valid;
+  float inv_n;
+  float loss;
+};
+
+WsLayout ws_layout(int64_t N, int64_t H) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t n = static_cast<size_t>(N);
+  const size_t nblk = (n + COMBINE_THREADS - 1) / COMBINE_THREADS;
+  L.ctrl = take(256);
+  L.lse2 = take(n * 4);
+  L.zy = take(n * 4);
+  L.part_m = take(static_cast<size_t>(MAX_SPLITS) * n * 4);
+  L.part_l = take(static_cast<size_t>(MAX_SPLITS) * n * 4);
+  L.blk_loss = take(nblk * 8);
+  L.blk_cnt = take(nblk * 4);
+  L.G = take(n * VC * 2);
+  L.lo = take(n * static_cast<size_t>(H) * 2);
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------ device info --
+struct DevInfo {
+  bool ok = false;
+  bool sm100 = false;
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+DevInfo g_dev[64];
+bool g_attr_set[64];
+
+cudaError_t device_info(DevInfo* out, int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_dev[dev].ok) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    g_dev[dev].sm100 = (major == 10 && minor == 0);
+    g_dev[dev].num_sms = sms;
+    g_dev[dev].ok = true;
+  }
+  *out = g_dev[dev];
+  *dev_out = dev;
+  return cudaSuccess;
+}
+
+cudaError_t set_kernel_attrs(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_attr_set[dev]) return cudaSuccess;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_GRAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_DW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_DX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES)) != cudaSuccess)
+    return e;
+  g_attr_set[dev] = true;
+  return cudaSuccess;
+}
+
+// ------------------------------------------------------------ tensor maps --
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool get_encode() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return false;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return true;
+}
+
+// 2-D bf16 row-major tensor [outer][inner], 128-B swizzled boxes of
+// box_inner x box_outer elements; out-of-range elements read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+              uint32_t box_inner, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ plan --
+struct Plan {
+  int tiles_m;        // 128-token tiles
+  int vtiles;         // 256-wide vocabulary tiles
+  int splits;         // pass-1 vocabulary splits
+  int lse_grid;
+  int num_chunks;
+  int launches;
+  int num_sms;
+};
+
+// Pass 1: pick the number of vocabulary splits whose units, dealt round-robin
+// to one persistent CTA per SM, give the smallest largest per-CTA tile count.
+int choose_splits(int tiles_m, int vtiles, int sms) {
+  int best = 1;
+  long long best_cost = LLONG_MAX;
+  const int smax = std::min(MAX_SPLITS, vtiles);
+  std::vector<long long> load;
+  for (int S = 1; S <= smax; ++S) {
+    const long long units = static_cast<long long>(tiles_m) * S;
+    const int grid = static_cast<int>(std::min<long long>(units, sms));
+    load.assign(grid, 0);
+    for (long long u = 0; u < units; ++u) {
+      const long long s = u / tiles_m;
+      const long long n = ((s + 1) * vtiles) / S - (s * vtiles) / S;
+      load[u % grid] += n + 1;  // +1: per-unit pipeline fill and partial write
+    }
+    const long long cost = *std::max_element(load.begin(), load.end());
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
+Plan make_plan(int64_t N, int64_t H, int64_t V, int sms) {
+  (void)H;
+  Plan p{};
+  p.num_sms = sms;
+  p.tiles_m = static_cast<int>((N + BM - 1) / BM);
+  p.vtiles = static_cast<int>((V + BN - 1) / BN);
+  p.splits = choose_splits(p.tiles_m, p.vtiles, sms);
+  p.lse_grid = static_cast<int>(std::min<long long>(static_cast<long long>(p.tiles_m) * p.splits, sms));
+  p.num_chunks = static_cast<int>((V + VC - 1) / VC);
+  p.launches = 2 + 3 * p.num_chunks;
+  return p;
+}
+
+// ------------------------------------------------------------- profiling --
+struct Prof {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;  // pairs
+  std::vector<int> kind;
+  size_t used = 0;
+};
+Prof g_prof;
+constexpr size_t PROF_PAIRS = 16384;
+
+void prof_begin(cudaStream_t s, int k, size_t* slot) {
+  *slot = SIZE_MAX;
+  if (!g_prof.on || g_prof.used >= PROF_PAIRS) return;
+  *slot = g_prof.used++;
+  g_prof.kind[*slot] = k;
+  cudaEventRecord(g_prof.ev[2 * *slot], s);
+}
+void prof_end(cudaStream_t s, size_t slot) {
+  if (slot != SIZE_MAX) cudaEventRecord(g_prof.ev[2 * slot + 1], s);
+}
+
+// ---------------------------------------------------------------- checks --
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+flce_status_t check_sizes(int64_t N, int64_t H, int64_t V) {
+  if (N <= 0 || H <= 0 || V <= 0) return FLCE_ERR_INVALID_ARGUMENT;
+  if (N > (1ll << 30) || V > (1ll << 30) || H > (1ll << 20)) return FLCE_ERR_INVALID_ARGUMENT;
+  if (H % 8 != 0) return FLCE_ERR_UNSUPPORTED;
+  return FLCE_OK;
+}
+
+flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N, int64_t H, int64_t V,
+                         const void* dX, const void* dW, const void* ws) {
+  const flce_status_t s = check_sizes(N, H, V);
+  if (s != FLCE_OK) return s;
+  if (!X || !W || !y || !dX || !dW || !ws) return FLCE_ERR_INVALID_ARGUMENT;
+  if (!aligned(X, 16) || !aligned(W, 16) || !aligned(dX, 16) || !aligned(dW, 16) || !aligned(y, 4) ||
+      !aligned(ws, 256))
+    return FLCE_ERR_UNSUPPORTED;
+  return FLCE_OK;
+}
+
+// --------------------------------------------------------------- enqueue --
+template <int KIND>
+cudaError_t launch_gemm(int grid, cudaStream_t s, const CUtensorMap& mA, const CUtensorMap& mB,
+                        const GemmArgs& a, int kind) {
+  size_t slot;
+  prof_begin(s, kind, &slot);
+  flce_gemm_kernel<KIND><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, a);
+  prof_end(s, slot);
+  return cudaGetLastError();
+}
+
+flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
+                      int32_t ignore_index, float* d_loss, int32_t* d_status, uint16_t* dX, uint16_t* dW,
+                      void* workspace, cudaStream_t stream) {
+  DevInfo di;
+  int dev;
+  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
+  if (set_kernel_attrs(dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (!get_encode()) return FLCE_ERR_CUDA;
+
+  const WsLayout L = ws_layout(N, H);
+  const Plan P = make_plan(N, H, V, di.num_sms);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
+  float* lse2 = reinterpret_cast<float*>(ws + L.lse2);
+  float* zy = reinterpret_cast<float*>(ws + L.zy);
+  float* part_m = reinterpret_cast<float*>(ws + L.part_m);
+  float* part_l = reinterpret_cast<float*>(ws + L.part_l);
+  uint16_t* G = reinterpret_cast<uint16_t*>(ws + L.G);
+  uint16_t* lo = reinterpret_cast<uint16_t*>(ws + L.lo);
+
+  CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn;
+  const uint64_t n = static_cast<uint64_t>(N), h = static_cast<uint64_t>(H), v = static_cast<uint64_t>(V);
+  bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BN) &&
+            make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
+            make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK);
+  if (!ok) return FLCE_ERR_CUDA;
+
+  if (cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (d_status != &ctrl->status && cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+
+  GemmArgs a{};
+  a.N = static_cast<int>(N);
+  a.H = static_cast<int>(H);
+  a.V = static_cast<int>(V);
+  a.ignore_index = ignore_index;
+  a.Vc = VC;
+  a.y = y;
+  a.part_m = part_m;
+  a.part_l = part_l;
+  a.zy = zy;
+  a.lse2 = lse2;
+  a.inv_n = &ctrl->inv_n;
+  a.G = G;
+  a.dW = dW;
+  a.dX = dX;
+  a.lo = lo;
+  a.status = d_status;
+  a.timeout_ns = DEFAULT_TIMEOUT_NS;
+
+  // Pass 1: logits tile by tile, online log-sum-exp per (row, split).
+  {
+    GemmArgs p1 = a;
+    p1.tiles_m = P.tiles_m;
+    p1.tiles_n = P.vtiles;
+    p1.k_blocks = static_cast<int>((H + BK - 1) / BK);
+    p1.splits = P.splits;
+    p1.num_units = P.tiles_m * P.splits;
+    p1.vbase = 0;
+    p1.vcount = static_cast<int>(V);
+    if (launch_gemm<KIND_LSE>(P.lse_grid, stream, mX_k, mW_k, p1, KIND_LSE) != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  // Combine the splits: lse, loss, n_valid, 1/n.
+  {
+    CombineArgs c{};
+    c.N = static_cast<int>(N);
+    c.V = static_cast<int>(V);
+    c.ignore_index = ignore_index;
+    c.splits = P.splits;
+    c.y = y;
+    c.part_m = part_m;
+    c.part_l = part_l;
+    c.zy = zy;
+    c.lse2 = lse2;
+    c.blk_loss = reinterpret_cast<double*>(ws + L.blk_loss);
+    c.blk_cnt = reinterpret_cast<int*>(ws + L.blk_cnt);
+    c.ticket = &ctrl->ticket;
+    c.n_valid = &ctrl->n_valid;
+    c.inv_n = &ctrl->inv_n;
+    c.loss = d_loss;
+    c.status = d_status;
+    const int grid = static_cast<int>((N + COMBINE_THREADS - 1) / COMBINE_THREADS);
+    size_t slot;
+    prof_begin(stream, KIND_COMBINE, &slot);
+    flce_combine_kernel<<<grid, COMBINE_THREADS, 0, stream>>>(c);
+    prof_end(stream, slot);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  // Pass 2, one vocabulary chunk at a time.
+  for (int ch = 0; ch < P.num_chunks; ++ch) {
+    const int vbase = ch * VC;
+    const int vcount = static_cast<int>(std::min<int64_t>(VC, V - vbase));
+    GemmArgs b = a;
+    b.vbase = vbase;
+    b.vcount = vcount;
+    b.first_chunk = ch == 0;
+    b.last_chunk = ch == P.num_chunks - 1;
+    {  // recompute logits, G chunk
+      GemmArgs g = b;
+      g.tiles_m = P.tiles_m;
+      g.tiles_n = (vcount + BN - 1) / BN;
+      g.k_blocks = static_cast<int>((H + BK - 1) / BK);
+      g.num_units = g.tiles_m * g.tiles_n;
+      const int grid = std::min(g.num_units, di.num_sms);
+      if (launch_gemm<KIND_GRAD>(grid, stream, mX_k, mW_k, g, KIND_GRAD) != cudaSuccess) return FLCE_ERR_CUDA;
+    }
+    {  // dW rows of the chunk
+      GemmArgs d = b;
+      d.tiles_m = (vcount + BM - 1) / BM;
+      d.tiles_n = static_cast<int>((H + BN - 1) / BN);
+      d.k_blocks = static_cast<int>((N + BK - 1) / BK);
+      d.num_units = d.tiles_m * d.tiles_n;
+      const int grid = std::min(d.num_units, di.num_sms);
+      if (launch_gemm<KIND_DW>(grid, stream, mG_mn, mX_mn, d, KIND_DW) != cudaSuccess) return FLCE_ERR_CUDA;
+    }
+    {  // dX accumulation
+      GemmArgs d = b;
+      d.tiles_m = P.tiles_m;
+      d.tiles_n = static_cast<int>((H + BN - 1) / BN);
+      d.k_blocks = (vcount + BK - 1) / BK;
+      d.num_units = d.tiles_m * d.tiles_n;
+      const int grid = std::min(d.num_units, di.num_sms);
+      if (launch_gemm<KIND_DX>(grid, stream, mG_k, mW_mn, d, KIND_DX) != cudaSuccess) return FLCE_ERR_CUDA;
+    }
+  }
+  return FLCE_OK;
+}
+
+}  // namespace
+
+// ================================================================== C ABI ==
+extern "C" {
+
+const char* flce_status_string(int s) {
+  switch (s) {
+    case FLCE_OK: return "FLCE_OK";
+    case FLCE_ERR_INVALID_ARGUMENT: return "FLCE_ERR_INVALID_ARGUMENT";
+    case FLCE_ERR_UNSUPPORTED: return "FLCE_ERR_UNSUPPORTED";
+    case FLCE_ERR_WORKSPACE_TOO_SMALL: return "FLCE_ERR_WORKSPACE_TOO_SMALL";
+    case FLCE_ERR_TARGET_OUT_OF_RANGE: return "FLCE_ERR_TARGET_OUT_OF_RANGE";
+    case FLCE_ERR_TIMEOUT: return "FLCE_ERR_TIMEOUT";
+    case FLCE_ERR_CUDA: return "FLCE_ERR_CUDA";
+    default: return "FLCE_UNKNOWN_STATUS";
+  }
+}
+
+size_t flce_workspace_size(int64_t N, int64_t H, int64_t V) {
+  if (check_sizes(N, H, V == 0 ? 1 : V) != FLCE_OK) return 0;
+  return ws_layout(N, H).total;
+}
+
+flce_status_t flce_forward_backward(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H,
+                                    int64_t V, int32_t ignore_index, float* loss, uint16_t* dX, uint16_t* dW,
+                                    void* workspace, cudaStream_t stream) {
+  if (!loss) return FLCE_ERR_INVALID_ARGUMENT;
+  flce_status_t s = check_args(X, W, y, N, H, V, dX, dW, workspace);
+  if (s != FLCE_OK) return s;
+  const WsLayout L = ws_layout(N, H);
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(static_cast<uint8_t*>(workspace) + L.ctrl);
+  s = enqueue(X, W, y, N, H, V, ignore_index, &ctrl->loss, &ctrl->status, dX, dW, workspace, stream);
+  if (s != FLCE_OK) return s;
+  Ctrl host{};
+  if (cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  *loss = host.loss;
+  return static_cast<flce_status_t>(host.status);
+}
+
+flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N,
+                                          int64_t H, int64_t V, int32_t ignore_index, float* d_loss,
+                                          int32_t* d_status, uint16_t* dX, uint16_t* dW, void* workspace,
+                                          size_t workspace_bytes, cudaStream_t stream) {
+  if (!d_loss || !d_status) return FLCE_ERR_INVALID_ARGUMENT;
+  const flce_status_t s = check_args(X, W, y, N, H, V, dX, dW, workspace);
+  if (s != FLCE_OK) return s;
+  if (!aligned(d_status, 4) || !aligned(d_loss, 4)) return FLCE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, stream);
+}
+
+flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_W, const int32_t* h_y, int64_t N,
+                                         int64_t H, int64_t V, int32_t ignore_index, float* h_loss, uint16_t* h_dX,
+                                         uint16_t* h_dW, uint16_t* d_X, uint16_t* d_W, int32_t* d_y,
+                                         uint16_t* d_dX, uint16_t* d_dW, void* workspace, size_t workspace_bytes,
+                                         cudaStream_t stream) {
+  if (!h_X || !h_W || !h_y || !h_loss || !h_dX || !h_dW) return FLCE_ERR_INVALID_ARGUMENT;
+  flce_status_t s = check_args(d_X, d_W, d_y, N, H, V, d_dX, d_dW, workspace);
+  if (s != FLCE_OK) return s;
+  const WsLayout L = ws_layout(N, H);
+  if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  const size_t xb = static_cast<size_t>(N) * H * 2, wb = static_cast<size_t>(V) * H * 2, yb = N * 4;
+  if (cudaMemcpyAsync(d_X, h_X, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(d_W, h_W, wb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(d_y, h_y, yb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(static_cast<uint8_t*>(workspace) + L.ctrl);
+  s = enqueue(d_X, d_W, d_y, N, H, V, ignore_index, &ctrl->loss, &ctrl->status, d_dX, d_dW, workspace, stream);
+  if (s != FLCE_OK) return s;
+  Ctrl host{};
+  if (cudaMemcpyAsync(h_dX, d_dX, xb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaMemcpyAsync(h_dW, d_dW, wb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  *h_loss = host.loss;
+  return static_cast<flce_status_t>(host.status);
+}
+
+flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out) {
+  if (!out) return FLCE_ERR_INVALID_ARGUMENT;
+  const flce_status_t s = check_sizes(N, H, V);
+  if (s != FLCE_OK) return s;
+  int sms = 148;
+  DevInfo di;
+  int dev;
+  if (device_info(&di, &dev) == cudaSuccess && di.num_sms > 0) sms = di.num_sms;
+  const Plan P = make_plan(N, H, V, sms);
+  out->workspace_bytes = static_cast<int64_t>(ws_layout(N, H).total);
+  out->vocab_chunk = VC;
+  out->num_chunks = P.num_chunks;
+  out->lse_splits = P.splits;
+  out->launches = P.launches;
+  out->num_sms = sms;
+  return FLCE_OK;
+}
+
+const char* flce_kernel_name(int kind) {
+  switch (kind) {
+    case KIND_LSE: return "pass1_logits_lse";
+    case KIND_COMBINE: return "combine_lse_loss";
+    case KIND_GRAD: return "pass2_logits_grad";
+    case KIND_DW: return "dW_contraction";
+    case KIND_DX: return "dX_contraction";
+    default: return "unknown";
+  }
+}
+
+flce_status_t flce_profile_enable(int on) {
+  if (on && g_prof.ev.empty()) {
+    g_prof.ev.resize(2 * PROF_PAIRS);
+    g_prof.kind.resize(PROF_PAIRS);
+    for (auto& e : g_prof.ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  g_prof.on = on != 0;
+  g_prof.used = 0;
+  return FLCE_OK;
+}
+
+flce_status_t flce_profile_read(int32_t* launches, double* total_ms) {
+  if (!launches || !total_ms) return FLCE_ERR_INVALID_ARGUMENT;
+  for (int k = 0; k < FLCE_NUM_KERNEL_KINDS; ++k) {
+    launches[k] = 0;
+    total_ms[k] = 0.0;
+  }
+  for (size_t i = 0; i < g_prof.used; ++i) {
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return FLCE_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) return FLCE_ERR_CUDA;
+    launches[g_prof.kind[i]] += 1;
+    total_ms[g_prof.kind[i]] += ms;
+  }
+  g_prof.used = 0;
+  return FLCE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,585 @@
+// Device code of the fused linear + cross-entropy head.
+//
+// One persistent, warp-specialised tcgen05 GEMM template serves all four
+// tensor-core steps; they differ in which operands the TMA engine streams in,
+// in which of them are MN-major, and in the epilogue that turns the fp32
+// accumulator tile in tensor memory into the step's output:
+//
+//   KIND_LSE  (pass 1)  z = X W^T per [128 tokens x 256 vocab] tile; the
+//                       epilogue keeps an online row max and sum of
+//                       exponentials over the tiles of one vocabulary split and
+//                       picks out the target logit.  No logit leaves the chip.
+//   KIND_GRAD (pass 2)  recomputes the logits of one vocabulary chunk and writes
+//                       G = (softmax - onehot) / n in bf16 into the chunk buffer.
+//   KIND_DW             dW[chunk rows] = G_c^T X       (K = tokens)
+//   KIND_DX             dX += G_c W_c                  (K = chunk vocabulary)
+//
+// These follow the pages' description of the fused head: the loss and its
+// gradient are computed chunk by chunk over the vocabulary, the logits are
+// recomputed rather than stored ("Liger Kernel explained", cross-entropy head
+// section), and the (batch, sequence, vocab) tensor is never allocated
+// ("Liger-Kernel: Triton kernels that replace HF training ops", section "What
+// actually gets replaced").
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 issues UMMAs and
+// owns the tensor-memory allocation, warps 2..5 run the epilogue (warp w reads
+// TMEM lanes 32*(w%4) .. 32*(w%4)+31, one accumulator row per thread).
+#pragma once
+
+#include <cfloat>
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace flce {
+
+constexpr int BM = 128;        // accumulator rows (TMEM lanes)
+constexpr int BN = 256;        // accumulator columns
+constexpr int BK = 64;         // K per pipeline stage: one 128-B swizzle row of bf16
+constexpr int UMMA_K = 16;     // K per tcgen05.mma kind::f16
+constexpr int STAGES = 4;
+constexpr int A_TILE_BYTES = BM * BK * 2;
+constexpr int B_TILE_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
+constexpr int MN_BOX_BYTES = 64 * BK * 2;  // one 64(MN) x 64(K) MN-major box
+constexpr int NUM_THREADS = 192;
+constexpr int ACC_COLS = BN;
+constexpr int TMEM_COLS = 2 * ACC_COLS;    // double-buffered accumulator
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr double LN2 = 0.6931471805599453;
+
+enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_GRAD = 2, KIND_DW = 3, KIND_DX = 4 };
+enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
+
+struct GemmArgs {
+  int N, H, V, ignore_index;
+  int tiles_m, tiles_n;   // tile grid of the launch
+  int k_blocks;           // BK-wide steps along K
+  int num_units;          // LSE: tiles_m * splits; otherwise tiles_m * tiles_n
+  int splits;             // LSE: vocabulary splits
+  int vbase, vcount;      // first vocabulary entry and entry count of this chunk
+  int Vc;                 // chunk width = row stride of the G buffer
+  int first_chunk, last_chunk;
+  const int32_t* y;
+  float* part_m;          // [splits][N] running max, log2 units
+  float* part_l;          // [splits][N] running sum of 2^(s - m)
+  float* zy;              // [N] target logit
+  const float* lse2;      // [N] log2-sum-exp2 of z*log2(e)
+  const float* inv_n;     // 1 / n_valid (0 when n_valid = 0)
+  uint16_t* G;            // [N][Vc] bf16
+  uint16_t* dW;           // [V][H] bf16
+  uint16_t* dX;           // [N][H] bf16, also the high half of the dX accumulator
+  uint16_t* lo;           // [N][H] bf16, low half of the dX accumulator
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+template <int KIND> struct KindTraits;
+template <> struct KindTraits<KIND_LSE>  { static constexpr bool A_MN = false, B_MN = false; };
+template <> struct KindTraits<KIND_GRAD> { static constexpr bool A_MN = false, B_MN = false; };
+template <> struct KindTraits<KIND_DW>   { static constexpr bool A_MN = true,  B_MN = true;  };
+template <> struct KindTraits<KIND_DX>   { static constexpr bool A_MN = false, B_MN = true;  };
+
+__device__ __forceinline__ void raise_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// Work unit u -> token/vocab tile row mb and the range [nb_begin, nb_end) of
+// tile columns it walks.  Pass 1 walks one vocabulary split per unit, with
+// units ordered split-major so that CTAs running at the same time share the
+// same W tiles through L2; the other kinds have one tile per unit.
+template <int KIND>
+__device__ __forceinline__ void unit_range(const GemmArgs& a, int u, int& mb, int& nb_begin, int& nb_end,
+                                           int& split) {
+  if constexpr (KIND == KIND_LSE) {
+    split = u / a.tiles_m;
+    mb = u - split * a.tiles_m;
+    nb_begin = static_cast<int>((static_cast<long long>(split) * a.tiles_n) / a.splits);
+    nb_end = static_cast<int>((static_cast<long long>(split + 1) * a.tiles_n) / a.splits);
+  } else {
+    split = 0;
+    nb_begin = u / a.tiles_m;
+    mb = u - nb_begin * a.tiles_m;
+    nb_end = nb_begin + 1;
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ void load_stage(const GemmArgs& a, const CUtensorMap* mA, const CUtensorMap* mB,
+                                           uint32_t sA, uint32_t sB, uint32_t bar, int mb, int nb, int kb) {
+  const int k0 = kb * BK;
+  if constexpr (KIND == KIND_LSE || KIND == KIND_GRAD) {
+    tma_load_2d(sA, mA, bar, k0, mb * BM);               // X rows, K-major
+    tma_load_2d(sB, mB, bar, k0, a.vbase + nb * BN);     // W rows, K-major
+  } else if constexpr (KIND == KIND_DW) {
+#pragma unroll
+    for (int i = 0; i < BM / 64; ++i)                    // G_c^T: vocab contiguous
+      tma_load_2d(sA + i * MN_BOX_BYTES, mA, bar, mb * BM + i * 64, k0);
+#pragma unroll
+    for (int i = 0; i < BN / 64; ++i)                    // X: hidden contiguous
+      tma_load_2d(sB + i * MN_BOX_BYTES, mB, bar, nb * BN + i * 64, k0);
+  } else {
+    tma_load_2d(sA, mA, bar, k0, mb * BM);               // G_c rows, K-major
+#pragma unroll
+    for (int i = 0; i < BN / 64; ++i)                    // W_c: hidden contiguous
+      tma_load_2d(sB + i * MN_BOX_BYTES, mB, bar, nb * BN + i * 64, a.vbase + k0);
+  }
+}
+
+template <bool MN>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
+  if constexpr (MN)
+    return sdesc_sw128(base + k * (UMMA_K * 128), MN_BOX_BYTES, 1024);
+  else
+    return sdesc_sw128(base + k * (UMMA_K * 2), 16, 1024);
+}
+
+// ------------------------------------------------------------- epilogues --
+
+struct LseState {
+  float run_m, run_l, zy_val;
+  int yr, row;
+  bool has_zy;
+};
+
+// Pass 1: fold one [128 x 256] logit tile into the running (max, sum) of the row.
+__device__ __forceinline__ void epi_lse_tile(const GemmArgs& a, uint32_t taddr, int nb, LseState& st) {
+  const int col_base = nb * BN;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_ld_wait();
+    const int col0 = col_base + c * 32;
+    const int lim = a.V - col0;
+    const int off = st.yr - col0;
+    if (static_cast<unsigned>(off) < 32u) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t)
+        if (t == off) st.zy_val = __uint_as_float(r[t]);
+      st.has_zy = true;
+    }
+    float s[32];
+    float cmax = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      s[t] = (t < lim) ? __uint_as_float(r[t]) * LOG2E : -INFINITY;
+      cmax = fmaxf(cmax, s[t]);
+    }
+    const float new_m = fmaxf(st.run_m, cmax);
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+    for (int t = 0; t < 32; t += 4) {
+      acc0 += ex2_approx(s[t + 0] - new_m);
+      acc1 += ex2_approx(s[t + 1] - new_m);
+      acc2 += ex2_approx(s[t + 2] - new_m);
+      acc3 += ex2_approx(s[t + 3] - new_m);
+    }
+    st.run_l = st.run_l * ex2_approx(st.run_m - new_m) + ((acc0 + acc1) + (acc2 + acc3));
+    st.run_m = new_m;
+  }
+}
+
+// Pass 2: G = valid * (softmax - onehot) / n for one tile, stored as bf16.
+__device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr, int mb, int nb,
+                                              int row_local) {
+  const int row = mb * BM + row_local;
+  const bool in_rows = row < a.N;
+  const int yr = in_rows ? a.y[row] : a.ignore_index;
+  const bool valid = in_rows && yr != a.ignore_index;
+  const float l2 = valid ? a.lse2[row] : 0.f;
+  const float scale = valid ? *a.inv_n : 0.f;
+  uint16_t* grow = a.G + static_cast<size_t>(in_rows ? row : 0) * a.Vc + nb * BN;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_ld_wait();
+    const int colg0 = a.vbase + nb * BN + c * 32;
+    const int lim = a.V - colg0;
+    float g[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t)
+      g[t] = (valid && t < lim) ? ex2_approx(fmaf(__uint_as_float(r[t]), LOG2E, -l2)) * scale : 0.f;
+    const int off = yr - colg0;
+    if (valid && static_cast<unsigned>(off) < 32u) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t)
+        if (t == off) g[t] -= scale;
+    }
+    if (in_rows) {
+      uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 v;
+        v.x = pack_bf16x2(g[8 * q + 0], g[8 * q + 1]);
+        v.y = pack_bf16x2(g[8 * q + 2], g[8 * q + 3]);
+        v.z = pack_bf16x2(g[8 * q + 4], g[8 * q + 5]);
+        v.w = pack_bf16x2(g[8 * q + 6], g[8 * q + 7]);
+        dst[q] = v;
+      }
+    }
+  }
+}
+
+// dW rows of this chunk: the K = tokens contraction is complete, round to bf16.
+__device__ __forceinline__ void epi_dw_tile(const GemmArgs& a, uint32_t taddr, int mb, int nb, int row_local) {
+  const int vrow_local = mb * BM + row_local;
+  const bool in_rows = vrow_local < a.vcount;
+  uint16_t* drow = a.dW + static_cast<size_t>(a.vbase + (in_rows ? vrow_local : 0)) * a.H;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_ld_wait();
+    const int col0 = nb * BN + c * 32;
+    if (in_rows) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (col0 + 8 * q < a.H) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+          v.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+          v.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+          v.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+          *reinterpret_cast<uint4*>(drow + col0 + 8 * q) = v;
+        }
+      }
+    }
+  }
+}
+
+// dX += G_c W_c.  The running sum lives in two bf16 words, hi (in dX itself) and
+// lo (workspace), with value = hi + lo: about 16 significant bits, enough for an
+// fp32-grade sum over the chunks, at the memory cost of one bf16 copy of dX.
+__device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, int mb, int nb, int row_local) {
+  const int row = mb * BM + row_local;
+  const bool in_rows = row < a.N;
+  const size_t rbase = static_cast<size_t>(in_rows ? row : 0) * a.H;
+  uint16_t* hrow = a.dX + rbase;
+  uint16_t* lrow = a.lo + rbase;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_ld_wait();
+    const int col0 = nb * BN + c * 32;
+    if (in_rows) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col = col0 + 8 * q;
+        if (col < a.H) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]);
+          if (!a.first_chunk) {
+            const uint4 h = *reinterpret_cast<const uint4*>(hrow + col);
+            const uint4 l = *reinterpret_cast<const uint4*>(lrow + col);
+            const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+            const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              v[2 * e] += bf16lo_to_f32(hw[e]) + bf16lo_to_f32(lw[e]);
+              v[2 * e + 1] += bf16hi_to_f32(hw[e]) + bf16hi_to_f32(lw[e]);
+            }
+          }
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            hw[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+            lw[e] = pack_bf16x2(v[2 * e] - bf16lo_to_f32(hw[e]), v[2 * e + 1] - bf16hi_to_f32(hw[e]));
+          }
+          *reinterpret_cast<uint4*>(hrow + col) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          if (!a.last_chunk)
+            *reinterpret_cast<uint4*>(lrow + col) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------ the kernel --
+
+template <int KIND>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    flce_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                     const GemmArgs a) {
+  using T = KindTraits<KIND>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;  // swizzle atoms need 1024-B alignment
+  uint8_t* base_ptr = smem_raw + (base - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + STAGES * STAGE_BYTES);
+  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 + b); };
+  const uint32_t done_bar = smem_u32(bars + 2 * STAGES + 4);
+  auto sA = [&](int s) { return base + s * STAGE_BYTES; };
+  auto sB = [&](int s) { return base + s * STAGE_BYTES + A_TILE_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&mapA);
+    prefetch_tmap(&mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    raise_status(a.status, ST_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < a.num_units; u += gridDim.x) {
+        int mb, nb0, nb1, split;
+        unit_range<KIND>(a, u, mb, nb0, nb1, split);
+        for (int nb = nb0; ok && nb < nb1; ++nb) {
+          for (int kb = 0; kb < a.k_blocks; ++kb) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
+              give_up();
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+            load_stage<KIND>(a, &mapA, &mapB, sA(stage), sB(stage), full_bar(stage), mb, nb, kb);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      if (!ok) {  // let copies already in flight land before the CTA can exit
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 100000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- UMMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, T::A_MN, T::B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < a.num_units; u += gridDim.x) {
+        int mb, nb0, nb1, split;
+        unit_range<KIND>(a, u, mb, nb0, nb1, split);
+        for (int nb = nb0; ok && nb < nb1; ++nb) {
+          if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+          for (int kb = 0; kb < a.k_blocks; ++kb) {
+            if (!mbar_wait(full_bar(stage), phase, abort_flag, a.timeout_ns)) {
+              give_up();
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k)
+              umma_bf16(d_tmem, operand_desc<T::A_MN>(sA(stage), k), operand_desc<T::B_MN>(sB(stage), k), IDESC,
+                        (kb | k) != 0);
+            umma_commit(empty_bar(stage));
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit(tfull_bar(acc));
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
+        }
+      }
+      // Every UMMA issued above has finished once this commit lands.
+      umma_commit(done_bar);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(done_bar, 0) && globaltimer_ns() - t0 < 50000000ull) {
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue --
+    const int q = warp & 3;
+    const int row_local = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < a.num_units; u += gridDim.x) {
+      int mb, nb0, nb1, split;
+      unit_range<KIND>(a, u, mb, nb0, nb1, split);
+      LseState st;
+      if constexpr (KIND == KIND_LSE) {
+        st.row = mb * BM + row_local;
+        st.yr = st.row < a.N ? a.y[st.row] : a.ignore_index;
+        st.run_m = -1e30f;
+        st.run_l = 0.f;
+        st.zy_val = 0.f;
+        st.has_zy = false;
+      }
+      for (int nb = nb0; nb < nb1; ++nb) {
+        const bool got = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.timeout_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+          give_up();
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
+        if constexpr (KIND == KIND_LSE) epi_lse_tile(a, taddr, nb, st);
+        if constexpr (KIND == KIND_GRAD) epi_grad_tile(a, taddr, mb, nb, row_local);
+        if constexpr (KIND == KIND_DW) epi_dw_tile(a, taddr, mb, nb, row_local);
+        if constexpr (KIND == KIND_DX) epi_dx_tile(a, taddr, mb, nb, row_local);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if constexpr (KIND == KIND_LSE) {
+        if (ok && st.row < a.N) {
+          a.part_m[static_cast<size_t>(split) * a.N + st.row] = st.run_m;
+          a.part_l[static_cast<size_t>(split) * a.N + st.row] = st.run_l;
+          if (st.has_zy) a.zy[st.row] = st.zy_val;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------ combine --
+
+struct CombineArgs {
+  int N, V, ignore_index, splits;
+  const int32_t* y;
+  const float* part_m;
+  const float* part_l;
+  const float* zy;
+  float* lse2;
+  double* blk_loss;
+  int* blk_cnt;
+  unsigned int* ticket;
+  int* n_valid;
+  float* inv_n;
+  float* loss;
+  int* status;
+};
+
+constexpr int COMBINE_THREADS = 256;
+
+// Merges the per-split (max, sum) pairs of each row into its log-sum-exp, forms
+// the row loss lse_i - z_{i,y_i} for valid rows and reduces the token mean.
+// Deterministic: a fixed tree inside each block, then the last block to finish
+// adds the block sums in block order, in fp64.
+__global__ void __launch_bounds__(COMBINE_THREADS) flce_combine_kernel(const CombineArgs a) {
+  const int i = blockIdx.x * COMBINE_THREADS + threadIdx.x;
+  double li = 0.0;
+  int vi = 0;
+  if (i < a.N) {
+    float M = -INFINITY;
+    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_m[static_cast<size_t>(s) * a.N + i]);
+    float L = 0.f;
+    for (int s = 0; s < a.splits; ++s)
+      L += a.part_l[static_cast<size_t>(s) * a.N + i] * exp2f(a.part_m[static_cast<size_t>(s) * a.N + i] - M);
+    const float l2 = M + log2f(L);
+    a.lse2[i] = l2;
+    const int yi = a.y[i];
+    if (yi != a.ignore_index) {
+      if (yi < 0 || yi >= a.V) {
+        raise_status(a.status, ST_TARGET_OUT_OF_RANGE);
+      } else {
+        li = static_cast<double>(l2) * LN2 - static_cast<double>(a.zy[i]);
+        vi = 1;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    li += __shfl_down_sync(0xffffffffu, li, o);
+    vi += __shfl_down_sync(0xffffffffu, vi, o);
+  }
+  __shared__ double wl[COMBINE_THREADS / 32];
+  __shared__ int wc[COMBINE_THREADS / 32];
+  __shared__ bool is_last;
+  if ((threadIdx.x & 31) == 0) {
+    wl[threadIdx.x >> 5] = li;
+    wc[threadIdx.x >> 5] = vi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double sl = 0.0;
+    int sc = 0;
+    for (int w = 0; w < COMBINE_THREADS / 32; ++w) {
+      sl += wl[w];
+      sc += wc[w];
+    }
+    a.blk_loss[blockIdx.x] = sl;
+    a.blk_cnt[blockIdx.x] = sc;
+    __threadfence();
+    is_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (is_last && threadIdx.x == 0) {
+    __threadfence();
+    const volatile double* bl = a.blk_loss;
+    const volatile int* bc = a.blk_cnt;
+    double tot = 0.0;
+    long long cnt = 0;
+    for (unsigned b = 0; b < gridDim.x; ++b) {
+      tot += bl[b];
+      cnt += bc[b];
+    }
+    *a.n_valid = static_cast<int>(cnt);
+    *a.inv_n = cnt ? static_cast<float>(1.0 / static_cast<double>(cnt)) : 0.f;
+    *a.loss = cnt ? static_cast<float>(tot / static_cast<double>(cnt)) : 0.f;
+    *a.ticket = 0u;
+  }
+}
+
+}  // namespace flce

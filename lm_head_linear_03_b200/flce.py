@@ -1,0 +1,212 @@
+"""ctypes binding of the FLCE C ABI (include/flce.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library ``_lib/libflce.so``.  PyTorch supplies device memory and streams.  If the
+library is missing, or the device is not sm_100, calls raise; there is no CPU
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libflce.so")
+
+FLCE_OK = 0
+STATUS_NAMES = {
+    0: "FLCE_OK",
+    1: "FLCE_ERR_INVALID_ARGUMENT",
+    2: "FLCE_ERR_UNSUPPORTED",
+    3: "FLCE_ERR_WORKSPACE_TOO_SMALL",
+    4: "FLCE_ERR_TARGET_OUT_OF_RANGE",
+    5: "FLCE_ERR_TIMEOUT",
+    6: "FLCE_ERR_CUDA",
+}
+NUM_KERNEL_KINDS = 5
+
+EXPORTED = (
+    "flce_status_string",
+    "flce_workspace_size",
+    "flce_forward_backward",
+    "flce_forward_backward_async",
+    "flce_forward_backward_host",
+    "flce_plan",
+    "flce_kernel_name",
+    "flce_profile_enable",
+    "flce_profile_read",
+)
+
+
+class FlceError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class PlanT(ctypes.Structure):
+    _fields_ = [
+        ("workspace_bytes", ctypes.c_int64),
+        ("vocab_chunk", ctypes.c_int32),
+        ("num_chunks", ctypes.c_int32),
+        ("lse_splits", ctypes.c_int32),
+        ("launches", ctypes.c_int32),
+        ("num_sms", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libflce.so (built by ``__graft_entry__.build()``) and declares the ABI."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"FLCE CUDA library not built: {path} is missing (run __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
+    i64, i32, vp, sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+    fp = ctypes.POINTER(ctypes.c_float)
+    lib.flce_status_string.argtypes = [ctypes.c_int]
+    lib.flce_status_string.restype = ctypes.c_char_p
+    lib.flce_workspace_size.argtypes = [i64, i64, i64]
+    lib.flce_workspace_size.restype = sz
+    lib.flce_forward_backward.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp, vp, vp]
+    lib.flce_forward_backward.restype = ctypes.c_int
+    lib.flce_forward_backward_async.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.flce_forward_backward_async.restype = ctypes.c_int
+    lib.flce_forward_backward_host.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp,
+                                               vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.flce_forward_backward_host.restype = ctypes.c_int
+    lib.flce_plan.argtypes = [i64, i64, i64, ctypes.POINTER(PlanT)]
+    lib.flce_plan.restype = ctypes.c_int
+    lib.flce_kernel_name.argtypes = [ctypes.c_int]
+    lib.flce_kernel_name.restype = ctypes.c_char_p
+    lib.flce_profile_enable.argtypes = [ctypes.c_int]
+    lib.flce_profile_enable.restype = ctypes.c_int
+    lib.flce_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)]
+    lib.flce_profile_read.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != FLCE_OK:
+        raise FlceError(status, where)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check_inputs(X, W, y):
+    if not (X.is_cuda and W.is_cuda and y.is_cuda):
+        raise ValueError("X, W and y must be CUDA tensors")
+    if X.dtype != torch.bfloat16 or W.dtype != torch.bfloat16 or y.dtype != torch.int32:
+        raise ValueError("expected X, W bf16 and y int32")
+    if X.dim() != 2 or W.dim() != 2 or y.dim() != 1:
+        raise ValueError("expected X[N,H], W[V,H], y[N]")
+    if X.shape[1] != W.shape[1] or y.shape[0] != X.shape[0]:
+        raise ValueError(f"shape mismatch: X{tuple(X.shape)} W{tuple(W.shape)} y{tuple(y.shape)}")
+    if not (X.is_contiguous() and W.is_contiguous() and y.is_contiguous()):
+        raise ValueError("X, W and y must be contiguous")
+
+
+def workspace_size(N: int, H: int, V: int) -> int:
+    return int(load_library().flce_workspace_size(N, H, V))
+
+
+def plan(N: int, H: int, V: int) -> PlanT:
+    p = PlanT()
+    _check(load_library().flce_plan(N, H, V, ctypes.byref(p)), "flce_plan")
+    return p
+
+
+def alloc_workspace(N: int, H: int, V: int, device=None) -> torch.Tensor:
+    """A uint8 device buffer of flce_workspace_size bytes (torch's allocator
+    hands out 512-B aligned blocks)."""
+    return torch.empty(workspace_size(N, H, V), dtype=torch.uint8, device=device or "cuda")
+
+
+def forward_backward(X, W, y, ignore_index: int = -100, *, dX=None, dW=None, workspace=None, stream=None):
+    """Synchronous call: returns (loss: float, dX, dW).  Raises FlceError on any
+    host- or device-detected error."""
+    lib = load_library()
+    _check_inputs(X, W, y)
+    N, H = X.shape
+    V = W.shape[0]
+    dX = torch.empty_like(X) if dX is None else dX
+    dW = torch.empty_like(W) if dW is None else dW
+    workspace = alloc_workspace(N, H, V, X.device) if workspace is None else workspace
+    loss = ctypes.c_float(0.0)
+    st = lib.flce_forward_backward(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, ctypes.byref(loss),
+                                   _ptr(dX), _ptr(dW), _ptr(workspace), _stream_handle(stream))
+    _check(st, "flce_forward_backward")
+    return loss.value, dX, dW
+
+
+def forward_backward_async(X, W, y, ignore_index: int = -100, *, out=None, workspace=None, stream=None):
+    """Enqueues the call and returns device tensors (loss[1] f32, status[1] i32, dX, dW)
+    without waiting.  ``out`` may pass preallocated (loss, status, dX, dW)."""
+    lib = load_library()
+    _check_inputs(X, W, y)
+    N, H = X.shape
+    V = W.shape[0]
+    if out is None:
+        out = (torch.empty(1, dtype=torch.float32, device=X.device),
+               torch.empty(1, dtype=torch.int32, device=X.device),
+               torch.empty_like(X), torch.empty_like(W))
+    loss, status, dX, dW = out
+    workspace = alloc_workspace(N, H, V, X.device) if workspace is None else workspace
+    st = lib.flce_forward_backward_async(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, _ptr(loss),
+                                         _ptr(status), _ptr(dX), _ptr(dW), _ptr(workspace),
+                                         workspace.numel(), _stream_handle(stream))
+    _check(st, "flce_forward_backward_async")
+    return loss, status, dX, dW
+
+
+def forward_backward_host(hX, hW, hy, dev_bufs, ignore_index: int = -100, *, h_out=None, stream=None):
+    """End-to-end call on host tensors: copies in, computes, copies loss, dX and
+    dW back.  ``dev_bufs`` = (d_X, d_W, d_y, d_dX, d_dW, workspace) on the device;
+    ``h_out`` = optional host (dX, dW) outputs (pinned for full bandwidth)."""
+    lib = load_library()
+    N, H = hX.shape
+    V = hW.shape[0]
+    d_X, d_W, d_y, d_dX, d_dW, ws = dev_bufs
+    if h_out is None:
+        h_out = (torch.empty_like(hX), torch.empty_like(hW))
+    h_dX, h_dW = h_out
+    loss = ctypes.c_float(0.0)
+    st = lib.flce_forward_backward_host(_ptr(hX), _ptr(hW), _ptr(hy), N, H, V, ignore_index, ctypes.byref(loss),
+                                        _ptr(h_dX), _ptr(h_dW), _ptr(d_X), _ptr(d_W), _ptr(d_y), _ptr(d_dX),
+                                        _ptr(d_dW), _ptr(ws), ws.numel(), _stream_handle(stream))
+    _check(st, "flce_forward_backward_host")
+    return loss.value, h_dX, h_dW
+
+
+def kernel_names():
+    lib = load_library()
+    return [lib.flce_kernel_name(k).decode() for k in range(NUM_KERNEL_KINDS)]
+
+
+def profile_enable(on: bool = True):
+    _check(load_library().flce_profile_enable(1 if on else 0), "flce_profile_enable")
+
+
+def profile_read():
+    """{kernel name: (launches, total ms)} since the last read."""
+    lib = load_library()
+    n = (ctypes.c_int32 * NUM_KERNEL_KINDS)()
+    ms = (ctypes.c_double * NUM_KERNEL_KINDS)()
+    _check(lib.flce_profile_read(n, ms), "flce_profile_read")
+    names = kernel_names()
+    return {names[k]: (int(n[k]), float(ms[k])) for k in range(NUM_KERNEL_KINDS)}

@@ -1,0 +1,212 @@
+"""CUDA path against the fp64 oracle, element by element, through the C ABI.
+
+Tolerances are the ones the target states: loss relative error <= 1e-4; dX and
+dW relative Frobenius error <= 1e-2 and max-abs error <= 2^-7 * max|grad|.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_linear_03_b200.inputs import WORKLOADS, custom, make_inputs
+from oracle import flce_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-4
+FRO_RTOL = 1e-2
+MAXABS_FRAC = 2.0 ** -7
+
+
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import lm_head_linear_03_b200 as F
+    F.load_library()
+    return F
+
+
+def _np(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def assert_grad_close(got, ref, what):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    nref = np.linalg.norm(ref)
+    if nref == 0.0:
+        assert np.all(got == 0.0), f"{what}: expected exact zeros"
+        return
+    fro = np.linalg.norm(got - ref) / nref
+    mx = np.max(np.abs(got - ref))
+    lim = MAXABS_FRAC * np.max(np.abs(ref))
+    assert fro <= FRO_RTOL, f"{what}: relative Frobenius error {fro:.3e}"
+    assert mx <= lim, f"{what}: max-abs error {mx:.3e} > {lim:.3e}"
+
+
+def assert_loss_close(got, ref, what="loss"):
+    if ref == 0.0:
+        assert got == 0.0, f"{what}: {got} != 0"
+        return
+    assert abs(got - ref) <= LOSS_RTOL * abs(ref), f"{what}: {got} vs {ref}"
+
+
+def run_full_oracle_case(X, W, y, ignore_index=-100):
+    F = _lib()
+    loss, dX, dW = F.forward_backward(X.cuda(), W.cuda(), y.cuda(), ignore_index)
+    rl, rdX, rdW, _, _ = O.flce_reference(X, W, y, ignore_index)
+    assert_loss_close(loss, rl)
+    assert_grad_close(_np(dX), rdX, "dX")
+    assert_grad_close(_np(dW), rdW, "dW")
+    return loss, dX, dW
+
+
+# Sizes the oracle finishes in seconds that still span several 128 x 256 tiles,
+# several 2048-wide vocabulary chunks and ragged tails in N, H and V.
+SMALL = [
+    WORKLOADS["tiny"],
+    custom("ragged_all_dims", N=300, H=136, V=5000, ignore_frac=0.1),
+    custom("multi_chunk_tail64", N=520, H=264, V=6208, ignore_frac=0.05),   # V mod 256 = 64
+    custom("single_token", N=1, H=64, V=300),
+    custom("h_min", N=130, H=8, V=700, ignore_frac=0.2),
+    custom("tiny_vocab", N=200, H=128, V=2, ignore_frac=0.1),
+    custom("vocab_below_tile", N=129, H=96, V=100),
+    custom("all_valid_zipf", N=384, H=512, V=9000, targets="zipf"),
+    custom("prompt_mask", N=640, H=256, V=3000, ignore_prefix=200),
+    custom("long_k", N=256, H=4096, V=1024, ignore_frac=0.1),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_small_against_full_oracle(w):
+    X, W, y = make_inputs(w)
+    run_full_oracle_case(X, W, y)
+
+
+def test_all_rows_ignored_gives_zero():
+    w = custom("all_ignored", N=200, H=64, V=1000)
+    X, W, y = make_inputs(w)
+    y[:] = -100
+    loss, dX, dW = run_full_oracle_case(X, W, y)
+    assert loss == 0.0
+    assert torch.count_nonzero(dX).item() == 0 and torch.count_nonzero(dW).item() == 0
+
+
+def test_zero_weight_gives_log_v():
+    w = custom("w_zero", N=257, H=64, V=5000, ignore_frac=0.1)
+    X, W, y = make_inputs(w)
+    W.zero_()
+    loss, dX, _ = run_full_oracle_case(X, W, y)
+    assert abs(loss - math.log(5000)) <= 1e-6 * math.log(5000)
+    assert torch.count_nonzero(dX).item() == 0
+
+
+def test_large_logit_range():
+    """|z| up to ~80: the online max shift must keep every exponential finite."""
+    w = custom("large_logits", N=256, H=256, V=3000, ignore_frac=0.1, x_std=4.0, w_std=0.3)
+    X, W, y = make_inputs(w)
+    z = X.float() @ W.float().T
+    assert z.abs().max().item() > 60
+    run_full_oracle_case(X, W, y)
+
+
+def test_target_zero_everywhere():
+    w = custom("all_target_zero", N=300, H=128, V=2500)
+    X, W, y = make_inputs(w)
+    y[:] = 0
+    run_full_oracle_case(X, W, y)
+
+
+def test_other_ignore_index():
+    w = custom("ignore_minus_one", N=256, H=128, V=1500)
+    X, W, y = make_inputs(w)
+    y[::7] = -1
+    run_full_oracle_case(X, W, y, ignore_index=-1)
+
+
+def test_repeat_calls_identical():
+    """Same inputs, same workspace: bit-identical results (no atomics in the sums)."""
+    F = _lib()
+    X, W, y = (t.cuda() for t in make_inputs(custom("det", N=384, H=256, V=4500, ignore_frac=0.1)))
+    ws = F.alloc_workspace(384, 256, 4500)
+    l1, dX1, dW1 = F.forward_backward(X, W, y, workspace=ws)
+    l2, dX2, dW2 = F.forward_backward(X, W, y, workspace=ws)
+    assert l1 == l2 and torch.equal(dX1, dX2) and torch.equal(dW1, dW2)
+
+
+def test_async_matches_sync():
+    F = _lib()
+    X, W, y = (t.cuda() for t in make_inputs(WORKLOADS["tiny"]))
+    l1, dX1, dW1 = F.forward_backward(X, W, y)
+    loss, status, dX2, dW2 = F.forward_backward_async(X, W, y)
+    torch.cuda.synchronize()
+    assert status.item() == 0 and loss.item() == l1
+    assert torch.equal(dX1, dX2) and torch.equal(dW1, dW2)
+
+
+def test_host_entry_matches_device_entry():
+    F = _lib()
+    w = custom("host", N=300, H=136, V=5000, ignore_frac=0.1)
+    X, W, y = make_inputs(w)
+    l1, dX1, dW1 = F.forward_backward(X.cuda(), W.cuda(), y.cuda())
+    hX, hW, hy = X.pin_memory(), W.pin_memory(), y.pin_memory()
+    dev = (torch.empty_like(X, device="cuda"), torch.empty_like(W, device="cuda"),
+           torch.empty_like(y, device="cuda"), torch.empty_like(X, device="cuda"),
+           torch.empty_like(W, device="cuda"), F.alloc_workspace(w.N, w.H, w.V))
+    l2, hdX, hdW = F.forward_backward_host(hX, hW, hy, dev)
+    assert l1 == l2 and torch.equal(dX1.cpu(), hdX) and torch.equal(dW1.cpu(), hdW)
+
+
+def test_target_out_of_range_reported():
+    F = _lib()
+    X, W, y = make_inputs(custom("oor", N=256, H=64, V=1000))
+    y[17] = 1000
+    with pytest.raises(F.FlceError) as e:
+        F.forward_backward(X.cuda(), W.cuda(), y.cuda())
+    assert e.value.status == 4
+    y[17] = -5
+    with pytest.raises(F.FlceError) as e:
+        F.forward_backward(X.cuda(), W.cuda(), y.cuda())
+    assert e.value.status == 4
+    # the device stays usable
+    y[17] = 3
+    run_full_oracle_case(X, W, y)
+
+
+def test_host_argument_errors():
+    F = _lib()
+    X = torch.zeros(64, 12, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(100, 12, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(64, dtype=torch.int32, device="cuda")
+    with pytest.raises(F.FlceError) as e:  # H % 8 != 0
+        F.forward_backward(X, W, y)
+    assert e.value.status == 2
+    X = torch.zeros(64, 16, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(100, 16, dtype=torch.bfloat16, device="cuda")
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(F.FlceError) as e:
+        F.forward_backward_async(X, W, y, workspace=small)
+    assert e.value.status == 3
+
+
+def test_workspace_independent_of_vocab():
+    F = _lib()
+    sizes = {F.workspace_size(8192, 4096, V) for V in (1, 1000, 32064, 128256, 256000, 10 ** 6)}
+    assert len(sizes) == 1
+    assert F.workspace_size(8192, 4096, 128256) <= 0.05 * 8192 * 128256 * 2
+
+
+def test_peak_device_bytes_equal_buffers_plus_workspace():
+    """No hidden allocation: the call's peak is inputs + outputs + workspace."""
+    F = _lib()
+    w = custom("peak", N=1024, H=512, V=20000, ignore_frac=0.1)
+    X, W, y = (t.cuda() for t in make_inputs(w))
+    dX, dW = torch.empty_like(X), torch.empty_like(W)
+    ws = F.alloc_workspace(w.N, w.H, w.V)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    F.forward_backward(X, W, y, dX=dX, dW=dW, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.cuda.max_memory_allocated() == base
