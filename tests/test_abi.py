@@ -1,0 +1,86 @@
+"""The C ABI without a GPU: the library loads, exports every function the header
+declares, and answers the host-only queries (no kernel is launched here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(flce_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    from lm_head_linear_03_b200 import flce
+    return flce.load_library()
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for must in ("flce_forward_backward", "flce_workspace_size", "flce_forward_backward_async"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_binding_covers_the_header():
+    from lm_head_linear_03_b200 import flce
+    assert set(declared_functions()) <= set(flce.EXPORTED)
+
+
+def test_status_strings(lib):
+    lib.flce_status_string.restype = ctypes.c_char_p
+    assert lib.flce_status_string(0) == b"FLCE_OK"
+    assert lib.flce_status_string(4) == b"FLCE_ERR_TARGET_OUT_OF_RANGE"
+    assert lib.flce_status_string(99) == b"FLCE_UNKNOWN_STATUS"
+
+
+def test_workspace_size_independent_of_vocab(lib):
+    from lm_head_linear_03_b200 import flce
+    sizes = {flce.workspace_size(8192, 4096, v) for v in (1, 2, 4096, 32064, 128256, 256000, 1 << 24)}
+    assert len(sizes) == 1
+    # the Llama-3-8B head workload stays within 5% of its N x V x 2-byte logits
+    assert flce.workspace_size(8192, 4096, 128256) <= 0.05 * 8192 * 128256 * 2
+    assert flce.workspace_size(0, 4096, 10) == 0
+    assert flce.workspace_size(16, 12, 10) == 0  # H % 8 != 0
+
+
+def test_plan_is_host_only(lib):
+    from lm_head_linear_03_b200 import flce
+    p = flce.plan(8192, 4096, 128256)
+    assert p.vocab_chunk == 2048 and p.num_chunks == 63
+    assert 1 <= p.lse_splits <= 64
+    assert p.launches == 2 + 3 * p.num_chunks
+
+
+def test_argument_errors_before_any_launch(lib):
+    """NULL pointers and bad sizes are rejected on the host, so these calls are
+    safe without a device."""
+    i64 = ctypes.c_int64
+    f = ctypes.c_float(0)
+    assert lib.flce_forward_backward(None, None, None, i64(8), i64(8), i64(8), -100, ctypes.byref(f),
+                                     None, None, None, None) == 1
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.flce_forward_backward(fake, fake, fake, i64(8), i64(12), i64(8), -100, ctypes.byref(f),
+                                     fake, fake, fake, None) == 2  # H % 8
+    assert lib.flce_forward_backward(fake, fake, fake, i64(0), i64(8), i64(8), -100, ctypes.byref(f),
+                                     fake, fake, fake, None) == 1
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.flce_forward_backward(odd, fake, fake, i64(8), i64(8), i64(8), -100, ctypes.byref(f),
+                                     fake, fake, fake, None) == 2  # misaligned X
