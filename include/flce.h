@@ -116,6 +116,33 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
                                          void* workspace, size_t workspace_bytes,
                                          cudaStream_t stream);
 
+/* Allocation-free variant of flce_forward_backward, for callers that cannot
+ * allocate device memory: a plug-in or custom operator that is handed only the
+ * tensors it works on and has no allocator to ask for scratch, and processes
+ * where a framework's memory pool has already reserved nearly all of the GPU,
+ * so that a raw cudaMalloc from a library would fail.  The published
+ * fused-head method has no counterpart of this entry: it exists only for such
+ * callers.
+ *
+ * Arguments are those of flce_forward_backward minus the workspace (X, W, y,
+ * dX, dW on the device; loss on the host; synchronous).  Scratch comes from a
+ * fixed array of FLCE_NOALLOC_SCRATCH_BYTES in the library's device module,
+ * held on every GPU that loads the library until the process exits.  Sizes
+ * whose flce_workspace_size exceeds it are rejected with
+ * FLCE_ERR_WORKSPACE_TOO_SMALL before anything runs.
+ *
+ * The first call on a device looks the array's device address up (a
+ * cudaGetSymbolAddress, no allocation); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents; each call clears the words that must start at zero.  Calls that
+ * overlap on the GPU (several streams or host threads at once) race on the
+ * array and must be serialised by the caller. */
+#define FLCE_NOALLOC_SCRATCH_BYTES (16u << 20)
+flce_status_t flce_forward_backward_noalloc(const uint16_t* X, const uint16_t* W, const int32_t* y,
+                                            int64_t N, int64_t H, int64_t V, int32_t ignore_index,
+                                            float* loss, uint16_t* dX, uint16_t* dW,
+                                            cudaStream_t stream);
+
 /* How a call of these sizes is split into launches (host-only query). */
 typedef struct {
   int64_t workspace_bytes; /* same as flce_workspace_size */

@@ -513,3 +513,44 @@ flce_status_t flce_profile_read(int32_t* launches, double* total_ms) {
 }
 
 }  // extern "C"
+
+// ============================================================ no-alloc entry ==
+// Scratch of flce_forward_backward_noalloc.  It is part of the library's device
+// module, so a caller of that entry never needs an allocation.  In host code
+// the name stands for a host-side shadow; the device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FLCE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64];
+
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+extern "C" flce_status_t flce_forward_backward_noalloc(const uint16_t* X, const uint16_t* W, const int32_t* y,
+                                                       int64_t N, int64_t H, int64_t V, int32_t ignore_index,
+                                                       float* loss, uint16_t* dX, uint16_t* dW,
+                                                       cudaStream_t stream) {
+  if (!loss) return FLCE_ERR_INVALID_ARGUMENT;
+  const flce_status_t s = check_sizes(N, H, V);
+  if (s != FLCE_OK) return s;
+  if (ws_layout(N, H).total > static_cast<size_t>(FLCE_NOALLOC_SCRATCH_BYTES)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return FLCE_ERR_CUDA;
+  return flce_forward_backward(X, W, y, N, H, V, ignore_index, loss, dX, dW, scratch, stream);
+}

@@ -37,7 +37,9 @@ EXPORTED = (
     "flce_kernel_name",
     "flce_profile_enable",
     "flce_profile_read",
+    "flce_forward_backward_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class FlceError(RuntimeError):
@@ -89,6 +91,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_profile_enable.restype = ctypes.c_int
     lib.flce_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)]
     lib.flce_profile_read.restype = ctypes.c_int
+    lib.flce_forward_backward_noalloc.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp, vp]
+    lib.flce_forward_backward_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -210,3 +214,21 @@ def profile_read():
     _check(lib.flce_profile_read(n, ms), "flce_profile_read")
     names = kernel_names()
     return {names[k]: (int(n[k]), float(ms[k])) for k in range(NUM_KERNEL_KINDS)}
+
+
+def forward_backward_noalloc(X, W, y, ignore_index: int = -100, *, dX=None, dW=None, stream=None):
+    """Like :func:`forward_backward` but with no workspace: the library uses its
+    fixed device scratch array (NOALLOC_SCRATCH_BYTES), for callers that cannot
+    allocate device memory.  Larger problems raise FLCE_ERR_WORKSPACE_TOO_SMALL;
+    overlapping calls race on the shared array."""
+    lib = load_library()
+    _check_inputs(X, W, y)
+    N, H = X.shape
+    V = W.shape[0]
+    dX = torch.empty_like(X) if dX is None else dX
+    dW = torch.empty_like(W) if dW is None else dW
+    loss = ctypes.c_float(0.0)
+    st = lib.flce_forward_backward_noalloc(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index,
+                                           ctypes.byref(loss), _ptr(dX), _ptr(dW), _stream_handle(stream))
+    _check(st, "flce_forward_backward_noalloc")
+    return loss.value, dX, dW
