@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--shape", default=None,
+                    help="N,H,V: a smaller slice of the workload (uniform targets), for profiling")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -222,13 +224,20 @@ def cpu_baseline(w, rows: int):
                       f"W[{w.V},{w.H}] (loss, dX rows, full dW update); {dt:.2f} s"}
 
 
+def workload(args):
+    from lm_head_linear_03_b200.inputs import WORKLOADS, custom
+    if args.shape:
+        N, H, V = (int(v) for v in args.shape.split(","))
+        return custom(f"slice_{N}x{H}x{V}", N=N, H=H, V=V)
+    return WORKLOADS[args.workload]
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: each step is a bounded sample of the
     workload, timed on the host cores; rank 0 only."""
-    from lm_head_linear_03_b200.inputs import WORKLOADS
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     rows = 32
     for _ in range(args.warmup):
         oracle_sample(w, rows)
@@ -251,9 +260,9 @@ def run_reference(args, world, rank):
 # -------------------------------------------------------------------- ours --
 def run_ours(args, world, rank, local):
     import lm_head_linear_03_b200 as F
-    from lm_head_linear_03_b200.inputs import WORKLOADS, make_inputs
+    from lm_head_linear_03_b200.inputs import make_inputs
     F.load_library()
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     dev = torch.device("cuda", local)
     X, W, y = make_inputs(w, dev)
     N, H, V = w.N, w.H, w.V
@@ -361,7 +370,7 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": w.name, "N": N, "H": H, "V": V, "ignored_rows": w.n_ignored,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (W is 1.05 GB vs 126 MB L2); no flush"},
+                   "l2": f"inputs larger than L2 (W is {V * H * 2 / 1e9:.2f} GB vs 126 MB L2); no flush"},
         "tflops": tflops,
         "pct_of_measured_bf16_peak": 100.0 * tflops / pk["bf16_tflops"],
         "pct_of_measured_bf16_sustained": 100.0 * tflops / sustained,

@@ -131,13 +131,14 @@ bool get_encode() {
 // 2-D bf16 row-major tensor [outer][inner], 128-B swizzled boxes of
 // box_inner x box_outer elements; out-of-range elements read as zero.
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer, bool swizzle = true) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -236,10 +237,10 @@ flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N,
 // --------------------------------------------------------------- enqueue --
 template <int KIND>
 cudaError_t launch_gemm(int grid, cudaStream_t s, const CUtensorMap& mA, const CUtensorMap& mB,
-                        const GemmArgs& a, int kind) {
+                        const CUtensorMap& mHi, const CUtensorMap& mLo, const GemmArgs& a, int kind) {
   size_t slot;
   prof_begin(s, kind, &slot);
-  flce_gemm_kernel<KIND><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, a);
+  flce_gemm_kernel<KIND><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mHi, mLo, a);
   prof_end(s, slot);
   return cudaGetLastError();
 }
@@ -265,11 +266,12 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   uint16_t* G = reinterpret_cast<uint16_t*>(ws + L.G);
   uint16_t* lo = reinterpret_cast<uint16_t*>(ws + L.lo);
 
-  CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn;
+  CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn, mHi, mLo;
   const uint64_t n = static_cast<uint64_t>(N), h = static_cast<uint64_t>(H), v = static_cast<uint64_t>(V);
   bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BN) &&
             make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
-            make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK);
+            make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK) &&
+            make_map(&mHi, dX, h, n, h * 2, BN, BM, false) && make_map(&mLo, lo, h, n, h * 2, BN, BM, false);
   if (!ok) return FLCE_ERR_CUDA;
 
   if (cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), stream) != cudaSuccess) return FLCE_ERR_CUDA;
@@ -305,7 +307,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     p1.num_units = P.tiles_m * P.splits;
     p1.vbase = 0;
     p1.vcount = static_cast<int>(V);
-    if (launch_gemm<KIND_LSE>(P.lse_grid, stream, mX_k, mW_k, p1, KIND_LSE) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (launch_gemm<KIND_LSE>(P.lse_grid, stream, mX_k, mW_k, mHi, mLo, p1, KIND_LSE) != cudaSuccess) return FLCE_ERR_CUDA;
   }
   // Combine the splits: lse, loss, n_valid, 1/n.
   {
@@ -349,7 +351,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       g.k_blocks = static_cast<int>((H + BK - 1) / BK);
       g.num_units = g.tiles_m * g.tiles_n;
       const int grid = std::min(g.num_units, di.num_sms);
-      if (launch_gemm<KIND_GRAD>(grid, stream, mX_k, mW_k, g, KIND_GRAD) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (launch_gemm<KIND_GRAD>(grid, stream, mX_k, mW_k, mHi, mLo, g, KIND_GRAD) != cudaSuccess) return FLCE_ERR_CUDA;
     }
     {  // dW rows of the chunk
       GemmArgs d = b;
@@ -358,7 +360,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       d.k_blocks = static_cast<int>((N + BK - 1) / BK);
       d.num_units = d.tiles_m * d.tiles_n;
       const int grid = std::min(d.num_units, di.num_sms);
-      if (launch_gemm<KIND_DW>(grid, stream, mG_mn, mX_mn, d, KIND_DW) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (launch_gemm<KIND_DW>(grid, stream, mG_mn, mX_mn, mHi, mLo, d, KIND_DW) != cudaSuccess) return FLCE_ERR_CUDA;
     }
     {  // dX accumulation
       GemmArgs d = b;
@@ -367,7 +369,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       d.k_blocks = (vcount + BK - 1) / BK;
       d.num_units = d.tiles_m * d.tiles_n;
       const int grid = std::min(d.num_units, di.num_sms);
-      if (launch_gemm<KIND_DX>(grid, stream, mG_k, mW_mn, d, KIND_DX) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (launch_gemm<KIND_DX>(grid, stream, mG_k, mW_mn, mHi, mLo, d, KIND_DX) != cudaSuccess) return FLCE_ERR_CUDA;
     }
   }
   return FLCE_OK;

@@ -253,18 +253,39 @@ __device__ __forceinline__ void epi_dw_tile(const GemmArgs& a, uint32_t taddr, i
 // dX += G_c W_c.  The running sum lives in two bf16 words, hi (in dX itself) and
 // lo (workspace), with value = hi + lo: about 16 significant bits, enough for an
 // fp32-grade sum over the chunks, at the memory cost of one bf16 copy of dX.
+// The hi/lo words of the next 32 columns are loaded while the current ones are
+// combined and stored, so two chunks of reads are in flight per thread.
+__device__ __forceinline__ void dx_load_hl(const uint16_t* hrow, const uint16_t* lrow, int col0, int H, uint4 (&h)[4],
+                                           uint4 (&l)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + 8 * q < H) {
+      h[q] = *reinterpret_cast<const uint4*>(hrow + col0 + 8 * q);
+      l[q] = *reinterpret_cast<const uint4*>(lrow + col0 + 8 * q);
+    } else {
+      h[q] = make_uint4(0, 0, 0, 0);
+      l[q] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
 __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, int mb, int nb, int row_local) {
   const int row = mb * BM + row_local;
   const bool in_rows = row < a.N;
+  const bool accumulate = !a.first_chunk;
   const size_t rbase = static_cast<size_t>(in_rows ? row : 0) * a.H;
   uint16_t* hrow = a.dX + rbase;
   uint16_t* lrow = a.lo + rbase;
+  uint4 hc[4], lc[4];
+  if (in_rows && accumulate) dx_load_hl(hrow, lrow, nb * BN, a.H, hc, lc);
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
     const int col0 = nb * BN + c * 32;
+    uint4 hn[4], ln[4];
+    if (in_rows && accumulate && c + 1 < BN / 32) dx_load_hl(hrow, lrow, col0 + 32, a.H, hn, ln);
     if (in_rows) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -273,11 +294,9 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, i
           float v[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]);
-          if (!a.first_chunk) {
-            const uint4 h = *reinterpret_cast<const uint4*>(hrow + col);
-            const uint4 l = *reinterpret_cast<const uint4*>(lrow + col);
-            const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
-            const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
+          if (accumulate) {
+            const uint32_t hw[4] = {hc[q].x, hc[q].y, hc[q].z, hc[q].w};
+            const uint32_t lw[4] = {lc[q].x, lc[q].y, lc[q].z, lc[q].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               v[2 * e] += bf16lo_to_f32(hw[e]) + bf16lo_to_f32(lw[e]);
@@ -296,6 +315,11 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, i
         }
       }
     }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      hc[q] = hn[q];
+      lc[q] = ln[q];
+    }
   }
 }
 
@@ -304,6 +328,7 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, i
 template <int KIND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     flce_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                     const __grid_constant__ CUtensorMap mapHi, const __grid_constant__ CUtensorMap mapLo,
                      const GemmArgs a) {
   using T = KindTraits<KIND>;
   extern __shared__ uint8_t smem_raw[];
@@ -366,6 +391,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int mb, nb0, nb1, split;
         unit_range<KIND>(a, u, mb, nb0, nb1, split);
         for (int nb = nb0; ok && nb < nb1; ++nb) {
+          if constexpr (KIND == KIND_DX) {
+            // the epilogue of this tile reads back the running dX sum: pull it
+            // into L2 now, a whole mainloop ahead of the read
+            if (!a.first_chunk) {
+              tma_prefetch_l2_2d(&mapHi, nb * BN, mb * BM);
+              tma_prefetch_l2_2d(&mapLo, nb * BN, mb * BM);
+            }
+          }
           for (int kb = 0; kb < a.k_blocks; ++kb) {
             if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
               give_up();
