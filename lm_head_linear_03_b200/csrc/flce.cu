@@ -67,6 +67,7 @@ struct DevInfo {
   bool ok = false;
   bool sm100 = false;
   int num_sms = 0;
+  int max_clusters = 0;  // SM pairs that can run a GEMM kernel at the same time
 };
 
 std::mutex g_mu;
@@ -109,6 +110,22 @@ cudaError_t set_kernel_attrs(int dev) {
   if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_DX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SMEM_BYTES)) != cudaSuccess)
     return e;
+  // How many SM pairs the GEMM kernels can occupy at once (persistent grids).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 1024, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = CLUSTER;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters, flce_gemm_kernel<KIND_LSE>, &cfg)) != cudaSuccess) return e;
+  if (clusters <= 0) return cudaErrorInvalidConfiguration;
+  g_dev[dev].max_clusters = clusters;
   g_attr_set[dev] = true;
   return cudaSuccess;
 }
@@ -145,17 +162,17 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
 
 // ------------------------------------------------------------------ plan --
 struct Plan {
-  int tiles_m;        // 128-token tiles
+  int tiles_m;        // 256-token tiles (one per SM pair)
   int vtiles;         // 256-wide vocabulary tiles
   int splits;         // pass-1 vocabulary splits
-  int lse_grid;
+  int lse_clusters;   // SM pairs of the pass-1 launch
   int num_chunks;
   int launches;
-  int num_sms;
+  int clusters;       // SM pairs available
 };
 
 // Pass 1: pick the number of vocabulary splits whose units, dealt round-robin
-// to one persistent CTA per SM, give the smallest largest per-CTA tile count.
+// to the persistent SM pairs, give the smallest largest per-pair tile count.
 int choose_splits(int tiles_m, int vtiles, int sms) {
   int best = 1;
   long long best_cost = LLONG_MAX;
@@ -179,14 +196,15 @@ int choose_splits(int tiles_m, int vtiles, int sms) {
   return best;
 }
 
-Plan make_plan(int64_t N, int64_t H, int64_t V, int sms) {
+Plan make_plan(int64_t N, int64_t H, int64_t V, int clusters) {
   (void)H;
   Plan p{};
-  p.num_sms = sms;
-  p.tiles_m = static_cast<int>((N + BM - 1) / BM);
+  p.clusters = clusters;
+  p.tiles_m = static_cast<int>((N + CM - 1) / CM);
   p.vtiles = static_cast<int>((V + BN - 1) / BN);
-  p.splits = choose_splits(p.tiles_m, p.vtiles, sms);
-  p.lse_grid = static_cast<int>(std::min<long long>(static_cast<long long>(p.tiles_m) * p.splits, sms));
+  p.splits = choose_splits(p.tiles_m, p.vtiles, clusters);
+  p.lse_clusters =
+      static_cast<int>(std::min<long long>(static_cast<long long>(p.tiles_m) * p.splits, clusters));
   p.num_chunks = static_cast<int>((V + VC - 1) / VC);
   p.launches = 2 + 3 * p.num_chunks;
   return p;
@@ -235,12 +253,13 @@ flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N,
 }
 
 // --------------------------------------------------------------- enqueue --
+// `grid` counts SM pairs (clusters of two CTAs).
 template <int KIND>
 cudaError_t launch_gemm(int grid, cudaStream_t s, const CUtensorMap& mA, const CUtensorMap& mB,
                         const CUtensorMap& mHi, const CUtensorMap& mLo, const GemmArgs& a, int kind) {
   size_t slot;
   prof_begin(s, kind, &slot);
-  flce_gemm_kernel<KIND><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mHi, mLo, a);
+  flce_gemm_kernel<KIND><<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mHi, mLo, a);
   prof_end(s, slot);
   return cudaGetLastError();
 }
@@ -255,8 +274,9 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   if (set_kernel_attrs(dev) != cudaSuccess) return FLCE_ERR_CUDA;
   if (!get_encode()) return FLCE_ERR_CUDA;
 
+  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;  // now with max_clusters
   const WsLayout L = ws_layout(N, H);
-  const Plan P = make_plan(N, H, V, di.num_sms);
+  const Plan P = make_plan(N, H, V, di.max_clusters);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
   float* lse2 = reinterpret_cast<float*>(ws + L.lse2);
@@ -268,7 +288,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
 
   CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn, mHi, mLo;
   const uint64_t n = static_cast<uint64_t>(N), h = static_cast<uint64_t>(H), v = static_cast<uint64_t>(V);
-  bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BN) &&
+  bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BNH) &&
             make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
             make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK) &&
             make_map(&mHi, dX, h, n, h * 2, BN, BM, false) && make_map(&mLo, lo, h, n, h * 2, BN, BM, false);
@@ -307,7 +327,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     p1.num_units = P.tiles_m * P.splits;
     p1.vbase = 0;
     p1.vcount = static_cast<int>(V);
-    if (launch_gemm<KIND_LSE>(P.lse_grid, stream, mX_k, mW_k, mHi, mLo, p1, KIND_LSE) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (launch_gemm<KIND_LSE>(P.lse_clusters, stream, mX_k, mW_k, mHi, mLo, p1, KIND_LSE) != cudaSuccess) return FLCE_ERR_CUDA;
   }
   // Combine the splits: lse, loss, n_valid, 1/n.
   {
@@ -350,16 +370,16 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       g.tiles_n = (vcount + BN - 1) / BN;
       g.k_blocks = static_cast<int>((H + BK - 1) / BK);
       g.num_units = g.tiles_m * g.tiles_n;
-      const int grid = std::min(g.num_units, di.num_sms);
+      const int grid = std::min(g.num_units, P.clusters);
       if (launch_gemm<KIND_GRAD>(grid, stream, mX_k, mW_k, mHi, mLo, g, KIND_GRAD) != cudaSuccess) return FLCE_ERR_CUDA;
     }
     {  // dW rows of the chunk
       GemmArgs d = b;
-      d.tiles_m = (vcount + BM - 1) / BM;
+      d.tiles_m = (vcount + CM - 1) / CM;
       d.tiles_n = static_cast<int>((H + BN - 1) / BN);
       d.k_blocks = static_cast<int>((N + BK - 1) / BK);
       d.num_units = d.tiles_m * d.tiles_n;
-      const int grid = std::min(d.num_units, di.num_sms);
+      const int grid = std::min(d.num_units, P.clusters);
       if (launch_gemm<KIND_DW>(grid, stream, mG_mn, mX_mn, mHi, mLo, d, KIND_DW) != cudaSuccess) return FLCE_ERR_CUDA;
     }
     {  // dX accumulation
@@ -368,7 +388,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       d.tiles_n = static_cast<int>((H + BN - 1) / BN);
       d.k_blocks = (vcount + BK - 1) / BK;
       d.num_units = d.tiles_m * d.tiles_n;
-      const int grid = std::min(d.num_units, di.num_sms);
+      const int grid = std::min(d.num_units, P.clusters);
       if (launch_gemm<KIND_DX>(grid, stream, mG_k, mW_mn, mHi, mLo, d, KIND_DX) != cudaSuccess) return FLCE_ERR_CUDA;
     }
   }
@@ -460,11 +480,17 @@ flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out) {
   if (!out) return FLCE_ERR_INVALID_ARGUMENT;
   const flce_status_t s = check_sizes(N, H, V);
   if (s != FLCE_OK) return s;
-  int sms = 148;
+  int sms = 148, clusters = 74;
   DevInfo di;
   int dev;
-  if (device_info(&di, &dev) == cudaSuccess && di.num_sms > 0) sms = di.num_sms;
-  const Plan P = make_plan(N, H, V, sms);
+  if (device_info(&di, &dev) == cudaSuccess && di.num_sms > 0) {
+    sms = di.num_sms;
+    if (di.sm100 && set_kernel_attrs(dev) == cudaSuccess && device_info(&di, &dev) == cudaSuccess)
+      clusters = di.max_clusters;
+    else
+      clusters = sms / CLUSTER;
+  }
+  const Plan P = make_plan(N, H, V, clusters);
   out->workspace_bytes = static_cast<int64_t>(ws_layout(N, H).total);
   out->vocab_chunk = VC;
   out->num_chunks = P.num_chunks;

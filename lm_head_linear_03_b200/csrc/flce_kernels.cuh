@@ -21,9 +21,16 @@
 // ("Liger-Kernel: Triton kernels that replace HF training ops", section "What
 // actually gets replaced").
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 issues UMMAs and
-// owns the tensor-memory allocation, warps 2..5 run the epilogue (warp w reads
-// TMEM lanes 32*(w%4) .. 32*(w%4)+31, one accumulator row per thread).
+// The CTAs run in pairs (clusters of two on neighbouring SMs).  A pair owns one
+// 256 x 256 accumulator tile: each CTA loads 128 rows of A and 128 columns of B
+// into its own shared memory, the leader CTA issues cta_group::2 UMMAs that read
+// both halves, and each CTA's tensor memory receives its 128 rows.  Per SM this
+// halves the B-operand traffic of a 128 x 256 single-CTA tile.
+//
+// Warp roles (192 threads per CTA): warp 0 issues TMA loads, warp 1 issues UMMAs
+// (leader CTA only) and owns the tensor-memory allocation, warps 2..5 run the
+// epilogue (warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31, one accumulator row
+// per thread).
 #pragma once
 
 #include <cfloat>
@@ -33,18 +40,23 @@
 
 namespace flce {
 
-constexpr int BM = 128;        // accumulator rows (TMEM lanes)
-constexpr int BN = 256;        // accumulator columns
+constexpr int CLUSTER = 2;     // SM pair: the two CTAs of a cluster share one UMMA tile
+constexpr int BM = 128;        // accumulator rows per CTA (TMEM lanes)
+constexpr int CM = CLUSTER * BM;  // rows of the pair's tile (UMMA M = 256)
+constexpr int BN = 256;        // accumulator columns (UMMA N)
+constexpr int BNH = BN / CLUSTER; // B columns each CTA of the pair holds
 constexpr int BK = 64;         // K per pipeline stage: one 128-B swizzle row of bf16
 constexpr int UMMA_K = 16;     // K per tcgen05.mma kind::f16
-constexpr int STAGES = 4;
+constexpr int STAGES = 6;
 constexpr int A_TILE_BYTES = BM * BK * 2;
-constexpr int B_TILE_BYTES = BN * BK * 2;
+constexpr int B_TILE_BYTES = BNH * BK * 2;
 constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
 constexpr int MN_BOX_BYTES = 64 * BK * 2;  // one 64(MN) x 64(K) MN-major box
 constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 4;
 constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;    // double-buffered accumulator
+constexpr int NUM_BARRIERS = 2 * STAGES + 4 + 1;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr double LN2 = 0.6931471805599453;
@@ -105,25 +117,31 @@ __device__ __forceinline__ void unit_range(const GemmArgs& a, int u, int& mb, in
   }
 }
 
+// TMA loads of one pipeline stage for the CTA of rank `rank` in the pair: its
+// 128 rows of A and its 128 columns of B.  Completion is counted on the
+// leader's full barrier `bar`.
 template <int KIND>
 __device__ __forceinline__ void load_stage(const GemmArgs& a, const CUtensorMap* mA, const CUtensorMap* mB,
-                                           uint32_t sA, uint32_t sB, uint32_t bar, int mb, int nb, int kb) {
+                                           uint32_t sA, uint32_t sB, uint32_t bar, int mb, int nb, int kb,
+                                           int rank) {
   const int k0 = kb * BK;
+  const int m0 = mb * CM + rank * BM;
+  const int n0 = nb * BN + rank * BNH;
   if constexpr (KIND == KIND_LSE || KIND == KIND_GRAD) {
-    tma_load_2d(sA, mA, bar, k0, mb * BM);               // X rows, K-major
-    tma_load_2d(sB, mB, bar, k0, a.vbase + nb * BN);     // W rows, K-major
+    tma_load_2d_pair(sA, mA, bar, k0, m0);               // X rows, K-major
+    tma_load_2d_pair(sB, mB, bar, k0, a.vbase + n0);     // W rows, K-major
   } else if constexpr (KIND == KIND_DW) {
 #pragma unroll
     for (int i = 0; i < BM / 64; ++i)                    // G_c^T: vocab contiguous
-      tma_load_2d(sA + i * MN_BOX_BYTES, mA, bar, mb * BM + i * 64, k0);
+      tma_load_2d_pair(sA + i * MN_BOX_BYTES, mA, bar, m0 + i * 64, k0);
 #pragma unroll
-    for (int i = 0; i < BN / 64; ++i)                    // X: hidden contiguous
-      tma_load_2d(sB + i * MN_BOX_BYTES, mB, bar, nb * BN + i * 64, k0);
+    for (int i = 0; i < BNH / 64; ++i)                   // X: hidden contiguous
+      tma_load_2d_pair(sB + i * MN_BOX_BYTES, mB, bar, n0 + i * 64, k0);
   } else {
-    tma_load_2d(sA, mA, bar, k0, mb * BM);               // G_c rows, K-major
+    tma_load_2d_pair(sA, mA, bar, k0, m0);               // G_c rows, K-major
 #pragma unroll
-    for (int i = 0; i < BN / 64; ++i)                    // W_c: hidden contiguous
-      tma_load_2d(sB + i * MN_BOX_BYTES, mB, bar, nb * BN + i * 64, a.vbase + k0);
+    for (int i = 0; i < BNH / 64; ++i)                   // W_c: hidden contiguous
+      tma_load_2d_pair(sB + i * MN_BOX_BYTES, mB, bar, n0 + i * 64, a.vbase + k0);
   }
 }
 
@@ -182,9 +200,9 @@ __device__ __forceinline__ void epi_lse_tile(const GemmArgs& a, uint32_t taddr, 
 }
 
 // Pass 2: G = valid * (softmax - onehot) / n for one tile, stored as bf16.
-__device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr, int mb, int nb,
+__device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb,
                                               int row_local) {
-  const int row = mb * BM + row_local;
+  const int row = row0 + row_local;
   const bool in_rows = row < a.N;
   const int yr = in_rows ? a.y[row] : a.ignore_index;
   const bool valid = in_rows && yr != a.ignore_index;
@@ -224,8 +242,8 @@ __device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr,
 }
 
 // dW rows of this chunk: the K = tokens contraction is complete, round to bf16.
-__device__ __forceinline__ void epi_dw_tile(const GemmArgs& a, uint32_t taddr, int mb, int nb, int row_local) {
-  const int vrow_local = mb * BM + row_local;
+__device__ __forceinline__ void epi_dw_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local) {
+  const int vrow_local = row0 + row_local;
   const bool in_rows = vrow_local < a.vcount;
   uint16_t* drow = a.dW + static_cast<size_t>(a.vbase + (in_rows ? vrow_local : 0)) * a.H;
 #pragma unroll 1
@@ -269,8 +287,8 @@ __device__ __forceinline__ void dx_load_hl(const uint16_t* hrow, const uint16_t*
   }
 }
 
-__device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, int mb, int nb, int row_local) {
-  const int row = mb * BM + row_local;
+__device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local) {
+  const int row = row0 + row_local;
   const bool in_rows = row < a.N;
   const bool accumulate = !a.first_chunk;
   const size_t rbase = static_cast<size_t>(in_rows ? row : 0) * a.H;
@@ -326,40 +344,45 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, i
 // ------------------------------------------------------------ the kernel --
 
 template <int KIND>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     flce_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                      const __grid_constant__ CUtensorMap mapHi, const __grid_constant__ CUtensorMap mapLo,
                      const GemmArgs a) {
   using T = KindTraits<KIND>;
   extern __shared__ uint8_t smem_raw[];
+  // Same dynamic-smem base in both CTAs, so every offset below matches across the pair.
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;  // swizzle atoms need 1024-B alignment
   uint8_t* base_ptr = smem_raw + (base - raw_addr);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + STAGES * STAGE_BYTES);
-  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x / CLUSTER;
+  const int ncl = gridDim.x / CLUSTER;
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
   auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 + b); };
-  const uint32_t done_bar = smem_u32(bars + 2 * STAGES + 4);
+  const uint32_t fin_bar = smem_u32(bars + 2 * STAGES + 4);
   auto sA = [&](int s) { return base + s * STAGE_BYTES; };
   auto sB = [&](int s) { return base + s * STAGE_BYTES + A_TILE_BYTES; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(full_bar(s), 1);    // leader: its producer's arrive + both CTAs' bytes
+      mbar_init(empty_bar(s), 1);   // the leader's UMMA commit, multicast to both
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 4);
+      mbar_init(tfull_bar(b), 1);                 // UMMA commit, multicast to both
+      mbar_init(tempty_bar(b), CLUSTER * EPI_WARPS);  // leader: epilogue warps of both CTAs
     }
-    mbar_init(done_bar, 1);
+    mbar_init(fin_bar, 1);  // the peer's end-of-work signal
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -368,11 +391,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tmap(&mapB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -387,16 +410,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < a.num_units; u += gridDim.x) {
+      for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
         unit_range<KIND>(a, u, mb, nb0, nb1, split);
         for (int nb = nb0; ok && nb < nb1; ++nb) {
           if constexpr (KIND == KIND_DX) {
-            // the epilogue of this tile reads back the running dX sum: pull it
-            // into L2 now, a whole mainloop ahead of the read
+            // the epilogue of this tile reads back the running dX sum: pull this
+            // CTA's rows into L2 now, a whole mainloop ahead of the read
             if (!a.first_chunk) {
-              tma_prefetch_l2_2d(&mapHi, nb * BN, mb * BM);
-              tma_prefetch_l2_2d(&mapLo, nb * BN, mb * BM);
+              tma_prefetch_l2_2d(&mapHi, nb * BN, mb * CM + rank * BM);
+              tma_prefetch_l2_2d(&mapLo, nb * BN, mb * CM + rank * BM);
             }
           }
           for (int kb = 0; kb < a.k_blocks; ++kb) {
@@ -405,8 +428,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
-            load_stage<KIND>(a, &mapA, &mapB, sA(stage), sB(stage), full_bar(stage), mb, nb, kb);
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * STAGE_BYTES);
+            load_stage<KIND>(a, &mapA, &mapB, sA(stage), sB(stage), mapa_shared(full_bar(stage), 0), mb, nb,
+                             kb, rank);
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -414,26 +438,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!ok) {  // let copies already in flight land before the CTA can exit
+      // Tail: wait for the UMMA commits still headed for this CTA's empty
+      // barriers, so none lands after the CTA has gone.
+      for (int i = 0; i < STAGES; ++i) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          break;
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (*abort_flag) {  // let copies already in flight land before the CTA can exit
         const uint64_t t0 = globaltimer_ns();
         while (globaltimer_ns() - t0 < 100000ull) {
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------- UMMA issuer --
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, T::A_MN, T::B_MN);
+    // ------------------------------------------------ UMMA issuer (leader) --
+    if (leader && lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(CM, BN, T::A_MN, T::B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < a.num_units; u += gridDim.x) {
+      for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
         unit_range<KIND>(a, u, mb, nb0, nb1, split);
         for (int nb = nb0; ok && nb < nb1; ++nb) {
-          if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+          if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
             give_up();
             ok = false;
             break;
@@ -449,24 +485,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k)
-              umma_bf16(d_tmem, operand_desc<T::A_MN>(sA(stage), k), operand_desc<T::B_MN>(sB(stage), k), IDESC,
-                        (kb | k) != 0);
-            umma_commit(empty_bar(stage));
+              umma_bf16_pair(d_tmem, operand_desc<T::A_MN>(sA(stage), k), operand_desc<T::B_MN>(sB(stage), k),
+                             IDESC, (kb | k) != 0);
+            umma_commit_pair(empty_bar(stage), 0x3);
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
             }
           }
           if (!ok) break;
-          umma_commit(tfull_bar(acc));
+          umma_commit_pair(tfull_bar(acc), 0x3);
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1u;
         }
       }
-      // Every UMMA issued above has finished once this commit lands.
-      umma_commit(done_bar);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(done_bar, 0) && globaltimer_ns() - t0 < 50000000ull) {
+      // Tail: both accumulators released by the epilogues of both CTAs, so all
+      // UMMAs are done and no remote arrive is still on its way here.
+      for (int i = 0; i < 2; ++i) {
+        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          break;
+        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
       }
     }
   } else {
@@ -474,15 +515,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;
     const int row_local = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
+    const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < a.num_units; u += gridDim.x) {
+    for (int u = cid; ok && u < a.num_units; u += ncl) {
       int mb, nb0, nb1, split;
       unit_range<KIND>(a, u, mb, nb0, nb1, split);
+      const int row0 = mb * CM + rank * BM;
       LseState st;
       if constexpr (KIND == KIND_LSE) {
-        st.row = mb * BM + row_local;
+        st.row = row0 + row_local;
         st.yr = st.row < a.N ? a.y[st.row] : a.ignore_index;
         st.run_m = -1e30f;
         st.run_l = 0.f;
@@ -499,12 +543,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
         if constexpr (KIND == KIND_LSE) epi_lse_tile(a, taddr, nb, st);
-        if constexpr (KIND == KIND_GRAD) epi_grad_tile(a, taddr, mb, nb, row_local);
-        if constexpr (KIND == KIND_DW) epi_dw_tile(a, taddr, mb, nb, row_local);
-        if constexpr (KIND == KIND_DX) epi_dx_tile(a, taddr, mb, nb, row_local);
+        if constexpr (KIND == KIND_GRAD) epi_grad_tile(a, taddr, row0, nb, row_local);
+        if constexpr (KIND == KIND_DW) epi_dw_tile(a, taddr, row0, nb, row_local);
+        if constexpr (KIND == KIND_DX) epi_dx_tile(a, taddr, row0, nb, row_local);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
@@ -518,11 +562,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  // Wind-down: this CTA's work is done; tell the peer, wait (bounded) for the
+  // peer to say the same, then free the pair's tensor memory together.
   tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_cluster(mapa_shared(fin_bar, static_cast<uint32_t>(rank ^ 1)));
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_cluster(fin_bar, 0)) {
+      if (globaltimer_ns() - t0 > a.timeout_ns) {
+        raise_status(a.status, ST_TIMEOUT);
+        break;
+      }
+    }
+  }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
