@@ -147,15 +147,19 @@ bool get_encode() {
 
 // 2-D bf16 row-major tensor [outer][inner], 128-B swizzled boxes of
 // box_inner x box_outer elements; out-of-range elements read as zero.
+enum class Swz { k128, k64, none };
+
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-              uint32_t box_inner, uint32_t box_outer, bool swizzle = true) {
+              uint32_t box_inner, uint32_t box_outer, Swz swz = Swz::k128) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                              swz == Swz::k128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                              : swz == Swz::k64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_NONE,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -256,10 +260,11 @@ flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N,
 // `grid` counts SM pairs (clusters of two CTAs).
 template <int KIND>
 cudaError_t launch_gemm(int grid, cudaStream_t s, const CUtensorMap& mA, const CUtensorMap& mB,
-                        const CUtensorMap& mHi, const CUtensorMap& mLo, const GemmArgs& a, int kind) {
+                        const CUtensorMap& mHi, const CUtensorMap& mLo, const CUtensorMap& mOut,
+                        const CUtensorMap& mOutLo, const GemmArgs& a, int kind) {
   size_t slot;
   prof_begin(s, kind, &slot);
-  flce_gemm_kernel<KIND><<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mHi, mLo, a);
+  flce_gemm_kernel<KIND><<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mHi, mLo, mOut, mOutLo, a);
   prof_end(s, slot);
   return cudaGetLastError();
 }
@@ -291,7 +296,13 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BNH) &&
             make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
             make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK) &&
-            make_map(&mHi, dX, h, n, h * 2, BN, BM, false) && make_map(&mLo, lo, h, n, h * 2, BN, BM, false);
+            make_map(&mHi, dX, h, n, h * 2, BN, BM, Swz::none) && make_map(&mLo, lo, h, n, h * 2, BN, BM, Swz::none);
+  // 32 x 32 output boxes of the epilogues (64-byte swizzle)
+  CUtensorMap mGo, mDWo, mHio, mLoo;
+  ok = ok && make_map(&mGo, G, VC, n, VC * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
+       make_map(&mDWo, dW, h, v, h * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
+       make_map(&mHio, dX, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
+       make_map(&mLoo, lo, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64);
   if (!ok) return FLCE_ERR_CUDA;
 
   if (cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), stream) != cudaSuccess) return FLCE_ERR_CUDA;
@@ -327,7 +338,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     p1.num_units = P.tiles_m * P.splits;
     p1.vbase = 0;
     p1.vcount = static_cast<int>(V);
-    if (launch_gemm<KIND_LSE>(P.lse_clusters, stream, mX_k, mW_k, mHi, mLo, p1, KIND_LSE) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (launch_gemm<KIND_LSE>(P.lse_clusters, stream, mX_k, mW_k, mHi, mLo, mGo, mLoo, p1, KIND_LSE) != cudaSuccess) return FLCE_ERR_CUDA;
   }
   // Combine the splits: lse, loss, n_valid, 1/n.
   {
@@ -371,7 +382,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       g.k_blocks = static_cast<int>((H + BK - 1) / BK);
       g.num_units = g.tiles_m * g.tiles_n;
       const int grid = std::min(g.num_units, P.clusters);
-      if (launch_gemm<KIND_GRAD>(grid, stream, mX_k, mW_k, mHi, mLo, g, KIND_GRAD) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (launch_gemm<KIND_GRAD>(grid, stream, mX_k, mW_k, mHi, mLo, mGo, mLoo, g, KIND_GRAD) != cudaSuccess) return FLCE_ERR_CUDA;
     }
     {  // dW rows of the chunk
       GemmArgs d = b;
@@ -380,7 +391,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       d.k_blocks = static_cast<int>((N + BK - 1) / BK);
       d.num_units = d.tiles_m * d.tiles_n;
       const int grid = std::min(d.num_units, P.clusters);
-      if (launch_gemm<KIND_DW>(grid, stream, mG_mn, mX_mn, mHi, mLo, d, KIND_DW) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (launch_gemm<KIND_DW>(grid, stream, mG_mn, mX_mn, mHi, mLo, mDWo, mLoo, d, KIND_DW) != cudaSuccess) return FLCE_ERR_CUDA;
     }
     {  // dX accumulation
       GemmArgs d = b;
@@ -389,7 +400,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       d.k_blocks = (vcount + BK - 1) / BK;
       d.num_units = d.tiles_m * d.tiles_n;
       const int grid = std::min(d.num_units, P.clusters);
-      if (launch_gemm<KIND_DX>(grid, stream, mG_k, mW_mn, mHi, mLo, d, KIND_DX) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (launch_gemm<KIND_DX>(grid, stream, mG_k, mW_mn, mHi, mLo, mHio, mLoo, d, KIND_DX) != cudaSuccess) return FLCE_ERR_CUDA;
     }
   }
   return FLCE_OK;

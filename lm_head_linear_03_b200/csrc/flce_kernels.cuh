@@ -56,8 +56,16 @@ constexpr int NUM_THREADS = 192;
 constexpr int EPI_WARPS = 4;
 constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;    // double-buffered accumulator
-constexpr int NUM_BARRIERS = 2 * STAGES + 4 + 1;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
+// Epilogue staging: each epilogue warp owns two 4 KB buffers, each holding a
+// 32-row x 32-column bf16 box of the output (and, for dX, of the low half of
+// the running sum), stored with the 64-byte TMA swizzle.
+constexpr int EPI_BOX = 32;
+constexpr int EPI_BOX_BYTES = EPI_BOX * EPI_BOX * 2;
+constexpr int EPI_BUF_BYTES = 2 * EPI_BOX_BYTES;
+constexpr int EPI_WARP_BYTES = 2 * EPI_BUF_BYTES;
+constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP_BYTES;
+constexpr int NUM_BARRIERS = 2 * STAGES + 4 + 1 + 2 * EPI_WARPS;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr double LN2 = 0.6931471805599453;
 
@@ -199,16 +207,66 @@ __device__ __forceinline__ void epi_lse_tile(const GemmArgs& a, uint32_t taddr, 
   }
 }
 
+// Per-warp output staging.  A warp's 32 rows of one 32-column slice go through
+// shared memory and leave (or, for the dX sum, also arrive) as one TMA box, so
+// global memory sees whole 64-byte row segments instead of the one-row-per-
+// thread pattern of the tensor-memory layout.
+struct EpiStage {
+  uint8_t* ptr;    // this warp's staging area (generic pointer)
+  uint32_t addr;   // the same, shared address
+  uint32_t bar;    // two mbarriers for boxes loaded into the buffers (dX only)
+  uint32_t k;      // slices staged so far by this warp
+};
+
+// Byte offset of 16-byte chunk j (0..3) of row r in a 32 x 32 bf16 box stored
+// with the 64-byte swizzle (16-byte chunk index XOR bits 1..2 of the row).
+__device__ __forceinline__ uint32_t sw64(int r, int j) {
+  return static_cast<uint32_t>(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+}
+
+__device__ __forceinline__ void put_row32(uint8_t* box, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+    w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+    w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+    w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+    *reinterpret_cast<uint4*>(box + sw64(r, j)) = w;
+  }
+}
+
+// Store-only slice: make sure the buffer's previous store has read it, fill it
+// with fill(v) for this thread's row, then one lane ships the box.
+template <class Fill>
+__device__ __forceinline__ void stage_and_store(EpiStage& es, int lane, const CUtensorMap* map, int x, int y,
+                                                Fill fill) {
+  const uint32_t b = es.k & 1u;
+  if (lane == 0) bulk_wait_read<1>();
+  __syncwarp();
+  float v[32];
+  fill(v);
+  put_row32(es.ptr + b * EPI_BUF_BYTES, lane, v);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, es.addr + b * EPI_BUF_BYTES, x, y);
+    bulk_commit();
+  }
+  ++es.k;
+}
+
 // Pass 2: G = valid * (softmax - onehot) / n for one tile, stored as bf16.
-__device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb,
-                                              int row_local) {
+__device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local,
+                                              EpiStage& es, const CUtensorMap* mapG) {
   const int row = row0 + row_local;
+  const int lane = row_local & 31;
   const bool in_rows = row < a.N;
   const int yr = in_rows ? a.y[row] : a.ignore_index;
   const bool valid = in_rows && yr != a.ignore_index;
   const float l2 = valid ? a.lse2[row] : 0.f;
   const float scale = valid ? *a.inv_n : 0.f;
-  uint16_t* grow = a.G + static_cast<size_t>(in_rows ? row : 0) * a.Vc + nb * BN;
+  const int wrow0 = row0 + (row_local & ~31);
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
@@ -216,128 +274,114 @@ __device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr,
     tmem_ld_wait();
     const int colg0 = a.vbase + nb * BN + c * 32;
     const int lim = a.V - colg0;
-    float g[32];
-#pragma unroll
-    for (int t = 0; t < 32; ++t)
-      g[t] = (valid && t < lim) ? ex2_approx(fmaf(__uint_as_float(r[t]), LOG2E, -l2)) * scale : 0.f;
-    const int off = yr - colg0;
-    if (valid && static_cast<unsigned>(off) < 32u) {
+    stage_and_store(es, lane, mapG, nb * BN + c * 32, wrow0, [&](float (&g)[32]) {
 #pragma unroll
       for (int t = 0; t < 32; ++t)
-        if (t == off) g[t] -= scale;
-    }
-    if (in_rows) {
-      uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
+        g[t] = (valid && t < lim) ? ex2_approx(fmaf(__uint_as_float(r[t]), LOG2E, -l2)) * scale : 0.f;
+      const int off = yr - colg0;
+      if (valid && static_cast<unsigned>(off) < 32u) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 v;
-        v.x = pack_bf16x2(g[8 * q + 0], g[8 * q + 1]);
-        v.y = pack_bf16x2(g[8 * q + 2], g[8 * q + 3]);
-        v.z = pack_bf16x2(g[8 * q + 4], g[8 * q + 5]);
-        v.w = pack_bf16x2(g[8 * q + 6], g[8 * q + 7]);
-        dst[q] = v;
+        for (int t = 0; t < 32; ++t)
+          if (t == off) g[t] -= scale;
       }
-    }
+    });
   }
 }
 
 // dW rows of this chunk: the K = tokens contraction is complete, round to bf16.
-__device__ __forceinline__ void epi_dw_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local) {
-  const int vrow_local = row0 + row_local;
-  const bool in_rows = vrow_local < a.vcount;
-  uint16_t* drow = a.dW + static_cast<size_t>(a.vbase + (in_rows ? vrow_local : 0)) * a.H;
+__device__ __forceinline__ void epi_dw_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local,
+                                            EpiStage& es, const CUtensorMap* mapDW) {
+  const int lane = row_local & 31;
+  const int wrow0 = a.vbase + row0 + (row_local & ~31);
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
-    const int col0 = nb * BN + c * 32;
-    if (in_rows) {
+    stage_and_store(es, lane, mapDW, nb * BN + c * 32, wrow0, [&](float (&v)[32]) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (col0 + 8 * q < a.H) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-          v.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-          v.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-          v.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-          *reinterpret_cast<uint4*>(drow + col0 + 8 * q) = v;
-        }
-      }
-    }
+      for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+    });
   }
 }
 
 // dX += G_c W_c.  The running sum lives in two bf16 words, hi (in dX itself) and
 // lo (workspace), with value = hi + lo: about 16 significant bits, enough for an
 // fp32-grade sum over the chunks, at the memory cost of one bf16 copy of dX.
-// The hi/lo words of the next 32 columns are loaded while the current ones are
-// combined and stored, so two chunks of reads are in flight per thread.
-__device__ __forceinline__ void dx_load_hl(const uint16_t* hrow, const uint16_t* lrow, int col0, int H, uint4 (&h)[4],
-                                           uint4 (&l)[4]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    if (col0 + 8 * q < H) {
-      h[q] = *reinterpret_cast<const uint4*>(hrow + col0 + 8 * q);
-      l[q] = *reinterpret_cast<const uint4*>(lrow + col0 + 8 * q);
-    } else {
-      h[q] = make_uint4(0, 0, 0, 0);
-      l[q] = make_uint4(0, 0, 0, 0);
-    }
-  }
-}
-
-__device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local) {
-  const int row = row0 + row_local;
-  const bool in_rows = row < a.N;
+// Each 32-column slice of the warp's rows is read back (hi and lo boxes by TMA,
+// one slice ahead), combined with the accumulator and written back by TMA.
+__device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local,
+                                            EpiStage& es, const CUtensorMap* mapHi, const CUtensorMap* mapLo,
+                                            volatile int* abort_flag, bool& ok) {
+  const int lane = row_local & 31;
+  const int wrow0 = row0 + (row_local & ~31);
   const bool accumulate = !a.first_chunk;
-  const size_t rbase = static_cast<size_t>(in_rows ? row : 0) * a.H;
-  uint16_t* hrow = a.dX + rbase;
-  uint16_t* lrow = a.lo + rbase;
-  uint4 hc[4], lc[4];
-  if (in_rows && accumulate) dx_load_hl(hrow, lrow, nb * BN, a.H, hc, lc);
+  constexpr int SLICES = BN / 32;
+  auto fetch = [&](uint32_t b, int c) {  // lane 0: hi and lo boxes of slice c into buffer b
+    bulk_wait_read<0>();                 // the buffer's previous store has read it
+    fence_proxy_async_smem();
+    const uint32_t bar = es.bar + 8u * b;
+    mbar_arrive_expect_tx(bar, 2 * EPI_BOX_BYTES);
+    tma_load_2d(es.addr + b * EPI_BUF_BYTES, mapHi, bar, nb * BN + c * 32, wrow0);
+    tma_load_2d(es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, mapLo, bar, nb * BN + c * 32, wrow0);
+  };
+  if (accumulate && lane == 0) fetch(es.k & 1u, 0);
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = 0; c < SLICES; ++c) {
+    const uint32_t b = es.k & 1u;
+    if (accumulate) {
+      if (c + 1 < SLICES && lane == 0) fetch(b ^ 1u, c + 1);
+    } else {
+      if (lane == 0) bulk_wait_read<1>();
+    }
+    __syncwarp();
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
-    const int col0 = nb * BN + c * 32;
-    uint4 hn[4], ln[4];
-    if (in_rows && accumulate && c + 1 < BN / 32) dx_load_hl(hrow, lrow, col0 + 32, a.H, hn, ln);
-    if (in_rows) {
+    uint8_t* hbox = es.ptr + b * EPI_BUF_BYTES;
+    uint8_t* lbox = hbox + EPI_BOX_BYTES;
+    float v[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int col = col0 + 8 * q;
-        if (col < a.H) {
-          float v[8];
+    for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+    if (accumulate) {
+      const bool got = mbar_wait(es.bar + 8u * b, (es.k >> 1) & 1u, abort_flag, a.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        return;
+      }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]);
-          if (accumulate) {
-            const uint32_t hw[4] = {hc[q].x, hc[q].y, hc[q].z, hc[q].w};
-            const uint32_t lw[4] = {lc[q].x, lc[q].y, lc[q].z, lc[q].w};
+      for (int j = 0; j < 4; ++j) {
+        const uint4 h = *reinterpret_cast<const uint4*>(hbox + sw64(lane, j));
+        const uint4 l = *reinterpret_cast<const uint4*>(lbox + sw64(lane, j));
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+        const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              v[2 * e] += bf16lo_to_f32(hw[e]) + bf16lo_to_f32(lw[e]);
-              v[2 * e + 1] += bf16hi_to_f32(hw[e]) + bf16hi_to_f32(lw[e]);
-            }
-          }
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hw[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-            lw[e] = pack_bf16x2(v[2 * e] - bf16lo_to_f32(hw[e]), v[2 * e + 1] - bf16hi_to_f32(hw[e]));
-          }
-          *reinterpret_cast<uint4*>(hrow + col) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          if (!a.last_chunk)
-            *reinterpret_cast<uint4*>(lrow + col) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        for (int e = 0; e < 4; ++e) {
+          v[8 * j + 2 * e] += bf16lo_to_f32(hw[e]) + bf16lo_to_f32(lw[e]);
+          v[8 * j + 2 * e + 1] += bf16hi_to_f32(hw[e]) + bf16hi_to_f32(lw[e]);
         }
       }
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      hc[q] = hn[q];
-      lc[q] = ln[q];
+    for (int j = 0; j < 4; ++j) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = v[8 * j + 2 * e], x1 = v[8 * j + 2 * e + 1];
+        hw[e] = pack_bf16x2(x0, x1);
+        lw[e] = pack_bf16x2(x0 - bf16lo_to_f32(hw[e]), x1 - bf16hi_to_f32(hw[e]));
+      }
+      *reinterpret_cast<uint4*>(hbox + sw64(lane, j)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(lbox + sw64(lane, j)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(mapHi, es.addr + b * EPI_BUF_BYTES, nb * BN + c * 32, wrow0);
+      if (!a.last_chunk) tma_store_2d(mapLo, es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, nb * BN + c * 32, wrow0);
+      bulk_commit();
+    }
+    ++es.k;
   }
 }
 
@@ -347,6 +391,7 @@ template <int KIND>
 __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     flce_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                      const __grid_constant__ CUtensorMap mapHi, const __grid_constant__ CUtensorMap mapLo,
+                     const __grid_constant__ CUtensorMap mapOut, const __grid_constant__ CUtensorMap mapOutLo,
                      const GemmArgs a) {
   using T = KindTraits<KIND>;
   extern __shared__ uint8_t smem_raw[];
@@ -354,8 +399,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;  // swizzle atoms need 1024-B alignment
   uint8_t* base_ptr = smem_raw + (base - raw_addr);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + STAGES * STAGE_BYTES);
-  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin
+  uint8_t* epi_ptr = base_ptr + STAGES * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_ptr + EPI_BYTES);
+  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin, epi[EPI_WARPS][2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -383,12 +429,14 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       mbar_init(tempty_bar(b), CLUSTER * EPI_WARPS);  // leader: epilogue warps of both CTAs
     }
     mbar_init(fin_bar, 1);  // the peer's end-of-work signal
+    for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(smem_u32(bars + 2 * STAGES + 5 + e), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&mapA);
     prefetch_tmap(&mapB);
+    prefetch_tmap(&mapOut);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
@@ -517,6 +565,11 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
     const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
+    EpiStage es;
+    es.ptr = epi_ptr + q * EPI_WARP_BYTES;
+    es.addr = smem_u32(es.ptr);
+    es.bar = smem_u32(bars + 2 * STAGES + 5 + 2 * q);
+    es.k = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -543,9 +596,15 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
         if constexpr (KIND == KIND_LSE) epi_lse_tile(a, taddr, nb, st);
-        if constexpr (KIND == KIND_GRAD) epi_grad_tile(a, taddr, row0, nb, row_local);
-        if constexpr (KIND == KIND_DW) epi_dw_tile(a, taddr, row0, nb, row_local);
-        if constexpr (KIND == KIND_DX) epi_dx_tile(a, taddr, row0, nb, row_local);
+        if constexpr (KIND == KIND_GRAD) epi_grad_tile(a, taddr, row0, nb, row_local, es, &mapOut);
+        if constexpr (KIND == KIND_DW) epi_dw_tile(a, taddr, row0, nb, row_local, es, &mapOut);
+        if constexpr (KIND == KIND_DX) {
+          epi_dx_tile(a, taddr, row0, nb, row_local, es, &mapOut, &mapOutLo, abort_flag, ok);
+          if (!ok) {
+            give_up();
+            break;
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
@@ -560,6 +619,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         }
       }
     }
+    if (lane == 0) bulk_wait<0>();  // every staged box written out before the CTA winds down
   }
 
   // Wind-down: this CTA's work is done; tell the peer, wait (bounded) for the
