@@ -349,7 +349,10 @@ def run_ours(args, world, rank, local):
     dom = max(kinds, key=lambda k: kinds[k][1])
     n_launch, tot_ms = kinds[dom]
     per_step_launches = n_launch / args.steps
-    algo_flops_per_launch = (2.0 * N * H * V) / per_step_launches if dom != "combine_lse_loss" else None
+    # algorithmic FLOPs of one step, per kernel kind: pass 1 is one N x H x V
+    # GEMM; pass 2 recomputes the logits and runs the dX and dW contractions
+    flops_per_step_kind = {"pass1_logits_lse": 2.0 * N * H * V, "pass2_grad_dw_dx": 6.0 * N * H * V}
+    algo_flops_per_launch = flops_per_step_kind.get(dom, 0.0) / per_step_launches
     avg_ms = tot_ms / n_launch
     sustained = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     achieved = algo_flops_per_launch / (avg_ms * 1e-3) / 1e12

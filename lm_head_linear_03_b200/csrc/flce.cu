@@ -27,7 +27,7 @@ constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per bou
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t ctrl, lse2, zy, part_m, part_l, blk_loss, blk_cnt, G, lo, total;
+  size_t ctrl, counters, counters_bytes, lse2, zy, part_m, part_l, blk_loss, blk_cnt, G, lo, total;
 };
 
 // ctrl block: [0] status, [4] ticket, [8] n_valid, [12] inv_n, [16] loss
@@ -50,6 +50,10 @@ WsLayout ws_layout(int64_t N, int64_t H) {
   const size_t n = static_cast<size_t>(N);
   const size_t nblk = (n + COMBINE_THREADS - 1) / COMBINE_THREADS;
   L.ctrl = take(256);
+  // pass-2 completion counters: g_row[TM], x_row[TM], g_col[VC/BN], w_col[VC/BN]
+  const size_t tm = (n + CM - 1) / CM;
+  L.counters_bytes = (2 * tm + 2 * (VC / BN)) * 4;
+  L.counters = take(L.counters_bytes);
   L.lse2 = take(n * 4);
   L.zy = take(n * 4);
   L.part_m = take(static_cast<size_t>(MAX_SPLITS) * n * 4);
@@ -101,14 +105,8 @@ cudaError_t set_kernel_attrs(int dev) {
   if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SMEM_BYTES)) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_GRAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SMEM_BYTES)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_DW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SMEM_BYTES)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_DX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SMEM_BYTES)) != cudaSuccess)
+  if ((e = cudaFuncSetAttribute(flce_pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+      cudaSuccess)
     return e;
   // How many SM pairs the GEMM kernels can occupy at once (persistent grids).
   cudaLaunchConfig_t cfg = {};
@@ -122,8 +120,10 @@ cudaError_t set_kernel_attrs(int dev) {
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  int clusters = 0;
+  int clusters = 0, clusters2 = 0;
   if ((e = cudaOccupancyMaxActiveClusters(&clusters, flce_gemm_kernel<KIND_LSE>, &cfg)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters2, flce_pass2_kernel, &cfg)) != cudaSuccess) return e;
+  clusters = std::min(clusters, clusters2);
   if (clusters <= 0) return cudaErrorInvalidConfiguration;
   g_dev[dev].max_clusters = clusters;
   g_attr_set[dev] = true;
@@ -210,7 +210,7 @@ Plan make_plan(int64_t N, int64_t H, int64_t V, int clusters) {
   p.lse_clusters =
       static_cast<int>(std::min<long long>(static_cast<long long>(p.tiles_m) * p.splits, clusters));
   p.num_chunks = static_cast<int>((V + VC - 1) / VC);
-  p.launches = 2 + 3 * p.num_chunks;
+  p.launches = 3;  // pass 1, combine, pass 2
   return p;
 }
 
@@ -305,7 +305,8 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
        make_map(&mLoo, lo, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64);
   if (!ok) return FLCE_ERR_CUDA;
 
-  if (cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  // control words and pass-2 counters start at zero (they are contiguous)
+  if (cudaMemsetAsync(ctrl, 0, L.counters + L.counters_bytes - L.ctrl, stream) != cudaSuccess) return FLCE_ERR_CUDA;
   if (d_status != &ctrl->status && cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess)
     return FLCE_ERR_CUDA;
 
@@ -366,42 +367,46 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     prof_end(stream, slot);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
-  // Pass 2, one vocabulary chunk at a time.
-  for (int ch = 0; ch < P.num_chunks; ++ch) {
-    const int vbase = ch * VC;
-    const int vcount = static_cast<int>(std::min<int64_t>(VC, V - vbase));
+  // Pass 2: every chunk's logit recompute, dW and dX tiles in one persistent launch.
+  {
     GemmArgs b = a;
-    b.vbase = vbase;
-    b.vcount = vcount;
-    b.first_chunk = ch == 0;
-    b.last_chunk = ch == P.num_chunks - 1;
-    {  // recompute logits, G chunk
-      GemmArgs g = b;
-      g.tiles_m = P.tiles_m;
-      g.tiles_n = (vcount + BN - 1) / BN;
-      g.k_blocks = static_cast<int>((H + BK - 1) / BK);
-      g.num_units = g.tiles_m * g.tiles_n;
-      const int grid = std::min(g.num_units, P.clusters);
-      if (launch_gemm<KIND_GRAD>(grid, stream, mX_k, mW_k, mHi, mLo, mGo, mLoo, g, KIND_GRAD) != cudaSuccess) return FLCE_ERR_CUDA;
+    b.TM = P.tiles_m;
+    b.HN = static_cast<int>((H + BN - 1) / BN);
+    b.C = P.num_chunks;
+    b.VTf = VC / BN;
+    b.VT_last = static_cast<int>((V - static_cast<int64_t>(P.num_chunks - 1) * VC + BN - 1) / BN);
+    if (b.C == 1) b.VTf = b.VT_last;
+    long long total = static_cast<long long>(b.C == 1 ? b.VT_last : b.VTf) * b.TM;  // G(0)
+    for (int c = 0; c < b.C; ++c) {
+      const long long vt = c == b.C - 1 ? b.VT_last : b.VTf;
+      total += static_cast<long long>(b.TM) * b.HN + vt * b.HN;
+      if (c + 1 < b.C) total += static_cast<long long>(c + 1 == b.C - 1 ? b.VT_last : b.VTf) * b.TM;
     }
-    {  // dW rows of the chunk
-      GemmArgs d = b;
-      d.tiles_m = (vcount + CM - 1) / CM;
-      d.tiles_n = static_cast<int>((H + BN - 1) / BN);
-      d.k_blocks = static_cast<int>((N + BK - 1) / BK);
-      d.num_units = d.tiles_m * d.tiles_n;
-      const int grid = std::min(d.num_units, P.clusters);
-      if (launch_gemm<KIND_DW>(grid, stream, mG_mn, mX_mn, mHi, mLo, mDWo, mLoo, d, KIND_DW) != cudaSuccess) return FLCE_ERR_CUDA;
-    }
-    {  // dX accumulation
-      GemmArgs d = b;
-      d.tiles_m = P.tiles_m;
-      d.tiles_n = static_cast<int>((H + BN - 1) / BN);
-      d.k_blocks = (vcount + BK - 1) / BK;
-      d.num_units = d.tiles_m * d.tiles_n;
-      const int grid = std::min(d.num_units, P.clusters);
-      if (launch_gemm<KIND_DX>(grid, stream, mG_k, mW_mn, mHi, mLo, mHio, mLoo, d, KIND_DX) != cudaSuccess) return FLCE_ERR_CUDA;
-    }
+    b.total_items = total;
+    int* ctr = reinterpret_cast<int*>(ws + L.counters);
+    b.g_row = ctr;
+    b.x_row = ctr + b.TM;
+    b.g_col = ctr + 2 * b.TM;
+    b.w_col = ctr + 2 * b.TM + VC / BN;
+    Pass2Maps pm;
+    pm.Xk = mX_k;
+    pm.Wk = mW_k;
+    pm.Gmn = mG_mn;
+    pm.Xmn = mX_mn;
+    pm.Gk = mG_k;
+    pm.Wmn = mW_mn;
+    pm.Go = mGo;
+    pm.DWo = mDWo;
+    pm.Hio = mHio;
+    pm.Loo = mLoo;
+    pm.Hipf = mHi;
+    pm.Lopf = mLo;
+    const int grid = static_cast<int>(std::min<long long>(total, P.clusters));
+    size_t slot;
+    prof_begin(stream, KIND_PASS2, &slot);
+    flce_pass2_kernel<<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, stream>>>(pm, b);
+    prof_end(stream, slot);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
   return FLCE_OK;
 }
@@ -515,9 +520,7 @@ const char* flce_kernel_name(int kind) {
   switch (kind) {
     case KIND_LSE: return "pass1_logits_lse";
     case KIND_COMBINE: return "combine_lse_loss";
-    case KIND_GRAD: return "pass2_logits_grad";
-    case KIND_DW: return "dW_contraction";
-    case KIND_DX: return "dX_contraction";
+    case KIND_PASS2: return "pass2_grad_dw_dx";
     default: return "unknown";
   }
 }

@@ -69,7 +69,8 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*alignment*/
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr double LN2 = 0.6931471805599453;
 
-enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_GRAD = 2, KIND_DW = 3, KIND_DX = 4 };
+// GEMM kinds of the templated kernel, and kinds of launch for the profiler.
+enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_GRAD = 3, KIND_DW = 4, KIND_DX = 5 };
 enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
 
 struct GemmArgs {
@@ -93,6 +94,15 @@ struct GemmArgs {
   uint16_t* lo;           // [N][H] bf16, low half of the dX accumulator
   int* status;
   unsigned long long timeout_ns;
+  // pass 2 (one persistent launch over every chunk)
+  int TM, HN;             // 256-row token tiles, 256-column hidden tiles
+  int C;                  // vocabulary chunks
+  int VTf, VT_last;       // 256-wide vocabulary tiles in a full / the last chunk
+  long long total_items;
+  int* g_row;             // [TM]  G tiles finished per token tile    (x EPI_WARPS*CLUSTER)
+  int* g_col;             // [VTf] G tiles finished per chunk column  (x EPI_WARPS*CLUSTER)
+  int* x_row;             // [TM]  dX tiles finished per token tile   (x EPI_WARPS*CLUSTER)
+  int* w_col;             // [VTf] dW tiles finished per chunk column (x EPI_WARPS*CLUSTER)
 };
 
 template <int KIND> struct KindTraits;
@@ -257,8 +267,8 @@ __device__ __forceinline__ void stage_and_store(EpiStage& es, int lane, const CU
 }
 
 // Pass 2: G = valid * (softmax - onehot) / n for one tile, stored as bf16.
-__device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local,
-                                              EpiStage& es, const CUtensorMap* mapG) {
+__device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, int vbase, uint32_t taddr, int row0, int nb,
+                                              int row_local, EpiStage& es, const CUtensorMap* mapG) {
   const int row = row0 + row_local;
   const int lane = row_local & 31;
   const bool in_rows = row < a.N;
@@ -272,7 +282,7 @@ __device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr,
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
-    const int colg0 = a.vbase + nb * BN + c * 32;
+    const int colg0 = vbase + nb * BN + c * 32;
     const int lim = a.V - colg0;
     stage_and_store(es, lane, mapG, nb * BN + c * 32, wrow0, [&](float (&g)[32]) {
 #pragma unroll
@@ -289,10 +299,10 @@ __device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, uint32_t taddr,
 }
 
 // dW rows of this chunk: the K = tokens contraction is complete, round to bf16.
-__device__ __forceinline__ void epi_dw_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local,
+__device__ __forceinline__ void epi_dw_tile(int vbase, uint32_t taddr, int row0, int nb, int row_local,
                                             EpiStage& es, const CUtensorMap* mapDW) {
   const int lane = row_local & 31;
-  const int wrow0 = a.vbase + row0 + (row_local & ~31);
+  const int wrow0 = vbase + row0 + (row_local & ~31);
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
@@ -310,12 +320,12 @@ __device__ __forceinline__ void epi_dw_tile(const GemmArgs& a, uint32_t taddr, i
 // fp32-grade sum over the chunks, at the memory cost of one bf16 copy of dX.
 // Each 32-column slice of the warp's rows is read back (hi and lo boxes by TMA,
 // one slice ahead), combined with the accumulator and written back by TMA.
-__device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, int row0, int nb, int row_local,
-                                            EpiStage& es, const CUtensorMap* mapHi, const CUtensorMap* mapLo,
-                                            volatile int* abort_flag, bool& ok) {
+__device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk, bool last_chunk, uint32_t taddr,
+                                            int row0, int nb, int row_local, EpiStage& es, const CUtensorMap* mapHi,
+                                            const CUtensorMap* mapLo, volatile int* abort_flag, bool& ok) {
   const int lane = row_local & 31;
   const int wrow0 = row0 + (row_local & ~31);
-  const bool accumulate = !a.first_chunk;
+  const bool accumulate = !first_chunk;
   constexpr int SLICES = BN / 32;
   auto fetch = [&](uint32_t b, int c) {  // lane 0: hi and lo boxes of slice c into buffer b
     bulk_wait_read<0>();                 // the buffer's previous store has read it
@@ -378,7 +388,7 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, uint32_t taddr, i
     __syncwarp();
     if (lane == 0) {
       tma_store_2d(mapHi, es.addr + b * EPI_BUF_BYTES, nb * BN + c * 32, wrow0);
-      if (!a.last_chunk) tma_store_2d(mapLo, es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, nb * BN + c * 32, wrow0);
+      if (!last_chunk) tma_store_2d(mapLo, es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, nb * BN + c * 32, wrow0);
       bulk_commit();
     }
     ++es.k;
@@ -596,10 +606,11 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
         if constexpr (KIND == KIND_LSE) epi_lse_tile(a, taddr, nb, st);
-        if constexpr (KIND == KIND_GRAD) epi_grad_tile(a, taddr, row0, nb, row_local, es, &mapOut);
-        if constexpr (KIND == KIND_DW) epi_dw_tile(a, taddr, row0, nb, row_local, es, &mapOut);
+        if constexpr (KIND == KIND_GRAD) epi_grad_tile(a, a.vbase, taddr, row0, nb, row_local, es, &mapOut);
+        if constexpr (KIND == KIND_DW) epi_dw_tile(a.vbase, taddr, row0, nb, row_local, es, &mapOut);
         if constexpr (KIND == KIND_DX) {
-          epi_dx_tile(a, taddr, row0, nb, row_local, es, &mapOut, &mapOutLo, abort_flag, ok);
+          epi_dx_tile(a, a.first_chunk, a.last_chunk, taddr, row0, nb, row_local, es, &mapOut, &mapOutLo,
+                      abort_flag, ok);
           if (!ok) {
             give_up();
             break;
@@ -624,6 +635,393 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
 
   // Wind-down: this CTA's work is done; tell the peer, wait (bounded) for the
   // peer to say the same, then free the pair's tensor memory together.
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_cluster(mapa_shared(fin_bar, static_cast<uint32_t>(rank ^ 1)));
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_cluster(fin_bar, 0)) {
+      if (globaltimer_ns() - t0 > a.timeout_ns) {
+        raise_status(a.status, ST_TIMEOUT);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+// ===================================================== pass 2, one launch ==
+//
+// All of pass 2 runs as one persistent launch over a static queue of work
+// items, dealt round-robin to the SM pairs:
+//
+//   G(0)  |  dX(0) dW(0) G(1)  |  dX(1) dW(1) G(2)  | ... |  dX(C-1) dW(C-1)
+//
+// where G(c) are the logit-recompute tiles of chunk c (column-major), dX(c) the
+// dX += G_c W_c tiles and dW(c) the dW rows of chunk c.  There is one G buffer,
+// so items wait for what they read and for the readers of what they overwrite:
+//   dX(c) mainloop  after G(c) of its token tile (all its columns),
+//   dX(c) epilogue  after dX(c-1) of its token tile (running sum),
+//   dW(c) mainloop  after G(c) of its column (all token tiles),
+//   G(c)  epilogue  after dX(c-1) of its token tile and dW(c-1) of its column.
+// Every dependency points to an earlier item and all SM pairs are resident at
+// once, so the queue always drains.  Completion is counted per token tile /
+// column in monotonic counters: each epilogue warp adds one after its TMA
+// stores have landed, so a finished item adds EPI_WARPS * CLUSTER.
+
+enum : int { ITEM_GRAD = 0, ITEM_DW = 1, ITEM_DX = 2 };
+
+struct Item {
+  int kind, c, a, b;  // G: (tm, vb)  dW: (vm, hn)  dX: (tm, hn)
+};
+
+__device__ __forceinline__ int chunk_vtiles(const GemmArgs& p, int c) { return c == p.C - 1 ? p.VT_last : p.VTf; }
+
+__device__ __forceinline__ long long section_size(const GemmArgs& p, int c) {
+  long long n = static_cast<long long>(p.TM) * p.HN + static_cast<long long>(chunk_vtiles(p, c)) * p.HN;
+  if (c + 1 < p.C) n += static_cast<long long>(chunk_vtiles(p, c + 1)) * p.TM;
+  return n;
+}
+
+__device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
+  Item it;
+  const long long g0 = static_cast<long long>(chunk_vtiles(p, 0)) * p.TM;
+  if (i < g0) {
+    it.kind = ITEM_GRAD;
+    it.c = 0;
+    it.b = static_cast<int>(i / p.TM);
+    it.a = static_cast<int>(i - static_cast<long long>(it.b) * p.TM);
+    return it;
+  }
+  // sections 0 .. C-3 all have the size of section 0; the last two may be shorter
+  long long r = i - g0;
+  int c = 0;
+  if (p.C >= 3) {
+    const long long full = section_size(p, 0);
+    c = static_cast<int>(min(r / full, static_cast<long long>(p.C - 3)));
+    r -= static_cast<long long>(c) * full;
+  }
+  while (c + 1 < p.C && r >= section_size(p, c)) {
+    r -= section_size(p, c);
+    ++c;
+  }
+  const long long nx = static_cast<long long>(p.TM) * p.HN;
+  const long long nw = static_cast<long long>(chunk_vtiles(p, c)) * p.HN;
+  it.c = c;
+  if (r < nx) {
+    it.kind = ITEM_DX;
+    it.a = static_cast<int>(r / p.HN);
+    it.b = static_cast<int>(r - static_cast<long long>(it.a) * p.HN);
+  } else if (r < nx + nw) {
+    r -= nx;
+    it.kind = ITEM_DW;
+    it.a = static_cast<int>(r / p.HN);
+    it.b = static_cast<int>(r - static_cast<long long>(it.a) * p.HN);
+  } else {
+    r -= nx + nw;
+    it.kind = ITEM_GRAD;
+    it.c = c + 1;
+    it.b = static_cast<int>(r / p.TM);
+    it.a = static_cast<int>(r - static_cast<long long>(it.b) * p.TM);
+  }
+  return it;
+}
+
+constexpr int SIGNALS_PER_ITEM = EPI_WARPS * CLUSTER;
+
+// Pass-2 tensor maps, in one struct so they travel as one kernel parameter.
+struct Pass2Maps {
+  CUtensorMap Xk, Wk;      // G: X rows and W rows, K-major
+  CUtensorMap Gmn, Xmn;    // dW: G_c^T and X, MN-major
+  CUtensorMap Gk, Wmn;     // dX: G_c rows K-major, W_c MN-major
+  CUtensorMap Go, DWo;     // epilogue output boxes of G and dW
+  CUtensorMap Hio, Loo;    // epilogue boxes of the dX running sum (hi = dX, lo)
+  CUtensorMap Hipf, Lopf;  // whole-tile L2 prefetch of the running sum
+};
+
+__global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    flce_pass2_kernel(const __grid_constant__ Pass2Maps m, const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw_addr);
+  uint8_t* epi_ptr = base_ptr + STAGES * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_ptr + EPI_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool leader = rank == 0;
+  const long long cid = blockIdx.x / CLUSTER;
+  const long long ncl = gridDim.x / CLUSTER;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 + b); };
+  const uint32_t fin_bar = smem_u32(bars + 2 * STAGES + 4);
+  auto sA = [&](int s) { return base + s * STAGE_BYTES; };
+  auto sB = [&](int s) { return base + s * STAGE_BYTES + A_TILE_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), CLUSTER * EPI_WARPS);
+    }
+    mbar_init(fin_bar, 1);
+    for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(smem_u32(bars + 2 * STAGES + 5 + e), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&m.Xk);
+    prefetch_tmap(&m.Wk);
+    prefetch_tmap(&m.Gmn);
+    prefetch_tmap(&m.Xmn);
+    prefetch_tmap(&m.Gk);
+    prefetch_tmap(&m.Wmn);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    raise_status(a.status, ST_TIMEOUT);
+  };
+  // cumulative G tiles of token tile tm after chunk c
+  auto g_row_target = [&](int c) {
+    return SIGNALS_PER_ITEM * (c < a.C - 1 ? (c + 1) * a.VTf : (a.C - 1) * a.VTf + a.VT_last);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (long long u = cid; ok && u < a.total_items; u += ncl) {
+        const Item it = decode_item(a, u);
+        const int vbase = it.c * a.Vc;
+        const int vcount = min(a.Vc, a.V - vbase);
+        int kblocks;
+        if (it.kind == ITEM_GRAD) {
+          kblocks = (a.H + BK - 1) / BK;
+        } else if (it.kind == ITEM_DW) {
+          kblocks = (a.N + BK - 1) / BK;
+          ok = wait_counter(a.g_col + it.a, SIGNALS_PER_ITEM * a.TM * (it.c + 1), abort_flag, a.timeout_ns);
+        } else {
+          kblocks = (vcount + BK - 1) / BK;
+          ok = wait_counter(a.g_row + it.a, g_row_target(it.c), abort_flag, a.timeout_ns);
+          // pull this CTA's rows of the running sum into L2 if they are final already
+          if (ok && it.c > 0 && ld_acquire_gpu(a.x_row + it.a) >= SIGNALS_PER_ITEM * it.c * a.HN) {
+            fence_proxy_async_global();
+            tma_prefetch_l2_2d(&m.Hipf, it.b * BN, it.a * CM + rank * BM);
+            tma_prefetch_l2_2d(&m.Lopf, it.b * BN, it.a * CM + rank * BM);
+          }
+        }
+        if (!ok) {
+          give_up();
+          break;
+        }
+        fence_proxy_async_global();  // G written by other CTAs' TMA stores, read by TMA below
+        const int m0 = it.a * CM + rank * BM;
+        const int n0 = it.b * BN + rank * BNH;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * STAGE_BYTES);
+          const uint32_t bar = mapa_shared(full_bar(stage), 0);
+          const int k0 = kb * BK;
+          if (it.kind == ITEM_GRAD) {
+            tma_load_2d_pair(sA(stage), &m.Xk, bar, k0, m0);
+            tma_load_2d_pair(sB(stage), &m.Wk, bar, k0, vbase + n0);
+          } else if (it.kind == ITEM_DW) {
+#pragma unroll
+            for (int i = 0; i < BM / 64; ++i) tma_load_2d_pair(sA(stage) + i * MN_BOX_BYTES, &m.Gmn, bar, m0 + i * 64, k0);
+#pragma unroll
+            for (int i = 0; i < BNH / 64; ++i)
+              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, &m.Xmn, bar, n0 + i * 64, k0);
+          } else {
+            tma_load_2d_pair(sA(stage), &m.Gk, bar, k0, m0);
+#pragma unroll
+            for (int i = 0; i < BNH / 64; ++i)
+              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, &m.Wmn, bar, n0 + i * 64, vbase + k0);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      for (int i = 0; i < STAGES; ++i) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          break;
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (*abort_flag) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 100000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ UMMA issuer (leader) --
+    if (leader && lane == 0) {
+      constexpr uint32_t ID_GRAD = idesc_bf16_f32(CM, BN, false, false);
+      constexpr uint32_t ID_DW = idesc_bf16_f32(CM, BN, true, true);
+      constexpr uint32_t ID_DX = idesc_bf16_f32(CM, BN, false, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (long long u = cid; ok && u < a.total_items; u += ncl) {
+        const Item it = decode_item(a, u);
+        const int vcount = min(a.Vc, a.V - it.c * a.Vc);
+        const int kblocks = it.kind == ITEM_GRAD ? (a.H + BK - 1) / BK
+                            : it.kind == ITEM_DW ? (a.N + BK - 1) / BK
+                                                 : (vcount + BK - 1) / BK;
+        const uint32_t idesc = it.kind == ITEM_GRAD ? ID_GRAD : it.kind == ITEM_DW ? ID_DW : ID_DX;
+        const bool a_mn = it.kind == ITEM_DW;
+        const bool b_mn = it.kind != ITEM_GRAD;
+        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, a.timeout_ns)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            const uint64_t ad = a_mn ? operand_desc<true>(sA(stage), k) : operand_desc<false>(sA(stage), k);
+            const uint64_t bd = b_mn ? operand_desc<true>(sB(stage), k) : operand_desc<false>(sB(stage), k);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          umma_commit_pair(empty_bar(stage), 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(tfull_bar(acc), 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      for (int i = 0; i < 2; ++i) {
+        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          break;
+        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue --
+    const int q = warp & 3;
+    const int row_local = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
+    const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
+    EpiStage es;
+    es.ptr = epi_ptr + q * EPI_WARP_BYTES;
+    es.addr = smem_u32(es.ptr);
+    es.bar = smem_u32(bars + 2 * STAGES + 5 + 2 * q);
+    es.k = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (long long u = cid; ok && u < a.total_items; u += ncl) {
+      const Item it = decode_item(a, u);
+      const int vbase = it.c * a.Vc;
+      const int row0 = it.a * CM + rank * BM;
+      // wait for the previous readers (G) / writers (dX) of what this tile writes
+      if (lane == 0) {
+        if (it.kind == ITEM_GRAD && it.c > 0) {
+          ok = wait_counter(a.x_row + it.a, SIGNALS_PER_ITEM * it.c * a.HN, abort_flag, a.timeout_ns) &&
+               wait_counter(a.w_col + it.b, SIGNALS_PER_ITEM * it.c * a.HN, abort_flag, a.timeout_ns);
+        } else if (it.kind == ITEM_DX && it.c > 0) {
+          ok = wait_counter(a.x_row + it.a, SIGNALS_PER_ITEM * it.c * a.HN, abort_flag, a.timeout_ns);
+        }
+        if (ok) fence_proxy_async_global();
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) {
+        give_up();
+        break;
+      }
+      const bool got = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        give_up();
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
+      if (it.kind == ITEM_GRAD) {
+        epi_grad_tile(a, vbase, taddr, row0, it.b, row_local, es, &m.Go);
+      } else if (it.kind == ITEM_DW) {
+        epi_dw_tile(vbase, taddr, row0, it.b, row_local, es, &m.DWo);
+      } else {
+        epi_dx_tile(a, it.c == 0, it.c == a.C - 1, taddr, row0, it.b, row_local, es, &m.Hio, &m.Loo, abort_flag,
+                    ok);
+        if (!ok) {
+          give_up();
+          break;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+      // this warp's boxes have landed: count the tile as done for its readers
+      if (lane == 0) {
+        bulk_wait<0>();
+        fence_proxy_async_global();
+        if (it.kind == ITEM_GRAD) {
+          red_release_gpu_add(a.g_row + it.a, 1);
+          red_release_gpu_add(a.g_col + it.b, 1);
+        } else if (it.kind == ITEM_DW) {
+          red_release_gpu_add(a.w_col + it.a, 1);
+        } else {
+          red_release_gpu_add(a.x_row + it.a, 1);
+        }
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
