@@ -102,8 +102,8 @@ cudaError_t set_kernel_attrs(int dev) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_attr_set[dev]) return cudaSuccess;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(flce_gemm_kernel<KIND_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SMEM_BYTES)) != cudaSuccess)
+  if ((e = cudaFuncSetAttribute(flce_pass1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+      cudaSuccess)
     return e;
   if ((e = cudaFuncSetAttribute(flce_pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
       cudaSuccess)
@@ -121,7 +121,7 @@ cudaError_t set_kernel_attrs(int dev) {
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int clusters = 0, clusters2 = 0;
-  if ((e = cudaOccupancyMaxActiveClusters(&clusters, flce_gemm_kernel<KIND_LSE>, &cfg)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters, flce_pass1_kernel, &cfg)) != cudaSuccess) return e;
   if ((e = cudaOccupancyMaxActiveClusters(&clusters2, flce_pass2_kernel, &cfg)) != cudaSuccess) return e;
   clusters = std::min(clusters, clusters2);
   if (clusters <= 0) return cudaErrorInvalidConfiguration;
@@ -257,18 +257,6 @@ flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N,
 }
 
 // --------------------------------------------------------------- enqueue --
-// `grid` counts SM pairs (clusters of two CTAs).
-template <int KIND>
-cudaError_t launch_gemm(int grid, cudaStream_t s, const CUtensorMap& mA, const CUtensorMap& mB,
-                        const CUtensorMap& mHi, const CUtensorMap& mLo, const CUtensorMap& mOut,
-                        const CUtensorMap& mOutLo, const GemmArgs& a, int kind) {
-  size_t slot;
-  prof_begin(s, kind, &slot);
-  flce_gemm_kernel<KIND><<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mHi, mLo, mOut, mOutLo, a);
-  prof_end(s, slot);
-  return cudaGetLastError();
-}
-
 flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
                       int32_t ignore_index, float* d_loss, int32_t* d_status, uint16_t* dX, uint16_t* dW,
                       void* workspace, cudaStream_t stream) {
@@ -337,9 +325,11 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     p1.k_blocks = static_cast<int>((H + BK - 1) / BK);
     p1.splits = P.splits;
     p1.num_units = P.tiles_m * P.splits;
-    p1.vbase = 0;
-    p1.vcount = static_cast<int>(V);
-    if (launch_gemm<KIND_LSE>(P.lse_clusters, stream, mX_k, mW_k, mHi, mLo, mGo, mLoo, p1, KIND_LSE) != cudaSuccess) return FLCE_ERR_CUDA;
+    size_t slot;
+    prof_begin(stream, KIND_LSE, &slot);
+    flce_pass1_kernel<<<CLUSTER * P.lse_clusters, NUM_THREADS, SMEM_BYTES, stream>>>(mX_k, mW_k, p1);
+    prof_end(stream, slot);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
   // Combine the splits: lse, loss, n_valid, 1/n.
   {

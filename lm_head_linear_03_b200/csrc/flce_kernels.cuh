@@ -69,19 +69,17 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*alignment*/
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr double LN2 = 0.6931471805599453;
 
-// GEMM kinds of the templated kernel, and kinds of launch for the profiler.
-enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_GRAD = 3, KIND_DW = 4, KIND_DX = 5 };
+// Kinds of launch, as the profiler reports them.
+enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2 };
 enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
 
 struct GemmArgs {
   int N, H, V, ignore_index;
-  int tiles_m, tiles_n;   // tile grid of the launch
-  int k_blocks;           // BK-wide steps along K
-  int num_units;          // LSE: tiles_m * splits; otherwise tiles_m * tiles_n
-  int splits;             // LSE: vocabulary splits
-  int vbase, vcount;      // first vocabulary entry and entry count of this chunk
-  int Vc;                 // chunk width = row stride of the G buffer
-  int first_chunk, last_chunk;
+  int tiles_m, tiles_n;   // pass 1: 256-token tiles, 256-wide vocabulary tiles
+  int k_blocks;           // pass 1: BK-wide steps along K = H
+  int num_units;          // pass 1: tiles_m * splits
+  int splits;             // pass 1: vocabulary splits
+  int Vc;                 // pass 2: chunk width = row stride of the G buffer
   const int32_t* y;
   float* part_m;          // [splits][N] running max, log2 units
   float* part_l;          // [splits][N] running sum of 2^(s - m)
@@ -105,62 +103,31 @@ struct GemmArgs {
   int* w_col;             // [VTf] dW tiles finished per chunk column (x EPI_WARPS*CLUSTER)
 };
 
-template <int KIND> struct KindTraits;
-template <> struct KindTraits<KIND_LSE>  { static constexpr bool A_MN = false, B_MN = false; };
-template <> struct KindTraits<KIND_GRAD> { static constexpr bool A_MN = false, B_MN = false; };
-template <> struct KindTraits<KIND_DW>   { static constexpr bool A_MN = true,  B_MN = true;  };
-template <> struct KindTraits<KIND_DX>   { static constexpr bool A_MN = false, B_MN = true;  };
-
 __device__ __forceinline__ void raise_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
-// Work unit u -> token/vocab tile row mb and the range [nb_begin, nb_end) of
-// tile columns it walks.  Pass 1 walks one vocabulary split per unit, with
-// units ordered split-major so that CTAs running at the same time share the
-// same W tiles through L2; the other kinds have one tile per unit.
-template <int KIND>
+// Pass-1 work unit u -> token tile mb, vocabulary split `split` and the range
+// [nb_begin, nb_end) of 256-wide vocabulary tiles it walks.  Units are ordered
+// split-major, so that SM pairs running at the same time share the same W
+// tiles through L2.
 __device__ __forceinline__ void unit_range(const GemmArgs& a, int u, int& mb, int& nb_begin, int& nb_end,
                                            int& split) {
-  if constexpr (KIND == KIND_LSE) {
-    split = u / a.tiles_m;
-    mb = u - split * a.tiles_m;
-    nb_begin = static_cast<int>((static_cast<long long>(split) * a.tiles_n) / a.splits);
-    nb_end = static_cast<int>((static_cast<long long>(split + 1) * a.tiles_n) / a.splits);
-  } else {
-    split = 0;
-    nb_begin = u / a.tiles_m;
-    mb = u - nb_begin * a.tiles_m;
-    nb_end = nb_begin + 1;
-  }
+  split = u / a.tiles_m;
+  mb = u - split * a.tiles_m;
+  nb_begin = static_cast<int>((static_cast<long long>(split) * a.tiles_n) / a.splits);
+  nb_end = static_cast<int>((static_cast<long long>(split + 1) * a.tiles_n) / a.splits);
 }
 
-// TMA loads of one pipeline stage for the CTA of rank `rank` in the pair: its
-// 128 rows of A and its 128 columns of B.  Completion is counted on the
-// leader's full barrier `bar`.
-template <int KIND>
-__device__ __forceinline__ void load_stage(const GemmArgs& a, const CUtensorMap* mA, const CUtensorMap* mB,
-                                           uint32_t sA, uint32_t sB, uint32_t bar, int mb, int nb, int kb,
-                                           int rank) {
+// Pass-1 TMA loads of one pipeline stage for the CTA of rank `rank` in the pair:
+// its 128 rows of X and its 128 rows of W, both K-major.  X is read again by
+// every vocabulary tile (keep it in L2); W streams through once.
+__device__ __forceinline__ void load_stage_pass1(const CUtensorMap* mX, const CUtensorMap* mW, uint32_t sA,
+                                                 uint32_t sB, uint32_t bar, int mb, int nb, int kb, int rank,
+                                                 uint64_t keep, uint64_t stream) {
   const int k0 = kb * BK;
-  const int m0 = mb * CM + rank * BM;
-  const int n0 = nb * BN + rank * BNH;
-  if constexpr (KIND == KIND_LSE || KIND == KIND_GRAD) {
-    tma_load_2d_pair(sA, mA, bar, k0, m0);               // X rows, K-major
-    tma_load_2d_pair(sB, mB, bar, k0, a.vbase + n0);     // W rows, K-major
-  } else if constexpr (KIND == KIND_DW) {
-#pragma unroll
-    for (int i = 0; i < BM / 64; ++i)                    // G_c^T: vocab contiguous
-      tma_load_2d_pair(sA + i * MN_BOX_BYTES, mA, bar, m0 + i * 64, k0);
-#pragma unroll
-    for (int i = 0; i < BNH / 64; ++i)                   // X: hidden contiguous
-      tma_load_2d_pair(sB + i * MN_BOX_BYTES, mB, bar, n0 + i * 64, k0);
-  } else {
-    tma_load_2d_pair(sA, mA, bar, k0, m0);               // G_c rows, K-major
-#pragma unroll
-    for (int i = 0; i < BNH / 64; ++i)                   // W_c: hidden contiguous
-      tma_load_2d_pair(sB + i * MN_BOX_BYTES, mB, bar, n0 + i * 64, a.vbase + k0);
-  }
+  tma_load_2d_pair(sA, mX, bar, k0, mb * CM + rank * BM, keep);
+  tma_load_2d_pair(sB, mW, bar, k0, nb * BN + rank * BNH, stream);
 }
 
 template <bool MN>
@@ -250,7 +217,7 @@ __device__ __forceinline__ void put_row32(uint8_t* box, int r, const float (&v)[
 // with fill(v) for this thread's row, then one lane ships the box.
 template <class Fill>
 __device__ __forceinline__ void stage_and_store(EpiStage& es, int lane, const CUtensorMap* map, int x, int y,
-                                                Fill fill) {
+                                                uint64_t policy, Fill fill) {
   const uint32_t b = es.k & 1u;
   if (lane == 0) bulk_wait_read<1>();
   __syncwarp();
@@ -260,7 +227,7 @@ __device__ __forceinline__ void stage_and_store(EpiStage& es, int lane, const CU
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    tma_store_2d(map, es.addr + b * EPI_BUF_BYTES, x, y);
+    tma_store_2d(map, es.addr + b * EPI_BUF_BYTES, x, y, policy);
     bulk_commit();
   }
   ++es.k;
@@ -284,7 +251,7 @@ __device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, int vbase, uint
     tmem_ld_wait();
     const int colg0 = vbase + nb * BN + c * 32;
     const int lim = a.V - colg0;
-    stage_and_store(es, lane, mapG, nb * BN + c * 32, wrow0, [&](float (&g)[32]) {
+    stage_and_store(es, lane, mapG, nb * BN + c * 32, wrow0, l2_evict_normal(), [&](float (&g)[32]) {
 #pragma unroll
       for (int t = 0; t < 32; ++t)
         g[t] = (valid && t < lim) ? ex2_approx(fmaf(__uint_as_float(r[t]), LOG2E, -l2)) * scale : 0.f;
@@ -308,7 +275,7 @@ __device__ __forceinline__ void epi_dw_tile(int vbase, uint32_t taddr, int row0,
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
-    stage_and_store(es, lane, mapDW, nb * BN + c * 32, wrow0, [&](float (&v)[32]) {
+    stage_and_store(es, lane, mapDW, nb * BN + c * 32, wrow0, l2_evict_first(), [&](float (&v)[32]) {
 #pragma unroll
       for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
     });
@@ -327,13 +294,14 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk,
   const int wrow0 = row0 + (row_local & ~31);
   const bool accumulate = !first_chunk;
   constexpr int SLICES = BN / 32;
+  const uint64_t stream = l2_evict_first();  // the running sum is touched once per chunk
   auto fetch = [&](uint32_t b, int c) {  // lane 0: hi and lo boxes of slice c into buffer b
     bulk_wait_read<0>();                 // the buffer's previous store has read it
     fence_proxy_async_smem();
     const uint32_t bar = es.bar + 8u * b;
     mbar_arrive_expect_tx(bar, 2 * EPI_BOX_BYTES);
-    tma_load_2d(es.addr + b * EPI_BUF_BYTES, mapHi, bar, nb * BN + c * 32, wrow0);
-    tma_load_2d(es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, mapLo, bar, nb * BN + c * 32, wrow0);
+    tma_load_2d(es.addr + b * EPI_BUF_BYTES, mapHi, bar, nb * BN + c * 32, wrow0, stream);
+    tma_load_2d(es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, mapLo, bar, nb * BN + c * 32, wrow0, stream);
   };
   if (accumulate && lane == 0) fetch(es.k & 1u, 0);
 #pragma unroll 1
@@ -387,8 +355,9 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk,
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(mapHi, es.addr + b * EPI_BUF_BYTES, nb * BN + c * 32, wrow0);
-      if (!last_chunk) tma_store_2d(mapLo, es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, nb * BN + c * 32, wrow0);
+      tma_store_2d(mapHi, es.addr + b * EPI_BUF_BYTES, nb * BN + c * 32, wrow0, stream);
+      if (!last_chunk)
+        tma_store_2d(mapLo, es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, nb * BN + c * 32, wrow0, stream);
       bulk_commit();
     }
     ++es.k;
@@ -397,13 +366,12 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk,
 
 // ------------------------------------------------------------ the kernel --
 
-template <int KIND>
+// Pass 1: z = X W^T tile by tile; each epilogue thread folds its row's logits
+// into a running (max, sum of exponentials) over the vocabulary split of the
+// unit, and picks out the target logit.  No logit leaves the chip.
 __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1)
-    flce_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                     const __grid_constant__ CUtensorMap mapHi, const __grid_constant__ CUtensorMap mapLo,
-                     const __grid_constant__ CUtensorMap mapOut, const __grid_constant__ CUtensorMap mapOutLo,
-                     const GemmArgs a) {
-  using T = KindTraits<KIND>;
+    flce_pass1_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
+                      const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   // Same dynamic-smem base in both CTAs, so every offset below matches across the pair.
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -444,9 +412,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&mapA);
-    prefetch_tmap(&mapB);
-    prefetch_tmap(&mapOut);
+    prefetch_tmap(&mapX);
+    prefetch_tmap(&mapW);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
@@ -465,21 +432,14 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
+      const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
-        unit_range<KIND>(a, u, mb, nb0, nb1, split);
+        unit_range(a, u, mb, nb0, nb1, split);
         for (int nb = nb0; ok && nb < nb1; ++nb) {
-          if constexpr (KIND == KIND_DX) {
-            // the epilogue of this tile reads back the running dX sum: pull this
-            // CTA's rows into L2 now, a whole mainloop ahead of the read
-            if (!a.first_chunk) {
-              tma_prefetch_l2_2d(&mapHi, nb * BN, mb * CM + rank * BM);
-              tma_prefetch_l2_2d(&mapLo, nb * BN, mb * CM + rank * BM);
-            }
-          }
           for (int kb = 0; kb < a.k_blocks; ++kb) {
             if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
               give_up();
@@ -487,8 +447,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
               break;
             }
             if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * STAGE_BYTES);
-            load_stage<KIND>(a, &mapA, &mapB, sA(stage), sB(stage), mapa_shared(full_bar(stage), 0), mb, nb,
-                             kb, rank);
+            load_stage_pass1(&mapX, &mapW, sA(stage), sB(stage), mapa_shared(full_bar(stage), 0), mb, nb, kb,
+                             rank, keep, stream);
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -517,7 +477,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   } else if (warp == 1) {
     // ------------------------------------------------ UMMA issuer (leader) --
     if (leader && lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(CM, BN, T::A_MN, T::B_MN);
+      constexpr uint32_t IDESC = idesc_bf16_f32(CM, BN, false, false);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -525,7 +485,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       bool ok = true;
       for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
-        unit_range<KIND>(a, u, mb, nb0, nb1, split);
+        unit_range(a, u, mb, nb0, nb1, split);
         for (int nb = nb0; ok && nb < nb1; ++nb) {
           if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
             give_up();
@@ -543,8 +503,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k)
-              umma_bf16_pair(d_tmem, operand_desc<T::A_MN>(sA(stage), k), operand_desc<T::B_MN>(sB(stage), k),
-                             IDESC, (kb | k) != 0);
+              umma_bf16_pair(d_tmem, operand_desc<false>(sA(stage), k), operand_desc<false>(sB(stage), k), IDESC,
+                             (kb | k) != 0);
             umma_commit_pair(empty_bar(stage), 0x3);
             if (++stage == STAGES) {
               stage = 0;
@@ -575,27 +535,19 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
     const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
-    EpiStage es;
-    es.ptr = epi_ptr + q * EPI_WARP_BYTES;
-    es.addr = smem_u32(es.ptr);
-    es.bar = smem_u32(bars + 2 * STAGES + 5 + 2 * q);
-    es.k = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int u = cid; ok && u < a.num_units; u += ncl) {
       int mb, nb0, nb1, split;
-      unit_range<KIND>(a, u, mb, nb0, nb1, split);
-      const int row0 = mb * CM + rank * BM;
+      unit_range(a, u, mb, nb0, nb1, split);
       LseState st;
-      if constexpr (KIND == KIND_LSE) {
-        st.row = row0 + row_local;
-        st.yr = st.row < a.N ? a.y[st.row] : a.ignore_index;
-        st.run_m = -1e30f;
-        st.run_l = 0.f;
-        st.zy_val = 0.f;
-        st.has_zy = false;
-      }
+      st.row = mb * CM + rank * BM + row_local;
+      st.yr = st.row < a.N ? a.y[st.row] : a.ignore_index;
+      st.run_m = -1e30f;
+      st.run_l = 0.f;
+      st.zy_val = 0.f;
+      st.has_zy = false;
       for (int nb = nb0; nb < nb1; ++nb) {
         const bool got = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.timeout_ns);
         if (!__all_sync(0xffffffffu, got)) {
@@ -605,32 +557,19 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
-        if constexpr (KIND == KIND_LSE) epi_lse_tile(a, taddr, nb, st);
-        if constexpr (KIND == KIND_GRAD) epi_grad_tile(a, a.vbase, taddr, row0, nb, row_local, es, &mapOut);
-        if constexpr (KIND == KIND_DW) epi_dw_tile(a.vbase, taddr, row0, nb, row_local, es, &mapOut);
-        if constexpr (KIND == KIND_DX) {
-          epi_dx_tile(a, a.first_chunk, a.last_chunk, taddr, row0, nb, row_local, es, &mapOut, &mapOutLo,
-                      abort_flag, ok);
-          if (!ok) {
-            give_up();
-            break;
-          }
-        }
+        epi_lse_tile(a, taddr, nb, st);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      if constexpr (KIND == KIND_LSE) {
-        if (ok && st.row < a.N) {
-          a.part_m[static_cast<size_t>(split) * a.N + st.row] = st.run_m;
-          a.part_l[static_cast<size_t>(split) * a.N + st.row] = st.run_l;
-          if (st.has_zy) a.zy[st.row] = st.zy_val;
-        }
+      if (ok && st.row < a.N) {
+        a.part_m[static_cast<size_t>(split) * a.N + st.row] = st.run_m;
+        a.part_l[static_cast<size_t>(split) * a.N + st.row] = st.run_l;
+        if (st.has_zy) a.zy[st.row] = st.zy_val;
       }
     }
-    if (lane == 0) bulk_wait<0>();  // every staged box written out before the CTA winds down
   }
 
   // Wind-down: this CTA's work is done; tell the peer, wait (bounded) for the
@@ -661,7 +600,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
 //
 //   G(0)  |  dX(0) dW(0) G(1)  |  dX(1) dW(1) G(2)  | ... |  dX(C-1) dW(C-1)
 //
-// where G(c) are the logit-recompute tiles of chunk c (column-major), dX(c) the
+// where G(c) are the logit-recompute tiles of chunk c (row by row, so that a
+// token tile's G rows are complete early for its dX tiles), dX(c) the
 // dX += G_c W_c tiles and dW(c) the dW rows of chunk c.  There is one G buffer,
 // so items wait for what they read and for the readers of what they overwrite:
 //   dX(c) mainloop  after G(c) of its token tile (all its columns),
@@ -691,10 +631,11 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
   Item it;
   const long long g0 = static_cast<long long>(chunk_vtiles(p, 0)) * p.TM;
   if (i < g0) {
+    const int vt = chunk_vtiles(p, 0);
     it.kind = ITEM_GRAD;
     it.c = 0;
-    it.b = static_cast<int>(i / p.TM);
-    it.a = static_cast<int>(i - static_cast<long long>(it.b) * p.TM);
+    it.a = static_cast<int>(i / vt);
+    it.b = static_cast<int>(i - static_cast<long long>(it.a) * vt);
     return it;
   }
   // sections 0 .. C-3 all have the size of section 0; the last two may be shorter
@@ -723,10 +664,11 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
     it.b = static_cast<int>(r - static_cast<long long>(it.a) * p.HN);
   } else {
     r -= nx + nw;
+    const int vt = chunk_vtiles(p, c + 1);
     it.kind = ITEM_GRAD;
     it.c = c + 1;
-    it.b = static_cast<int>(r / p.TM);
-    it.a = static_cast<int>(r - static_cast<long long>(it.b) * p.TM);
+    it.a = static_cast<int>(r / vt);
+    it.b = static_cast<int>(r - static_cast<long long>(it.a) * vt);
   }
   return it;
 }
@@ -811,6 +753,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
+      const uint64_t keep = l2_evict_last(), normal = l2_evict_normal(), stream = l2_evict_first();
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -830,8 +773,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
           // pull this CTA's rows of the running sum into L2 if they are final already
           if (ok && it.c > 0 && ld_acquire_gpu(a.x_row + it.a) >= SIGNALS_PER_ITEM * it.c * a.HN) {
             fence_proxy_async_global();
-            tma_prefetch_l2_2d(&m.Hipf, it.b * BN, it.a * CM + rank * BM);
-            tma_prefetch_l2_2d(&m.Lopf, it.b * BN, it.a * CM + rank * BM);
+            tma_prefetch_l2_2d(&m.Hipf, it.b * BN, it.a * CM + rank * BM, stream);
+            tma_prefetch_l2_2d(&m.Lopf, it.b * BN, it.a * CM + rank * BM, stream);
           }
         }
         if (!ok) {
@@ -851,19 +794,20 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
           const uint32_t bar = mapa_shared(full_bar(stage), 0);
           const int k0 = kb * BK;
           if (it.kind == ITEM_GRAD) {
-            tma_load_2d_pair(sA(stage), &m.Xk, bar, k0, m0);
-            tma_load_2d_pair(sB(stage), &m.Wk, bar, k0, vbase + n0);
+            tma_load_2d_pair(sA(stage), &m.Xk, bar, k0, m0, keep);
+            tma_load_2d_pair(sB(stage), &m.Wk, bar, k0, vbase + n0, normal);
           } else if (it.kind == ITEM_DW) {
 #pragma unroll
-            for (int i = 0; i < BM / 64; ++i) tma_load_2d_pair(sA(stage) + i * MN_BOX_BYTES, &m.Gmn, bar, m0 + i * 64, k0);
+            for (int i = 0; i < BM / 64; ++i)
+              tma_load_2d_pair(sA(stage) + i * MN_BOX_BYTES, &m.Gmn, bar, m0 + i * 64, k0, normal);
 #pragma unroll
             for (int i = 0; i < BNH / 64; ++i)
-              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, &m.Xmn, bar, n0 + i * 64, k0);
+              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, &m.Xmn, bar, n0 + i * 64, k0, keep);
           } else {
-            tma_load_2d_pair(sA(stage), &m.Gk, bar, k0, m0);
+            tma_load_2d_pair(sA(stage), &m.Gk, bar, k0, m0, normal);
 #pragma unroll
             for (int i = 0; i < BNH / 64; ++i)
-              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, &m.Wmn, bar, n0 + i * 64, vbase + k0);
+              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, &m.Wmn, bar, n0 + i * 64, vbase + k0, normal);
           }
           if (++stage == STAGES) {
             stage = 0;
