@@ -102,7 +102,7 @@ cudaError_t set_kernel_attrs(int dev) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_attr_set[dev]) return cudaSuccess;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(flce_pass1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+  if ((e = cudaFuncSetAttribute(flce_pass1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P1_SMEM_BYTES)) !=
       cudaSuccess)
     return e;
   if ((e = cudaFuncSetAttribute(flce_pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
@@ -121,7 +121,9 @@ cudaError_t set_kernel_attrs(int dev) {
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int clusters = 0, clusters2 = 0;
+  cfg.dynamicSmemBytes = P1_SMEM_BYTES;
   if ((e = cudaOccupancyMaxActiveClusters(&clusters, flce_pass1_kernel, &cfg)) != cudaSuccess) return e;
+  cfg.dynamicSmemBytes = SMEM_BYTES;
   if ((e = cudaOccupancyMaxActiveClusters(&clusters2, flce_pass2_kernel, &cfg)) != cudaSuccess) return e;
   clusters = std::min(clusters, clusters2);
   if (clusters <= 0) return cudaErrorInvalidConfiguration;
@@ -327,7 +329,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     p1.num_units = P.tiles_m * P.splits;
     size_t slot;
     prof_begin(stream, KIND_LSE, &slot);
-    flce_pass1_kernel<<<CLUSTER * P.lse_clusters, NUM_THREADS, SMEM_BYTES, stream>>>(mX_k, mW_k, p1);
+    flce_pass1_kernel<<<CLUSTER * P.lse_clusters, NUM_THREADS, P1_SMEM_BYTES, stream>>>(mX_k, mW_k, p1);
     prof_end(stream, slot);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }

@@ -66,6 +66,10 @@ constexpr int EPI_WARP_BYTES = 2 * EPI_BUF_BYTES;
 constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP_BYTES;
 constexpr int NUM_BARRIERS = 2 * STAGES + 4 + 1 + 2 * EPI_WARPS;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
+// Pass 1 stages nothing through shared memory in its epilogue and needs no
+// staging area (a seventh stage measured no faster).
+constexpr int P1_STAGES = STAGES;
+constexpr int P1_SMEM_BYTES = P1_STAGES * STAGE_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr double LN2 = 0.6931471805599453;
 
@@ -377,9 +381,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;  // swizzle atoms need 1024-B alignment
   uint8_t* base_ptr = smem_raw + (base - raw_addr);
-  uint8_t* epi_ptr = base_ptr + STAGES * STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_ptr + EPI_BYTES);
-  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin, epi[EPI_WARPS][2]
+  constexpr int STAGES = P1_STAGES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + STAGES * STAGE_BYTES);
+  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -407,7 +411,6 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       mbar_init(tempty_bar(b), CLUSTER * EPI_WARPS);  // leader: epilogue warps of both CTAs
     }
     mbar_init(fin_bar, 1);  // the peer's end-of-work signal
-    for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(smem_u32(bars + 2 * STAGES + 5 + e), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -600,8 +603,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
 //
 //   G(0)  |  dX(0) dW(0) G(1)  |  dX(1) dW(1) G(2)  | ... |  dX(C-1) dW(C-1)
 //
-// where G(c) are the logit-recompute tiles of chunk c (row by row, so that a
-// token tile's G rows are complete early for its dX tiles), dX(c) the
+// where G(c) are the logit-recompute tiles of chunk c (column-major), dX(c) the
 // dX += G_c W_c tiles and dW(c) the dW rows of chunk c.  There is one G buffer,
 // so items wait for what they read and for the readers of what they overwrite:
 //   dX(c) mainloop  after G(c) of its token tile (all its columns),
@@ -631,11 +633,10 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
   Item it;
   const long long g0 = static_cast<long long>(chunk_vtiles(p, 0)) * p.TM;
   if (i < g0) {
-    const int vt = chunk_vtiles(p, 0);
     it.kind = ITEM_GRAD;
     it.c = 0;
-    it.a = static_cast<int>(i / vt);
-    it.b = static_cast<int>(i - static_cast<long long>(it.a) * vt);
+    it.b = static_cast<int>(i / p.TM);
+    it.a = static_cast<int>(i - static_cast<long long>(it.b) * p.TM);
     return it;
   }
   // sections 0 .. C-3 all have the size of section 0; the last two may be shorter
@@ -664,11 +665,10 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
     it.b = static_cast<int>(r - static_cast<long long>(it.a) * p.HN);
   } else {
     r -= nx + nw;
-    const int vt = chunk_vtiles(p, c + 1);
     it.kind = ITEM_GRAD;
     it.c = c + 1;
-    it.a = static_cast<int>(r / vt);
-    it.b = static_cast<int>(r - static_cast<long long>(it.a) * vt);
+    it.b = static_cast<int>(r / p.TM);
+    it.a = static_cast<int>(r - static_cast<long long>(it.b) * p.TM);
   }
   return it;
 }
