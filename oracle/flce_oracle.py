@@ -36,6 +36,13 @@ Readings where the pages are silent: the mean runs over non-ignored rows; with
 no valid row the loss, dX and dW are all zero (PyTorch would give NaN); there is
 no bias, label smoothing, soft-cap or z-loss term.
 
+Reductions.  A drop-in replacement of the unfused head (same call signature)
+also offers PyTorch's other reductions; the oracle writes all three as one
+weighted sum over valid rows, ``loss = sum_valid s_i l_i`` with
+``s_i = 1/n`` ('mean'), ``1`` ('sum') or the caller's per-row upstream gradient
+``g_i`` ('none', default 1), and ``G_ij = s_i (exp(z_ij - lse_i) - [j == y_i])``
+for valid rows, so that dX and dW are the gradients of that loss.
+
 Inputs are converted exactly to fp64 (bf16 -> fp64 is exact).  A matrix product
 (numpy/BLAS in fp64) serves as a step; nothing is blocked, fused or reordered
 beyond what the definition states, except that the functions meant for full-size
@@ -84,8 +91,24 @@ def log_sum_exp(Z: np.ndarray) -> np.ndarray:
     return m + np.log(np.exp(Z - m[:, None]).sum(axis=1))
 
 
-def flce_reference(X, W, y, ignore_index: int = IGNORE_INDEX):
-    """The whole definition on full matrices: returns (loss, dX, dW, lse, n).
+def row_scale(valid: np.ndarray, reduction: str, grad_row_scale=None) -> np.ndarray:
+    """Weight s_i of each row's loss in the reduced loss (0 for ignored rows)."""
+    n = int(valid.sum())
+    if reduction == "mean":
+        s = np.full(valid.shape, (1.0 / n) if n else 0.0)
+    elif reduction == "sum":
+        s = np.ones(valid.shape)
+    elif reduction == "none":
+        s = np.ones(valid.shape) if grad_row_scale is None else _f64(grad_row_scale)
+    else:
+        raise ValueError(f"unknown reduction {reduction!r}")
+    return np.where(valid, s, 0.0)
+
+
+def flce_reference(X, W, y, ignore_index: int = IGNORE_INDEX, reduction: str = "mean", grad_row_scale=None,
+                   return_rows: bool = False):
+    """The whole definition on full matrices: returns (loss, dX, dW, lse, n),
+    plus the per-row losses when ``return_rows``.
 
     For shapes whose N x V fp64 logits fit in host memory.
     """
@@ -98,18 +121,20 @@ def flce_reference(X, W, y, ignore_index: int = IGNORE_INDEX):
     n = int(valid.sum())
     rows = np.arange(N)
     yv = np.where(valid, y, 0)
+    s = row_scale(valid, reduction, grad_row_scale)
 
     Z = X @ W.T                                   # z_ij = x_i . w_j
     lse = log_sum_exp(Z)
     row_loss = np.where(valid, lse - Z[rows, yv], 0.0)
-    loss = float(row_loss.sum() / n) if n else 0.0
+    loss = float((s * row_loss).sum())           # mean: (sum of valid l_i) / n
 
     G = np.exp(Z - lse[:, None])                  # softmax
     G[rows, yv] -= 1.0                            # minus the one-hot target
-    G *= valid[:, None]                           # ignored rows give nothing
-    G *= (1.0 / n) if n else 0.0                  # token mean
+    G *= s[:, None]                               # s_i: token mean (or sum / upstream weights); 0 on ignored rows
     dX = G @ W
     dW = G.T @ X
+    if return_rows:
+        return loss, dX, dW, lse, n, row_loss
     return loss, dX, dW, lse, n
 
 

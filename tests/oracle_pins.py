@@ -242,9 +242,32 @@ def pin_row_functions(orc):
     _close(orc.row_lse(X, W, rows), lse[rows], 1e-14, what="row_lse subset")
 
 
+def pin_reductions(orc):
+    """'sum' is n times 'mean' (loss and both gradients); 'none' with per-row
+    upstream weights g equals torch autograd of sum_i g_i * CE_i (reduction
+    'none'), and its row losses equal torch's per-row cross-entropy."""
+    X, W, y = _case(90, 13, 9, 21, n_ign=3)
+    n = int((y != IGN).sum())
+    lm, dXm, dWm, _, _ = orc.flce_reference(X, W, y, reduction="mean")
+    ls, dXs, dWs, _, _ = orc.flce_reference(X, W, y, reduction="sum")
+    assert abs(ls - n * lm) <= 1e-13 * abs(ls)
+    _close(dXs, n * dXm, 1e-13, what="sum vs mean dX")
+    _close(dWs, n * dWm, 1e-13, what="sum vs mean dW")
+    g = _rng(91).standard_normal(13)
+    ln, dXn, dWn, _, _, rows = orc.flce_reference(X, W, y, reduction="none", grad_row_scale=g, return_rows=True)
+    tX = torch.tensor(X, dtype=torch.float64, requires_grad=True)
+    tW = torch.tensor(W, dtype=torch.float64, requires_grad=True)
+    per_row = torch.nn.functional.cross_entropy(tX @ tW.T, torch.tensor(y), ignore_index=IGN, reduction="none")
+    (per_row * torch.tensor(g)).sum().backward()
+    _close(rows, per_row.detach().numpy(), 1e-12, what="row losses vs torch")
+    assert abs(ln - float((per_row.detach() * torch.tensor(g)).sum())) <= 1e-12 * max(1.0, abs(ln))
+    _close(dXn, tX.grad.numpy(), 1e-11, what="weighted dX vs autograd")
+    _close(dWn, tW.grad.numpy(), 1e-11, what="weighted dW vs autograd")
+
+
 ALL_PINS = [
     pin_zero_weight, pin_zero_input, pin_two_class, pin_large_logits,
     pin_torch_autograd, pin_finite_difference, pin_rows_of_g_sum_to_zero,
     pin_shift_invariance, pin_ignored_rows, pin_no_valid_rows, pin_target_range,
-    pin_permutations, pin_equal_logits, pin_row_functions,
+    pin_permutations, pin_equal_logits, pin_row_functions, pin_reductions,
 ]

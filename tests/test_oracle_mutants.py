@@ -13,10 +13,11 @@ from oracle import flce_oracle
 # (description, original text, mutated text); each original must occur in the source.
 MUTATIONS = [
     ("one-hot added instead of subtracted", "G[rows, yv] -= 1.0", "G[rows, yv] += 1.0"),
-    ("ignored rows not masked in G", "G *= valid[:, None]                           # ignored rows",
-     "G *= 1.0                                      # ignored rows"),
-    ("mean over all rows, not valid rows", "G *= (1.0 / n) if n else 0.0                  # token mean",
-     "G *= (1.0 / N) if n else 0.0                  # token mean"),
+    ("ignored rows not masked in G", "    return np.where(valid, s, 0.0)", "    return s"),
+    ("mean over all rows, not valid rows", 's = np.full(valid.shape, (1.0 / n) if n else 0.0)',
+     's = np.full(valid.shape, (1.0 / valid.size) if n else 0.0)'),
+    ("per-row upstream weights ignored", "G *= s[:, None]                               # s_i",
+     "G *= s[:, None] ** 0 * s[0]                   # s_i"),
     ("softmax not normalised", "G = np.exp(Z - lse[:, None])                  # softmax",
      "G = np.exp(Z)                                 # softmax"),
     ("max dropped from log-sum-exp", "return m + np.log(np.exp(Z - m[:, None]).sum(axis=1))",
