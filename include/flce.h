@@ -116,6 +116,35 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
                                          void* workspace, size_t workspace_bytes,
                                          cudaStream_t stream);
 
+/* Reductions of flce_forward_backward_ex.  All three are one weighted sum over
+ * the non-ignored rows, loss = sum_i s_i l_i with l_i = lse_i - z_{i,y_i}, and
+ * dX, dW are the gradients of that loss (G_ij = s_i (softmax_ij - [j == y_i])):
+ *   MEAN  s_i = 1/n_valid (the default of the other entry points)
+ *   SUM   s_i = 1
+ *   NONE  s_i = grad_row_scale[i], the caller's upstream gradient of row i's
+ *         loss (1 when grad_row_scale is NULL); the per-row losses themselves
+ *         come back in row_loss.
+ * These are PyTorch's cross_entropy reductions, which a drop-in replacement of
+ * the unfused head ("Liger-Kernel: Triton kernels that replace HF training
+ * ops", section "What actually gets replaced") has to offer; per-row weights
+ * and log-probabilities are also what a fused-linear preference loss builds on. */
+typedef enum { FLCE_REDUCTION_MEAN = 0, FLCE_REDUCTION_SUM = 1, FLCE_REDUCTION_NONE = 2 } flce_reduction_t;
+
+/* Asynchronous entry with every option.
+ *   reduction:      flce_reduction_t
+ *   grad_row_scale: DEVICE float[N] or NULL (used by NONE only)
+ *   d_loss:         DEVICE float, receives sum_i s_i l_i
+ *   d_row_loss:     DEVICE float[N] or NULL: l_i for valid rows, 0 for ignored rows
+ *   d_status:       DEVICE int32, 0 or a device-side flce_status_t
+ *   dX, dW:         device outputs; both NULL = forward only (loss and row
+ *                   losses, no gradient pass); exactly one NULL is an error
+ * Other arguments as flce_forward_backward_async. */
+flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N,
+                                       int64_t H, int64_t V, int32_t ignore_index, int32_t reduction,
+                                       const float* grad_row_scale, float* d_loss, float* d_row_loss,
+                                       int32_t* d_status, uint16_t* dX, uint16_t* dW, void* workspace,
+                                       size_t workspace_bytes, cudaStream_t stream);
+
 /* Allocation-free variant of flce_forward_backward, for callers that cannot
  * allocate device memory: a plug-in or custom operator that is handed only the
  * tensors it works on and has no allocator to ask for scratch, and processes

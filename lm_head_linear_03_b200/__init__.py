@@ -10,6 +10,7 @@ from .flce import (  # noqa: F401
     alloc_workspace,
     forward_backward,
     forward_backward_async,
+    forward_backward_ex,
     forward_backward_host,
     load_library,
     plan,

@@ -247,11 +247,14 @@ flce_status_t check_sizes(int64_t N, int64_t H, int64_t V) {
   return FLCE_OK;
 }
 
+// dX and dW may both be NULL only when `forward_only_ok` (no gradient pass).
 flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N, int64_t H, int64_t V,
-                         const void* dX, const void* dW, const void* ws) {
+                         const void* dX, const void* dW, const void* ws, bool forward_only_ok = false) {
   const flce_status_t s = check_sizes(N, H, V);
   if (s != FLCE_OK) return s;
-  if (!X || !W || !y || !dX || !dW || !ws) return FLCE_ERR_INVALID_ARGUMENT;
+  if (!X || !W || !y || !ws) return FLCE_ERR_INVALID_ARGUMENT;
+  const bool no_grads = !dX && !dW;
+  if ((!dX || !dW) && !(no_grads && forward_only_ok)) return FLCE_ERR_INVALID_ARGUMENT;
   if (!aligned(X, 16) || !aligned(W, 16) || !aligned(dX, 16) || !aligned(dW, 16) || !aligned(y, 4) ||
       !aligned(ws, 256))
     return FLCE_ERR_UNSUPPORTED;
@@ -259,9 +262,15 @@ flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N,
 }
 
 // --------------------------------------------------------------- enqueue --
+struct Options {
+  int reduction = RED_MEAN;
+  const float* grad_row_scale = nullptr;
+  float* row_loss = nullptr;
+};
+
 flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
                       int32_t ignore_index, float* d_loss, int32_t* d_status, uint16_t* dX, uint16_t* dW,
-                      void* workspace, cudaStream_t stream) {
+                      void* workspace, cudaStream_t stream, const Options& opt = Options()) {
   DevInfo di;
   int dev;
   if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
@@ -286,13 +295,14 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BNH) &&
             make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
             make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK) &&
-            make_map(&mHi, dX, h, n, h * 2, BN, BM, Swz::none) && make_map(&mLo, lo, h, n, h * 2, BN, BM, Swz::none);
+            (dX == nullptr || (make_map(&mHi, dX, h, n, h * 2, BN, BM, Swz::none) &&
+                               make_map(&mLo, lo, h, n, h * 2, BN, BM, Swz::none)));
   // 32 x 32 output boxes of the epilogues (64-byte swizzle)
   CUtensorMap mGo, mDWo, mHio, mLoo;
-  ok = ok && make_map(&mGo, G, VC, n, VC * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
-       make_map(&mDWo, dW, h, v, h * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
-       make_map(&mHio, dX, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
-       make_map(&mLoo, lo, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64);
+  ok = ok && (dX == nullptr || (make_map(&mGo, G, VC, n, VC * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
+                                make_map(&mDWo, dW, h, v, h * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
+                                make_map(&mHio, dX, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
+                                make_map(&mLoo, lo, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64)));
   if (!ok) return FLCE_ERR_CUDA;
 
   // control words and pass-2 counters start at zero (they are contiguous)
@@ -318,6 +328,8 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   a.lo = lo;
   a.status = d_status;
   a.timeout_ns = DEFAULT_TIMEOUT_NS;
+  a.reduction = opt.reduction;
+  a.grad_row_scale = opt.grad_row_scale;
 
   // Pass 1: logits tile by tile, online log-sum-exp per (row, split).
   {
@@ -352,6 +364,9 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     c.inv_n = &ctrl->inv_n;
     c.loss = d_loss;
     c.status = d_status;
+    c.reduction = opt.reduction;
+    c.grad_row_scale = opt.grad_row_scale;
+    c.row_loss = opt.row_loss;
     const int grid = static_cast<int>((N + COMBINE_THREADS - 1) / COMBINE_THREADS);
     size_t slot;
     prof_begin(stream, KIND_COMBINE, &slot);
@@ -359,8 +374,9 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     prof_end(stream, slot);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
-  // Pass 2: every chunk's logit recompute, dW and dX tiles in one persistent launch.
-  {
+  // Pass 2: every chunk's logit recompute, dW and dX tiles in one persistent launch
+  // (skipped for a forward-only call).
+  if (dX != nullptr) {
     GemmArgs b = a;
     b.TM = P.tiles_m;
     b.HN = static_cast<int>((H + BN - 1) / BN);
@@ -454,6 +470,26 @@ flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, 
   if (!aligned(d_status, 4) || !aligned(d_loss, 4)) return FLCE_ERR_UNSUPPORTED;
   if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, stream);
+}
+
+flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H,
+                                       int64_t V, int32_t ignore_index, int32_t reduction,
+                                       const float* grad_row_scale, float* d_loss, float* d_row_loss,
+                                       int32_t* d_status, uint16_t* dX, uint16_t* dW, void* workspace,
+                                       size_t workspace_bytes, cudaStream_t stream) {
+  if (!d_loss || !d_status) return FLCE_ERR_INVALID_ARGUMENT;
+  if (reduction != FLCE_REDUCTION_MEAN && reduction != FLCE_REDUCTION_SUM && reduction != FLCE_REDUCTION_NONE)
+    return FLCE_ERR_INVALID_ARGUMENT;
+  const flce_status_t s = check_args(X, W, y, N, H, V, dX, dW, workspace, true);
+  if (s != FLCE_OK) return s;
+  if (!aligned(d_status, 4) || !aligned(d_loss, 4) || !aligned(d_row_loss, 4) || !aligned(grad_row_scale, 4))
+    return FLCE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  Options opt;
+  opt.reduction = reduction;
+  opt.grad_row_scale = reduction == FLCE_REDUCTION_NONE ? grad_row_scale : nullptr;
+  opt.row_loss = d_row_loss;
+  return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, stream, opt);
 }
 
 flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_W, const int32_t* h_y, int64_t N,

@@ -73,6 +73,17 @@ constexpr int P1_SMEM_BYTES = P1_STAGES * STAGE_BYTES + 1024 /*alignment*/ + 256
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr double LN2 = 0.6931471805599453;
 
+// Reductions: the loss is sum_i s_i l_i over valid rows with s_i = 1/n, 1, or
+// the caller's per-row upstream gradient.
+enum : int { RED_MEAN = 0, RED_SUM = 1, RED_NONE = 2 };
+
+// Per-row weight s_i of a valid row (the reduction's scale of its loss and of its G row).
+__device__ __forceinline__ float row_weight(int reduction, const float* inv_n, const float* grad_row_scale, int row) {
+  if (reduction == RED_MEAN) return *inv_n;
+  if (reduction == RED_SUM) return 1.f;
+  return grad_row_scale ? grad_row_scale[row] : 1.f;
+}
+
 // Kinds of launch, as the profiler reports them.
 enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2 };
 enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
@@ -96,6 +107,8 @@ struct GemmArgs {
   uint16_t* lo;           // [N][H] bf16, low half of the dX accumulator
   int* status;
   unsigned long long timeout_ns;
+  int reduction;                 // RED_MEAN, RED_SUM, RED_NONE
+  const float* grad_row_scale;   // RED_NONE: per-row upstream gradient, or null for 1
   // pass 2 (one persistent launch over every chunk)
   int TM, HN;             // 256-row token tiles, 256-column hidden tiles
   int C;                  // vocabulary chunks
@@ -246,7 +259,7 @@ __device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, int vbase, uint
   const int yr = in_rows ? a.y[row] : a.ignore_index;
   const bool valid = in_rows && yr != a.ignore_index;
   const float l2 = valid ? a.lse2[row] : 0.f;
-  const float scale = valid ? *a.inv_n : 0.f;
+  const float scale = valid ? row_weight(a.reduction, a.inv_n, a.grad_row_scale, row) : 0.f;
   const int wrow0 = row0 + (row_local & ~31);
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
@@ -989,6 +1002,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
 
 struct CombineArgs {
   int N, V, ignore_index, splits;
+  int reduction;
+  const float* grad_row_scale;
+  float* row_loss;  // optional per-row losses
   const int32_t* y;
   const float* part_m;
   const float* part_l;
@@ -1022,14 +1038,18 @@ __global__ void __launch_bounds__(COMBINE_THREADS) flce_combine_kernel(const Com
     const float l2 = M + log2f(L);
     a.lse2[i] = l2;
     const int yi = a.y[i];
+    double row = 0.0;
     if (yi != a.ignore_index) {
       if (yi < 0 || yi >= a.V) {
         raise_status(a.status, ST_TARGET_OUT_OF_RANGE);
       } else {
-        li = static_cast<double>(l2) * LN2 - static_cast<double>(a.zy[i]);
+        row = static_cast<double>(l2) * LN2 - static_cast<double>(a.zy[i]);
         vi = 1;
+        // mean and sum add the plain row losses (the mean divides at the end)
+        li = a.reduction == RED_NONE && a.grad_row_scale ? row * static_cast<double>(a.grad_row_scale[i]) : row;
       }
     }
+    if (a.row_loss) a.row_loss[i] = static_cast<float>(row);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -1069,7 +1089,10 @@ __global__ void __launch_bounds__(COMBINE_THREADS) flce_combine_kernel(const Com
     }
     *a.n_valid = static_cast<int>(cnt);
     *a.inv_n = cnt ? static_cast<float>(1.0 / static_cast<double>(cnt)) : 0.f;
-    *a.loss = cnt ? static_cast<float>(tot / static_cast<double>(cnt)) : 0.f;
+    if (a.reduction == RED_MEAN)
+      *a.loss = cnt ? static_cast<float>(tot / static_cast<double>(cnt)) : 0.f;
+    else
+      *a.loss = static_cast<float>(tot);
     *a.ticket = 0u;
   }
 }

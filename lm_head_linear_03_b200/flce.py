@@ -38,7 +38,9 @@ EXPORTED = (
     "flce_profile_enable",
     "flce_profile_read",
     "flce_forward_backward_noalloc",
+    "flce_forward_backward_ex",
 )
+REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -91,6 +93,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_profile_enable.restype = ctypes.c_int
     lib.flce_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)]
     lib.flce_profile_read.restype = ctypes.c_int
+    lib.flce_forward_backward_ex.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.flce_forward_backward_ex.restype = ctypes.c_int
     lib.flce_forward_backward_noalloc.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp, vp]
     lib.flce_forward_backward_noalloc.restype = ctypes.c_int
     _lib = lib
@@ -176,6 +180,36 @@ def forward_backward_async(X, W, y, ignore_index: int = -100, *, out=None, works
                                          workspace.numel(), _stream_handle(stream))
     _check(st, "flce_forward_backward_async")
     return loss, status, dX, dW
+
+
+def forward_backward_ex(X, W, y, ignore_index: int = -100, *, reduction: str = "mean", grad_row_scale=None,
+                        row_loss: bool = False, grads: bool = True, workspace=None, stream=None):
+    """Asynchronous call with every option; returns device tensors
+    (loss[1], status[1], row_loss[N] or None, dX or None, dW or None).
+
+    reduction 'mean' | 'sum' | 'none'; grad_row_scale: fp32[N] upstream
+    gradient of each row's loss for 'none'; grads=False skips the gradient pass.
+    """
+    lib = load_library()
+    _check_inputs(X, W, y)
+    N, H = X.shape
+    V = W.shape[0]
+    dev = X.device
+    if grad_row_scale is not None and (grad_row_scale.dtype != torch.float32 or not grad_row_scale.is_cuda
+                                       or grad_row_scale.shape != (N,) or not grad_row_scale.is_contiguous()):
+        raise ValueError("grad_row_scale must be a contiguous CUDA float32 tensor of shape [N]")
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    rl = torch.empty(N, dtype=torch.float32, device=dev) if row_loss else None
+    dX = torch.empty_like(X) if grads else None
+    dW = torch.empty_like(W) if grads else None
+    workspace = alloc_workspace(N, H, V, dev) if workspace is None else workspace
+    vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
+    st = lib.flce_forward_backward_ex(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, REDUCTIONS[reduction],
+                                      vp(grad_row_scale), _ptr(loss), vp(rl), _ptr(status), vp(dX), vp(dW),
+                                      _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(st, "flce_forward_backward_ex")
+    return loss, status, rl, dX, dW
 
 
 def forward_backward_host(hX, hW, hy, dev_bufs, ignore_index: int = -100, *, h_out=None, stream=None):

@@ -210,3 +210,53 @@ def test_peak_device_bytes_equal_buffers_plus_workspace():
     F.forward_backward(X, W, y, dX=dX, dW=dW, workspace=ws)
     torch.cuda.synchronize()
     assert torch.cuda.max_memory_allocated() == base
+
+
+def _ex_case(w, **kw):
+    F = _lib()
+    X, W, y = make_inputs(w)
+    loss, status, rl, dX, dW = F.forward_backward_ex(X.cuda(), W.cuda(), y.cuda(), **kw)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return X, W, y, loss.item(), rl, dX, dW
+
+
+def test_reduction_sum():
+    w = custom("red_sum", N=300, H=136, V=5000, ignore_frac=0.1)
+    X, W, y, loss, rl, dX, dW = _ex_case(w, reduction="sum", row_loss=True)
+    ref, rdX, rdW, _, _, rows = O.flce_reference(X, W, y, reduction="sum", return_rows=True)
+    assert_loss_close(loss, ref)
+    assert_grad_close(_np(dX), rdX, "dX sum")
+    assert_grad_close(_np(dW), rdW, "dW sum")
+    r = rl.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(r - rows)) <= LOSS_RTOL * np.max(np.abs(rows))
+
+
+def test_reduction_none_with_upstream_weights():
+    """Per-row upstream gradients of both signs, the fused-linear core a
+    preference loss builds on (weighted per-token log-probabilities)."""
+    w = custom("red_none", N=520, H=264, V=6208, ignore_frac=0.05)
+    g = torch.randn(520, generator=torch.Generator().manual_seed(5)).float()
+    X, W, y, loss, rl, dX, dW = _ex_case(w, reduction="none", grad_row_scale=g.cuda(), row_loss=True)
+    ref, rdX, rdW, _, _, rows = O.flce_reference(X, W, y, reduction="none", grad_row_scale=g.double().numpy(),
+                                                 return_rows=True)
+    assert abs(loss - ref) <= LOSS_RTOL * float(np.sum(np.abs(g.double().numpy() * rows)))
+    assert_grad_close(_np(dX), rdX, "dX none")
+    assert_grad_close(_np(dW), rdW, "dW none")
+    r = rl.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(r - rows)) <= LOSS_RTOL * np.max(np.abs(rows))
+    assert np.all(r[y.numpy() == -100] == 0.0)
+
+
+def test_forward_only_matches_full_call():
+    F = _lib()
+    w = custom("fwd_only", N=384, H=256, V=4500, ignore_frac=0.1)
+    X, W, y = (t.cuda() for t in make_inputs(w))
+    full, _, _ = F.forward_backward(X, W, y)
+    loss, status, rl, dX, dW = F.forward_backward_ex(X, W, y, grads=False, row_loss=True)
+    torch.cuda.synchronize()
+    assert status.item() == 0 and dX is None and dW is None
+    assert loss.item() == full
+    ref, _, _, _, _, rows = O.flce_reference(X, W, y, return_rows=True)
+    r = rl.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(r - rows)) <= LOSS_RTOL * np.max(np.abs(rows))
