@@ -188,8 +188,9 @@ flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out);
  * returns, per kernel kind, the number of launches and their summed device
  * time in milliseconds, then clears the record.  kinds: 0 pass-1 GEMM +
  * online log-sum-exp, 1 combine, 2 pass 2 (logit recompute + G, dW and dX
- * contractions of every vocabulary chunk, one persistent launch). */
-#define FLCE_NUM_KERNEL_KINDS 3
+ * contractions of every vocabulary chunk, one persistent launch), 3 prep
+ * (valid rows per 256-row token tile). */
+#define FLCE_NUM_KERNEL_KINDS 4
 const char* flce_kernel_name(int kind);
 flce_status_t flce_profile_enable(int on);
 flce_status_t flce_profile_read(int32_t* launches, double* total_ms);

@@ -27,7 +27,7 @@ constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per bou
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t ctrl, counters, counters_bytes, lse2, zy, part_m, part_l, blk_loss, blk_cnt, G, lo, total;
+  size_t ctrl, counters, counters_bytes, tile_valid, lse2, zy, part_m, part_l, blk_loss, blk_cnt, G, lo, total;
 };
 
 // ctrl block: [0] status, [4] ticket, [8] n_valid, [12] inv_n, [16] loss
@@ -54,6 +54,7 @@ WsLayout ws_layout(int64_t N, int64_t H) {
   const size_t tm = (n + CM - 1) / CM;
   L.counters_bytes = (2 * tm + 2 * (VC / BN)) * 4;
   L.counters = take(L.counters_bytes);
+  L.tile_valid = take(tm * 4);
   L.lse2 = take(n * 4);
   L.zy = take(n * 4);
   L.part_m = take(static_cast<size_t>(MAX_SPLITS) * n * 4);
@@ -212,7 +213,7 @@ Plan make_plan(int64_t N, int64_t H, int64_t V, int clusters) {
   p.lse_clusters =
       static_cast<int>(std::min<long long>(static_cast<long long>(p.tiles_m) * p.splits, clusters));
   p.num_chunks = static_cast<int>((V + VC - 1) / VC);
-  p.launches = 3;  // pass 1, combine, pass 2
+  p.launches = 4;  // prep, pass 1, combine, pass 2
   return p;
 }
 
@@ -330,6 +331,17 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   a.timeout_ns = DEFAULT_TIMEOUT_NS;
   a.reduction = opt.reduction;
   a.grad_row_scale = opt.grad_row_scale;
+  a.tile_valid = reinterpret_cast<const int*>(ws + L.tile_valid);
+
+  // Valid rows per 256-row token tile.
+  {
+    size_t slot;
+    prof_begin(stream, KIND_PREP, &slot);
+    flce_prep_kernel<<<P.tiles_m, CM, 0, stream>>>(y, static_cast<int>(N), ignore_index,
+                                                   reinterpret_cast<int*>(ws + L.tile_valid));
+    prof_end(stream, slot);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  }
 
   // Pass 1: logits tile by tile, online log-sum-exp per (row, split).
   {
@@ -549,6 +561,7 @@ const char* flce_kernel_name(int kind) {
     case KIND_LSE: return "pass1_logits_lse";
     case KIND_COMBINE: return "combine_lse_loss";
     case KIND_PASS2: return "pass2_grad_dw_dx";
+    case KIND_PREP: return "prep_tile_valid";
     default: return "unknown";
   }
 }

@@ -85,7 +85,7 @@ __device__ __forceinline__ float row_weight(int reduction, const float* inv_n, c
 }
 
 // Kinds of launch, as the profiler reports them.
-enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2 };
+enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_PREP = 3 };
 enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
 
 struct GemmArgs {
@@ -109,6 +109,7 @@ struct GemmArgs {
   unsigned long long timeout_ns;
   int reduction;                 // RED_MEAN, RED_SUM, RED_NONE
   const float* grad_row_scale;   // RED_NONE: per-row upstream gradient, or null for 1
+  const int* tile_valid;         // [ceil(N/256)] valid rows per 256-row token tile (prep kernel)
   // pass 2 (one persistent launch over every chunk)
   int TM, HN;             // 256-row token tiles, 256-column hidden tiles
   int C;                  // vocabulary chunks
@@ -299,6 +300,23 @@ __device__ __forceinline__ void epi_dw_tile(int vbase, uint32_t taddr, int row0,
   }
 }
 
+// Writes a tile of zeros (rows row0.., columns nb*BN..) without reading the
+// accumulator: outputs of rows that are all ignored, or a contraction with
+// no k-block left.
+__device__ __forceinline__ void epi_zero_tile(uint32_t taddr, int row0, int nb, int row_local, EpiStage& es,
+                                              const CUtensorMap* map) {
+  (void)taddr;
+  const int lane = row_local & 31;
+  const int wrow0 = row0 + (row_local & ~31);
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    stage_and_store(es, lane, map, nb * BN + c * 32, wrow0, l2_evict_first(), [&](float (&v)[32]) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) v[t] = 0.f;
+    });
+  }
+}
+
 // dX += G_c W_c.  The running sum lives in two bf16 words, hi (in dX itself) and
 // lo (workspace), with value = hi + lo: about 16 significant bits, enough for an
 // fp32-grade sum over the chunks, at the memory cost of one bf16 copy of dX.
@@ -455,6 +473,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
         unit_range(a, u, mb, nb0, nb1, split);
+        if (a.tile_valid[mb] == 0) continue;  // every row of the tile is ignored
         for (int nb = nb0; ok && nb < nb1; ++nb) {
           for (int kb = 0; kb < a.k_blocks; ++kb) {
             if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
@@ -502,6 +521,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
         unit_range(a, u, mb, nb0, nb1, split);
+        if (a.tile_valid[mb] == 0) continue;  // every row of the tile is ignored
         for (int nb = nb0; ok && nb < nb1; ++nb) {
           if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
             give_up();
@@ -557,6 +577,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     for (int u = cid; ok && u < a.num_units; u += ncl) {
       int mb, nb0, nb1, split;
       unit_range(a, u, mb, nb0, nb1, split);
+      if (a.tile_valid[mb] == 0) continue;  // every row of the tile is ignored
       LseState st;
       st.row = mb * CM + rank * BM + row_local;
       st.yr = st.row < a.N ? a.y[st.row] : a.ignore_index;
@@ -774,8 +795,12 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         const Item it = decode_item(a, u);
         const int vbase = it.c * a.Vc;
         const int vcount = min(a.Vc, a.V - vbase);
+        // G and dX tiles of a token tile whose rows are all ignored are skipped
+        const bool skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
         int kblocks;
-        if (it.kind == ITEM_GRAD) {
+        if (skip) {
+          kblocks = 0;
+        } else if (it.kind == ITEM_GRAD) {
           kblocks = (a.H + BK - 1) / BK;
         } else if (it.kind == ITEM_DW) {
           kblocks = (a.N + BK - 1) / BK;
@@ -798,6 +823,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         const int m0 = it.a * CM + rank * BM;
         const int n0 = it.b * BN + rank * BNH;
         for (int kb = 0; kb < kblocks; ++kb) {
+          // dW: K runs over tokens; k-blocks of all-ignored token tiles add nothing
+          if (it.kind == ITEM_DW && a.tile_valid[kb / (CM / BK)] == 0) continue;
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
             give_up();
             ok = false;
@@ -858,9 +885,11 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       for (long long u = cid; ok && u < a.total_items; u += ncl) {
         const Item it = decode_item(a, u);
         const int vcount = min(a.Vc, a.V - it.c * a.Vc);
-        const int kblocks = it.kind == ITEM_GRAD ? (a.H + BK - 1) / BK
-                            : it.kind == ITEM_DW ? (a.N + BK - 1) / BK
-                                                 : (vcount + BK - 1) / BK;
+        const bool skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
+        const int kblocks = skip                  ? 0
+                            : it.kind == ITEM_GRAD ? (a.H + BK - 1) / BK
+                            : it.kind == ITEM_DW   ? (a.N + BK - 1) / BK
+                                                   : (vcount + BK - 1) / BK;
         const uint32_t idesc = it.kind == ITEM_GRAD ? ID_GRAD : it.kind == ITEM_DW ? ID_DW : ID_DX;
         const bool a_mn = it.kind == ITEM_DW;
         const bool b_mn = it.kind != ITEM_GRAD;
@@ -870,7 +899,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        uint32_t accumulate = 0;
         for (int kb = 0; kb < kblocks; ++kb) {
+          if (it.kind == ITEM_DW && a.tile_valid[kb / (CM / BK)] == 0) continue;
           if (!mbar_wait(full_bar(stage), phase, abort_flag, a.timeout_ns)) {
             give_up();
             ok = false;
@@ -881,7 +912,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
           for (int k = 0; k < BK / UMMA_K; ++k) {
             const uint64_t ad = a_mn ? operand_desc<true>(sA(stage), k) : operand_desc<false>(sA(stage), k);
             const uint64_t bd = b_mn ? operand_desc<true>(sB(stage), k) : operand_desc<false>(sB(stage), k);
-            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, accumulate);
+            accumulate = 1;
           }
           umma_commit_pair(empty_bar(stage), 0x3);
           if (++stage == STAGES) {
@@ -915,6 +947,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     es.addr = smem_u32(es.ptr);
     es.bar = smem_u32(bars + 2 * STAGES + 5 + 2 * q);
     es.k = 0;
+    // with every token ignored the dW contraction has no k-block at all
+    bool any_valid = false;
+    for (int t = 0; t < a.TM && !any_valid; ++t) any_valid = a.tile_valid[t] != 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -945,10 +980,18 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
-      if (it.kind == ITEM_GRAD) {
+      const bool skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
+      if (skip) {
+        // all rows ignored: nothing reads this tile's G rows; its dX rows are
+        // zero, written once by the first chunk
+        if (it.kind == ITEM_DX && it.c == 0) epi_zero_tile(taddr, row0, it.b, row_local, es, &m.Hio);
+      } else if (it.kind == ITEM_GRAD) {
         epi_grad_tile(a, vbase, taddr, row0, it.b, row_local, es, &m.Go);
       } else if (it.kind == ITEM_DW) {
-        epi_dw_tile(vbase, taddr, row0, it.b, row_local, es, &m.DWo);
+        if (any_valid)
+          epi_dw_tile(vbase, taddr, row0, it.b, row_local, es, &m.DWo);
+        else
+          epi_zero_tile(taddr, vbase + row0, it.b, row_local, es, &m.DWo);
       } else {
         epi_dx_tile(a, it.c == 0, it.c == a.C - 1, taddr, row0, it.b, row_local, es, &m.Hio, &m.Loo, abort_flag,
                     ok);
@@ -996,6 +1039,17 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
+}
+
+// ---------------------------------------------------------------- prep --
+
+// Valid (non-ignored) rows of each 256-row token tile, so that pass 1 and
+// pass 2 can skip tiles whose rows are all ignored (a prompt mask).
+__global__ void __launch_bounds__(CM) flce_prep_kernel(const int32_t* y, int N, int ignore_index, int* tile_valid) {
+  const int r = blockIdx.x * CM + threadIdx.x;
+  const int v = (r < N && y[r] != ignore_index) ? 1 : 0;
+  const int cnt = __syncthreads_count(v);
+  if (threadIdx.x == 0) tile_valid[blockIdx.x] = cnt;
 }
 
 // ------------------------------------------------------------ combine --

@@ -25,7 +25,7 @@ STATUS_NAMES = {
     5: "FLCE_ERR_TIMEOUT",
     6: "FLCE_ERR_CUDA",
 }
-NUM_KERNEL_KINDS = 3
+NUM_KERNEL_KINDS = 4
 
 EXPORTED = (
     "flce_status_string",

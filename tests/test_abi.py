@@ -66,7 +66,7 @@ def test_plan_is_host_only(lib):
     p = flce.plan(8192, 4096, 128256)
     assert p.vocab_chunk == 2048 and p.num_chunks == 63
     assert 1 <= p.lse_splits <= 64
-    assert p.launches == 3
+    assert p.launches == 4
 
 
 def test_argument_errors_before_any_launch(lib):

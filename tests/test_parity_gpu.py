@@ -260,3 +260,18 @@ def test_forward_only_matches_full_call():
     ref, _, _, _, _, rows = O.flce_reference(X, W, y, return_rows=True)
     r = rl.cpu().numpy().astype(np.float64)
     assert np.max(np.abs(r - rows)) <= LOSS_RTOL * np.max(np.abs(rows))
+
+
+@pytest.mark.parametrize("N,H,V,ignored", [
+    (1100, 136, 5000, slice(0, 600)),      # prompt mask covering two whole 256-row tiles
+    (1024, 264, 6208, slice(256, 512)),    # one whole tile in the middle
+    (768, 64, 2500, slice(0, 768)),        # every tile (all rows ignored)
+])
+def test_whole_ignored_token_tiles_are_skipped(N, H, V, ignored):
+    """Tiles whose rows are all ignored skip pass 1, the G and dX tiles and their
+    k-blocks of dW; results stay equal to the oracle's."""
+    w = custom(f"skip_{N}_{H}_{V}", N=N, H=H, V=V, ignore_frac=0.05)
+    X, W, y = make_inputs(w)
+    y[ignored] = -100
+    loss, dX, dW = run_full_oracle_case(X, W, y)
+    assert torch.count_nonzero(dX[ignored]).item() == 0
