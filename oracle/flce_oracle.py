@@ -19,6 +19,8 @@ cross-entropy" pipeline, only without keeping the logit tensor:
 * "Complete Guide to Liger Kernel", section LigerFusedLinearCrossEntropyLoss:
   ``loss = fused_loss_fn(hidden_states, weight, labels)`` with ``weight`` of
   shape ``(vocab_size, hidden_size)``.
+* The same guide, section LigerCrossEntropyLoss: cross-entropy computed from a
+  given ``(batch*seq, vocab)`` logit tensor and labels (:func:`ce_reference`).
 
 The oracle therefore *does* materialise the logits (that is the plain
 definition) and follows these steps, with ``n`` the number of non-ignored rows:
@@ -207,3 +209,29 @@ def dw_rows(X, W, y, vocab_rows, lse, n: int, ignore_index: int = IGNORE_INDEX, 
     G *= valid[:, None]
     G *= (1.0 / n) if n else 0.0
     return G.T @ X64
+
+
+# ---------------------------------------------------------------------------
+# Cross-entropy on given logits (no linear layer).
+# ---------------------------------------------------------------------------
+
+def ce_reference(Z, y, ignore_index: int = IGNORE_INDEX, reduction: str = "mean", grad_row_scale=None):
+    """Steps 1-4 on a given logit matrix Z[N,V]: returns (loss, dZ, lse, n, row_loss).
+
+    dZ = G is the gradient of the reduced loss with respect to the logits.
+    """
+    Z = _f64(Z)
+    y = _i64(y)
+    N, V = Z.shape
+    valid = valid_mask(y, V, ignore_index)
+    n = int(valid.sum())
+    rows = np.arange(N)
+    yv = np.where(valid, y, 0)
+    s = row_scale(valid, reduction, grad_row_scale)
+    lse = log_sum_exp(Z)
+    row_loss = np.where(valid, lse - Z[rows, yv], 0.0)
+    loss = float((s * row_loss).sum())
+    G = np.exp(Z - lse[:, None])
+    G[rows, yv] -= 1.0
+    G *= s[:, None]
+    return loss, G, lse, n, row_loss

@@ -265,9 +265,37 @@ def pin_reductions(orc):
     _close(dWn, tW.grad.numpy(), 1e-11, what="weighted dW vs autograd")
 
 
+def pin_ce_on_logits(orc):
+    """Cross-entropy on given logits: torch's cross_entropy + autograd on the
+    same fp64 logits for all three reductions, and the fused head's loss and
+    dX = G W, dW = G^T X when the logits are X W^T."""
+    r = _rng(100)
+    Z = r.standard_normal((17, 40)) * 3.0
+    y = r.integers(0, 40, size=17)
+    y[[2, 9]] = IGN
+    g = r.standard_normal(17)
+    for red, w in (("mean", None), ("sum", None), ("none", g)):
+        loss, dZ, lse, n, rows = orc.ce_reference(Z, y, reduction=red, grad_row_scale=w)
+        tZ = torch.tensor(Z, requires_grad=True)
+        per = torch.nn.functional.cross_entropy(tZ, torch.tensor(y), ignore_index=IGN, reduction="none")
+        scale = {"mean": torch.full((17,), 1.0 / n, dtype=torch.float64), "sum": torch.ones(17, dtype=torch.float64),
+                 "none": torch.tensor(g)}[red]
+        tl = (per * scale).sum()
+        tl.backward()
+        assert abs(loss - tl.item()) <= 1e-12 * max(1.0, abs(tl.item())), (red, loss, tl.item())
+        _close(dZ, tZ.grad.numpy(), 1e-12, atol=1e-16, what=f"dZ {red}")
+        _close(rows, per.detach().numpy(), 1e-12, what=f"row losses {red}")
+    X, W, yy = _case(101, 9, 6, 15, n_ign=2)
+    l1, dX, dW, _, _ = orc.flce_reference(X, W, yy)
+    l2, G, _, _, _ = orc.ce_reference(X @ W.T, yy)
+    assert abs(l1 - l2) <= 1e-13 * abs(l1)
+    _close(G @ W, dX, 1e-12, atol=1e-16, what="G W vs fused dX")
+    _close(G.T @ X, dW, 1e-12, atol=1e-16, what="G^T X vs fused dW")
+
+
 ALL_PINS = [
     pin_zero_weight, pin_zero_input, pin_two_class, pin_large_logits,
     pin_torch_autograd, pin_finite_difference, pin_rows_of_g_sum_to_zero,
     pin_shift_invariance, pin_ignored_rows, pin_no_valid_rows, pin_target_range,
-    pin_permutations, pin_equal_logits, pin_row_functions, pin_reductions,
+    pin_permutations, pin_equal_logits, pin_row_functions, pin_reductions, pin_ce_on_logits,
 ]

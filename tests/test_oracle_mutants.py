@@ -12,7 +12,8 @@ from oracle import flce_oracle
 
 # (description, original text, mutated text); each original must occur in the source.
 MUTATIONS = [
-    ("one-hot added instead of subtracted", "G[rows, yv] -= 1.0", "G[rows, yv] += 1.0"),
+    ("one-hot added instead of subtracted", "G[rows, yv] -= 1.0                            # minus the one-hot",
+     "G[rows, yv] += 1.0                            # minus the one-hot"),
     ("ignored rows not masked in G", "    return np.where(valid, s, 0.0)", "    return s"),
     ("mean over all rows, not valid rows", 's = np.full(valid.shape, (1.0 / n) if n else 0.0)',
      's = np.full(valid.shape, (1.0 / valid.size) if n else 0.0)'),
@@ -22,8 +23,9 @@ MUTATIONS = [
      "G = np.exp(Z)                                 # softmax"),
     ("max dropped from log-sum-exp", "return m + np.log(np.exp(Z - m[:, None]).sum(axis=1))",
      "return np.log(np.exp(Z - m[:, None]).sum(axis=1))"),
-    ("target logit added to the row loss", "row_loss = np.where(valid, lse - Z[rows, yv], 0.0)",
-     "row_loss = np.where(valid, lse + Z[rows, yv], 0.0)"),
+    ("target logit added to the row loss",
+     "row_loss = np.where(valid, lse - Z[rows, yv], 0.0)\n    loss = float((s * row_loss).sum())           # mean",
+     "row_loss = np.where(valid, lse + Z[rows, yv], 0.0)\n    loss = float((s * row_loss).sum())           # mean"),
     ("dW from X transposed against G", "dW = G.T @ X", "dW = (X.T @ G).T * 0 + G.T @ (X * 0.5)"),
     ("dX against the wrong operand", "dX = G @ W", "dX = G @ (W - W.mean(axis=0)) * 0.5"),
     ("full-size loss drops the target logit", "row_loss = np.where(valid, lse - zy, 0.0)",
@@ -31,6 +33,10 @@ MUTATIONS = [
     ("full-size dW one-hot sign", "G -= (y[:, None] == J[None, :])", "G += (y[:, None] == J[None, :])"),
     ("full-size dX ignores the valid mask", "    G *= valid[:, None]\n    G *= (1.0 / n) if n else 0.0\n    return G @ W64",
      "    G *= (1.0 / n) if n else 0.0\n    return G @ W64"),
+    ("logit CE: one-hot sign", "    G[rows, yv] -= 1.0\n    G *= s[:, None]\n    return loss, G, lse, n, row_loss",
+     "    G[rows, yv] += 1.0\n    G *= s[:, None]\n    return loss, G, lse, n, row_loss"),
+    ("logit CE: row loss without the target logit", "    row_loss = np.where(valid, lse - Z[rows, yv], 0.0)\n    loss = float((s * row_loss).sum())\n    G = np.exp(Z - lse[:, None])\n    G[rows, yv] -= 1.0\n    G *= s[:, None]\n    return loss, G",
+     "    row_loss = np.where(valid, lse, 0.0)\n    loss = float((s * row_loss).sum())\n    G = np.exp(Z - lse[:, None])\n    G[rows, yv] -= 1.0\n    G *= s[:, None]\n    return loss, G"),
     ("target range not checked", "bad = valid & ((y < 0) | (y >= V))", "bad = valid & (y < -10**9)"),
 ]
 
