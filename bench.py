@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--op", choices=["flce", "ce"], default="flce",
+                    help="flce: the fused head (default); ce: cross-entropy on given logits of the same workload")
     return ap.parse_args()
 
 
@@ -415,12 +417,79 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_ce(args, world, rank, local):
+    """Cross-entropy on a given [N, V] bf16 logit tensor of the workload's shape
+    (z ~ N(0, 0.02 * sqrt(H)), the spread of X W^T): memory bound, so the
+    roofline is HBM bytes (read the logits, write their gradient) per second."""
+    import lm_head_linear_03_b200 as F
+    from lm_head_linear_03_b200.inputs import make_targets
+    F.load_library()
+    w = workload(args)
+    dev = torch.device("cuda", local)
+    N, V = w.N, w.V
+    gen = torch.Generator(device=dev).manual_seed(w.seed)
+    Z = (torch.randn(N, V, generator=gen, device=dev) * (w.w_std * w.H ** 0.5)).to(torch.bfloat16)
+    y = make_targets(w, torch.Generator().manual_seed(w.seed)).to(dev)
+    dz = torch.empty_like(Z)
+    ws = torch.empty(int(F.load_library().flce_ce_workspace_size(N, V)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    lib = F.load_library()
+    from lm_head_linear_03_b200 import flce as B
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    st = torch.empty(1, dtype=torch.int32, device=dev)
+
+    def step():
+        r = lib.flce_cross_entropy(B._ptr(Z), B._ptr(y), N, V, -100, 0, None, B._ptr(loss), None, B._ptr(st),
+                                   B._ptr(dz), B._ptr(ws), ws.numel(), B._stream_handle(stream))
+        assert r == 0
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    F.profile_enable(True)
+    for _ in range(args.steps):
+        step()
+    prof = F.profile_read()
+    F.profile_enable(False)
+    n_rows, rows_ms = prof["ce_on_logits_rows"]
+    if rank != 0:
+        return
+    pk, pk_src = peaks()
+    algo = 2.0 * N * V * 2  # read the logits once, write the gradient once
+    achieved = algo / (rows_ms / n_rows * 1e-3) / 1e9
+    line = {
+        "metric": "cross-entropy on given logits fwd+bwd tokens/s (HBM-bound)", "value": world * N / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}_logits", "N": N, "V": V,
+                   "l2": f"logits {N * V * 2 / 1e9:.2f} GB > 126 MB L2; no flush"},
+        "roofline": {"kernel": "ce_on_logits_rows", "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{pk_src} hbm_gbs", "algorithmic_bytes_per_launch": algo},
+        "gpu_launches": 3 * args.steps, "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.op == "ce":
+            run_ce(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -145,6 +145,22 @@ flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, con
                                        int32_t* d_status, uint16_t* dX, uint16_t* dW, void* workspace,
                                        size_t workspace_bytes, cudaStream_t stream);
 
+/* Cross-entropy on a logit tensor the caller already holds, the unfused
+ * counterpart of the head ("Complete Guide to Liger Kernel", section
+ * LigerCrossEntropyLoss): the same loss, reductions and row losses as
+ * flce_forward_backward_ex, with z given instead of X W^T.
+ *   logits:  DEVICE bf16 [N][V], row-major
+ *   dlogits: DEVICE bf16 [N][V] receiving d loss / d logits, or NULL for a
+ *            forward-only call; may be the same pointer as logits (in place)
+ *   workspace: DEVICE, >= flce_ce_workspace_size(N, V) bytes (depends on N only),
+ *            256-byte aligned
+ * Asynchronous; d_loss, d_row_loss, d_status as in flce_forward_backward_ex. */
+size_t flce_ce_workspace_size(int64_t N, int64_t V);
+flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64_t N, int64_t V,
+                                 int32_t ignore_index, int32_t reduction, const float* grad_row_scale,
+                                 float* d_loss, float* d_row_loss, int32_t* d_status, uint16_t* dlogits,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Allocation-free variant of flce_forward_backward, for callers that cannot
  * allocate device memory: a plug-in or custom operator that is handed only the
  * tensors it works on and has no allocator to ask for scratch, and processes
@@ -189,8 +205,9 @@ flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out);
  * time in milliseconds, then clears the record.  kinds: 0 pass-1 GEMM +
  * online log-sum-exp, 1 combine, 2 pass 2 (logit recompute + G, dW and dX
  * contractions of every vocabulary chunk, one persistent launch), 3 prep
- * (valid rows per 256-row token tile). */
-#define FLCE_NUM_KERNEL_KINDS 4
+ * (valid rows per 256-row token tile), 4 cross-entropy on given logits (rows
+ * pass; its final sum is counted under kind 1). */
+#define FLCE_NUM_KERNEL_KINDS 5
 const char* flce_kernel_name(int kind);
 flce_status_t flce_profile_enable(int on);
 flce_status_t flce_profile_read(int32_t* launches, double* total_ms);

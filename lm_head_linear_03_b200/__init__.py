@@ -8,6 +8,7 @@ ABI is declared in ``include/flce.h``; ``flce.py`` is its ctypes binding.
 from .flce import (  # noqa: F401
     FlceError,
     alloc_workspace,
+    cross_entropy,
     forward_backward,
     forward_backward_async,
     forward_backward_ex,

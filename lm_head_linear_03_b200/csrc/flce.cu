@@ -67,6 +67,27 @@ WsLayout ws_layout(int64_t N, int64_t H) {
   return L;
 }
 
+// Workspace of the cross-entropy-on-logits entry: depends on N only.
+struct CeLayout {
+  size_t ctrl, tile_valid, row_acc, blk_sum, total;
+};
+CeLayout ce_ws_layout(int64_t N) {
+  CeLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t n = static_cast<size_t>(N);
+  L.ctrl = take(256);
+  L.tile_valid = take(((n + CM - 1) / CM) * 4);
+  L.row_acc = take(n * 8);
+  L.blk_sum = take(((n + COMBINE_THREADS - 1) / COMBINE_THREADS) * 8);
+  L.total = off;
+  return L;
+}
+
 // ------------------------------------------------------------ device info --
 struct DevInfo {
   bool ok = false;
@@ -504,6 +525,67 @@ flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, con
   return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, stream, opt);
 }
 
+size_t flce_ce_workspace_size(int64_t N, int64_t V) {
+  if (N <= 0 || V <= 0 || N > (1ll << 30) || V > (1ll << 30)) return 0;
+  return ce_ws_layout(N).total;
+}
+
+flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64_t N, int64_t V,
+                                 int32_t ignore_index, int32_t reduction, const float* grad_row_scale,
+                                 float* d_loss, float* d_row_loss, int32_t* d_status, uint16_t* dlogits,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (N <= 0 || V <= 0 || N > (1ll << 30) || V > (1ll << 30)) return FLCE_ERR_INVALID_ARGUMENT;
+  if (!logits || !y || !d_loss || !d_status || !workspace) return FLCE_ERR_INVALID_ARGUMENT;
+  if (reduction != FLCE_REDUCTION_MEAN && reduction != FLCE_REDUCTION_SUM && reduction != FLCE_REDUCTION_NONE)
+    return FLCE_ERR_INVALID_ARGUMENT;
+  if (!aligned(logits, 2) || !aligned(dlogits, 2) || !aligned(y, 4) || !aligned(workspace, 256) ||
+      !aligned(d_loss, 4) || !aligned(d_status, 4) || !aligned(d_row_loss, 4) || !aligned(grad_row_scale, 4))
+    return FLCE_ERR_UNSUPPORTED;
+  const CeLayout L = ce_ws_layout(N);
+  if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  DevInfo di;
+  int dev;
+  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int TM = static_cast<int>((N + CM - 1) / CM);
+  if (cudaMemsetAsync(ws + L.ctrl, 0, 256, stream) != cudaSuccess ||
+      cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  CeArgs c{};
+  c.logits = logits;
+  c.dlogits = dlogits;
+  c.y = y;
+  c.N = static_cast<int>(N);
+  c.V = static_cast<int>(V);
+  c.ignore_index = ignore_index;
+  c.reduction = reduction;
+  c.TM = TM;
+  c.grad_row_scale = reduction == FLCE_REDUCTION_NONE ? grad_row_scale : nullptr;
+  c.tile_valid = reinterpret_cast<const int*>(ws + L.tile_valid);
+  c.row_acc = reinterpret_cast<double*>(ws + L.row_acc);
+  c.row_loss = d_row_loss;
+  c.blk_sum = reinterpret_cast<double*>(ws + L.blk_sum);
+  c.ticket = reinterpret_cast<unsigned int*>(ws + L.ctrl + 4);
+  c.loss = d_loss;
+  c.status = d_status;
+  size_t slot;
+  prof_begin(stream, KIND_PREP, &slot);
+  flce_prep_kernel<<<TM, CM, 0, stream>>>(y, c.N, ignore_index, reinterpret_cast<int*>(ws + L.tile_valid));
+  prof_end(stream, slot);
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<int64_t>(N, static_cast<int64_t>(di.num_sms) * 4 * 64));
+  prof_begin(stream, KIND_CE, &slot);
+  flce_ce_rows_kernel<<<grid, CE_THREADS, 0, stream>>>(c);
+  prof_end(stream, slot);
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  prof_begin(stream, KIND_COMBINE, &slot);
+  flce_ce_reduce_kernel<<<static_cast<int>((N + COMBINE_THREADS - 1) / COMBINE_THREADS), COMBINE_THREADS, 0, stream>>>(c);
+  prof_end(stream, slot);
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  return FLCE_OK;
+}
+
 flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_W, const int32_t* h_y, int64_t N,
                                          int64_t H, int64_t V, int32_t ignore_index, float* h_loss, uint16_t* h_dX,
                                          uint16_t* h_dW, uint16_t* d_X, uint16_t* d_W, int32_t* d_y,
@@ -562,6 +644,7 @@ const char* flce_kernel_name(int kind) {
     case KIND_COMBINE: return "combine_lse_loss";
     case KIND_PASS2: return "pass2_grad_dw_dx";
     case KIND_PREP: return "prep_tile_valid";
+    case KIND_CE: return "ce_on_logits_rows";
     default: return "unknown";
   }
 }

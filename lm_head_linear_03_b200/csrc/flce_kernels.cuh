@@ -85,7 +85,7 @@ __device__ __forceinline__ float row_weight(int reduction, const float* inv_n, c
 }
 
 // Kinds of launch, as the profiler reports them.
-enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_PREP = 3 };
+enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_PREP = 3, KIND_CE = 4 };
 enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
 
 struct GemmArgs {
@@ -1145,6 +1145,223 @@ __global__ void __launch_bounds__(COMBINE_THREADS) flce_combine_kernel(const Com
     *a.inv_n = cnt ? static_cast<float>(1.0 / static_cast<double>(cnt)) : 0.f;
     if (a.reduction == RED_MEAN)
       *a.loss = cnt ? static_cast<float>(tot / static_cast<double>(cnt)) : 0.f;
+    else
+      *a.loss = static_cast<float>(tot);
+    *a.ticket = 0u;
+  }
+}
+
+// ======================================== cross-entropy on given logits ==
+//
+// The same loss and gradient from a logit tensor the caller already holds
+// ("Complete Guide to Liger Kernel", section LigerCrossEntropyLoss).  Memory
+// bound: one CTA per row reads the row once for its online (max, sum) and once
+// more (an L2 hit while the row is in flight) to write the bf16 gradient,
+// in place if the caller wishes.
+
+constexpr int CE_THREADS = 512;
+constexpr int CE_UNROLL = 4;  // 16-byte loads in flight per thread
+
+struct CeArgs {
+  const uint16_t* logits;  // [N][V] bf16
+  uint16_t* dlogits;       // [N][V] bf16 or null (forward only); may equal logits
+  const int32_t* y;
+  int N, V, ignore_index, reduction, TM;
+  const float* grad_row_scale;
+  const int* tile_valid;   // [TM] valid rows per 256-row tile (prep kernel)
+  double* row_acc;         // [N] weighted row losses for the deterministic sum
+  float* row_loss;         // [N] or null
+  double* blk_sum;         // [ceil(N / COMBINE_THREADS)]
+  unsigned int* ticket;
+  float* loss;
+  int* status;
+};
+
+__device__ __forceinline__ void lse_merge(float& m, float& l, float m2, float l2) {
+  const float mn = fmaxf(m, m2);
+  l = l * ex2_approx(m - mn) + l2 * ex2_approx(m2 - mn);
+  m = mn;
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = bf16lo_to_f32(w[e]);
+    f[2 * e + 1] = bf16hi_to_f32(w[e]);
+  }
+}
+
+__global__ void __launch_bounds__(CE_THREADS) flce_ce_rows_kernel(const CeArgs a) {
+  __shared__ float sm_m[CE_THREADS / 32], sm_l[CE_THREADS / 32];
+  __shared__ float s_zy, s_lse2;
+  __shared__ int s_n;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    int n = 0;
+    for (int t = 0; t < a.TM; ++t) n += a.tile_valid[t];
+    s_n = n;
+  }
+  const bool vec = (a.V & 7) == 0 && (reinterpret_cast<uintptr_t>(a.logits) & 15) == 0 &&
+                   (a.dlogits == nullptr || (reinterpret_cast<uintptr_t>(a.dlogits) & 15) == 0);
+#pragma unroll 1
+  for (int row = blockIdx.x; row < a.N; row += gridDim.x) {
+    const uint16_t* z = a.logits + static_cast<size_t>(row) * a.V;
+    const int yi = a.y[row];
+    const bool in_range = yi >= 0 && yi < a.V;
+    const bool valid = yi != a.ignore_index && in_range;
+    if (tid == 0 && yi != a.ignore_index && !in_range) raise_status(a.status, ST_TARGET_OUT_OF_RANGE);
+    if (tid == 0) s_zy = 0.f;
+    __syncthreads();
+    // ---- online max and sum of 2^(z log2 e) over the row
+    float m = -1e30f, l = 0.f;
+    if (vec) {
+      const uint4* zv = reinterpret_cast<const uint4*>(z);
+      const int nv = a.V >> 3;
+#pragma unroll 1
+      for (int base = tid; base < nv; base += CE_THREADS * CE_UNROLL) {
+        uint4 buf[CE_UNROLL];
+#pragma unroll
+        for (int u = 0; u < CE_UNROLL; ++u) {
+          const int j = base + u * CE_THREADS;
+          buf[u] = j < nv ? zv[j] : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < CE_UNROLL; ++u) {
+          const int j = base + u * CE_THREADS;
+          if (j < nv) {
+            float f[8];
+            unpack_bf16x8(buf[u], f);
+            if (static_cast<unsigned>(yi - 8 * j) < 8u) s_zy = f[yi - 8 * j];
+            float cm = f[0];
+#pragma unroll
+            for (int e = 1; e < 8; ++e) cm = fmaxf(cm, f[e]);
+            const float mn = fmaxf(m, cm * LOG2E);
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc += ex2_approx(fmaf(f[e], LOG2E, -mn));
+            l = l * ex2_approx(m - mn) + acc;
+            m = mn;
+          }
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int j = tid; j < a.V; j += CE_THREADS) {
+        const float f = __uint_as_float(static_cast<uint32_t>(z[j]) << 16);
+        if (j == yi) s_zy = f;
+        const float mn = fmaxf(m, f * LOG2E);
+        l = l * ex2_approx(m - mn) + ex2_approx(fmaf(f, LOG2E, -mn));
+        m = mn;
+      }
+    }
+    // ---- block reduction of (m, l), fixed order
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+      lse_merge(m, l, m2, l2);
+    }
+    if ((tid & 31) == 0) {
+      sm_m[tid >> 5] = m;
+      sm_l[tid >> 5] = l;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      float M = sm_m[0], L = sm_l[0];
+      for (int w = 1; w < CE_THREADS / 32; ++w) {
+        const float mn = fmaxf(M, sm_m[w]);
+        L = L * exp2f(M - mn) + sm_l[w] * exp2f(sm_m[w] - mn);
+        M = mn;
+      }
+      const float lse2 = M + log2f(L);
+      s_lse2 = lse2;
+      const double row_l = valid ? static_cast<double>(lse2) * LN2 - static_cast<double>(s_zy) : 0.0;
+      const double wgt = (a.reduction == RED_NONE && a.grad_row_scale && valid) ? a.grad_row_scale[row] : 1.0;
+      a.row_acc[row] = row_l * wgt;
+      if (a.row_loss) a.row_loss[row] = static_cast<float>(row_l);
+    }
+    __syncthreads();
+    // ---- gradient: s_i (softmax - onehot), bf16
+    if (a.dlogits) {
+      uint16_t* g = a.dlogits + static_cast<size_t>(row) * a.V;
+      const float inv_n = s_n ? 1.f / static_cast<float>(s_n) : 0.f;
+      const float sc = valid ? row_weight(a.reduction, &inv_n, a.grad_row_scale, row) : 0.f;
+      const float l2r = s_lse2;
+      if (vec) {
+        const uint4* zv = reinterpret_cast<const uint4*>(z);
+        uint4* gv = reinterpret_cast<uint4*>(g);
+        const int nv = a.V >> 3;
+#pragma unroll 1
+        for (int base = tid; base < nv; base += CE_THREADS * CE_UNROLL) {
+          uint4 buf[CE_UNROLL];
+#pragma unroll
+          for (int u = 0; u < CE_UNROLL; ++u) {
+            const int j = base + u * CE_THREADS;
+            buf[u] = (j < nv && valid) ? zv[j] : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int u = 0; u < CE_UNROLL; ++u) {
+            const int j = base + u * CE_THREADS;
+            if (j < nv) {
+              float f[8];
+              unpack_bf16x8(buf[u], f);
+              float o[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                o[e] = valid ? ex2_approx(fmaf(f[e], LOG2E, -l2r)) * sc : 0.f;
+              if (valid && static_cast<unsigned>(yi - 8 * j) < 8u) o[yi - 8 * j] -= sc;
+              gv[j] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                 pack_bf16x2(o[6], o[7]));
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int j = tid; j < a.V; j += CE_THREADS) {
+          float o = 0.f;
+          if (valid) {
+            const float f = __uint_as_float(static_cast<uint32_t>(z[j]) << 16);
+            o = ex2_approx(fmaf(f, LOG2E, -l2r)) * sc;
+            if (j == yi) o -= sc;
+          }
+          __nv_bfloat16 b = __float2bfloat16_rn(o);
+          g[j] = *reinterpret_cast<uint16_t*>(&b);
+        }
+      }
+    }
+    __syncthreads();  // s_zy / s_lse2 are reused by the next row
+  }
+}
+
+// Deterministic sum of the weighted row losses: fixed tree per block, then the
+// last block adds the block sums in order (fp64); 'mean' divides by n_valid.
+__global__ void __launch_bounds__(COMBINE_THREADS) flce_ce_reduce_kernel(const CeArgs a) {
+  const int i = blockIdx.x * COMBINE_THREADS + threadIdx.x;
+  double v = i < a.N ? a.row_acc[i] : 0.0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+  __shared__ double wsum[COMBINE_THREADS / 32];
+  __shared__ bool is_last;
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < COMBINE_THREADS / 32; ++w) t += wsum[w];
+    a.blk_sum[blockIdx.x] = t;
+    __threadfence();
+    is_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (is_last && threadIdx.x == 0) {
+    __threadfence();
+    const volatile double* b = a.blk_sum;
+    double tot = 0.0;
+    for (unsigned k = 0; k < gridDim.x; ++k) tot += b[k];
+    long long n = 0;
+    for (int t = 0; t < a.TM; ++t) n += a.tile_valid[t];
+    if (a.reduction == RED_MEAN)
+      *a.loss = n ? static_cast<float>(tot / static_cast<double>(n)) : 0.f;
     else
       *a.loss = static_cast<float>(tot);
     *a.ticket = 0u;

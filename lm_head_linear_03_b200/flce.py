@@ -25,7 +25,7 @@ STATUS_NAMES = {
     5: "FLCE_ERR_TIMEOUT",
     6: "FLCE_ERR_CUDA",
 }
-NUM_KERNEL_KINDS = 4
+NUM_KERNEL_KINDS = 5
 
 EXPORTED = (
     "flce_status_string",
@@ -39,6 +39,8 @@ EXPORTED = (
     "flce_profile_read",
     "flce_forward_backward_noalloc",
     "flce_forward_backward_ex",
+    "flce_ce_workspace_size",
+    "flce_cross_entropy",
 )
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -95,6 +97,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_profile_read.restype = ctypes.c_int
     lib.flce_forward_backward_ex.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.flce_forward_backward_ex.restype = ctypes.c_int
+    lib.flce_ce_workspace_size.argtypes = [i64, i64]
+    lib.flce_ce_workspace_size.restype = sz
+    lib.flce_cross_entropy.argtypes = [vp, vp, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.flce_cross_entropy.restype = ctypes.c_int
     lib.flce_forward_backward_noalloc.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp, vp]
     lib.flce_forward_backward_noalloc.restype = ctypes.c_int
     _lib = lib
@@ -210,6 +216,32 @@ def forward_backward_ex(X, W, y, ignore_index: int = -100, *, reduction: str = "
                                       _ptr(workspace), workspace.numel(), _stream_handle(stream))
     _check(st, "flce_forward_backward_ex")
     return loss, status, rl, dX, dW
+
+
+def cross_entropy(logits, y, ignore_index: int = -100, *, reduction: str = "mean", grad_row_scale=None,
+                  row_loss: bool = False, grad: str = "new", workspace=None, stream=None):
+    """Cross-entropy on given bf16 logits [N, V]; asynchronous.  Returns device
+    tensors (loss[1], status[1], row_loss[N] or None, dlogits or None).
+    grad: 'new' (a new tensor), 'inplace' (overwrite ``logits``) or 'none'."""
+    lib = load_library()
+    if not (logits.is_cuda and y.is_cuda) or logits.dtype != torch.bfloat16 or y.dtype != torch.int32:
+        raise ValueError("expected CUDA bf16 logits and int32 targets")
+    if logits.dim() != 2 or y.shape != (logits.shape[0],) or not (logits.is_contiguous() and y.is_contiguous()):
+        raise ValueError("expected contiguous logits [N, V] and targets [N]")
+    N, V = logits.shape
+    dev = logits.device
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    rl = torch.empty(N, dtype=torch.float32, device=dev) if row_loss else None
+    dz = {"new": lambda: torch.empty_like(logits), "inplace": lambda: logits, "none": lambda: None}[grad]()
+    if workspace is None:
+        workspace = torch.empty(int(lib.flce_ce_workspace_size(N, V)), dtype=torch.uint8, device=dev)
+    vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
+    st = lib.flce_cross_entropy(_ptr(logits), _ptr(y), N, V, ignore_index, REDUCTIONS[reduction], vp(grad_row_scale),
+                                _ptr(loss), vp(rl), _ptr(status), vp(dz), _ptr(workspace), workspace.numel(),
+                                _stream_handle(stream))
+    _check(st, "flce_cross_entropy")
+    return loss, status, rl, dz
 
 
 def forward_backward_host(hX, hW, hy, dev_bufs, ignore_index: int = -100, *, h_out=None, stream=None):
