@@ -133,6 +133,10 @@ typedef enum { FLCE_REDUCTION_MEAN = 0, FLCE_REDUCTION_SUM = 1, FLCE_REDUCTION_N
 /* Asynchronous entry with every option.
  *   reduction:      flce_reduction_t
  *   grad_row_scale: DEVICE float[N] or NULL (used by NONE only)
+ *   d_mean_count:   DEVICE int32 or NULL (MEAN only): divide by this count
+ *                   instead of this call's n_valid, e.g. the number of valid
+ *                   targets over every data-parallel rank, so that the ranks'
+ *                   losses and dW add up to those of the whole batch
  *   d_loss:         DEVICE float, receives sum_i s_i l_i
  *   d_row_loss:     DEVICE float[N] or NULL: l_i for valid rows, 0 for ignored rows
  *   d_status:       DEVICE int32, 0 or a device-side flce_status_t
@@ -141,9 +145,10 @@ typedef enum { FLCE_REDUCTION_MEAN = 0, FLCE_REDUCTION_SUM = 1, FLCE_REDUCTION_N
  * Other arguments as flce_forward_backward_async. */
 flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N,
                                        int64_t H, int64_t V, int32_t ignore_index, int32_t reduction,
-                                       const float* grad_row_scale, float* d_loss, float* d_row_loss,
-                                       int32_t* d_status, uint16_t* dX, uint16_t* dW, void* workspace,
-                                       size_t workspace_bytes, cudaStream_t stream);
+                                       const float* grad_row_scale, const int32_t* d_mean_count,
+                                       float* d_loss, float* d_row_loss, int32_t* d_status, uint16_t* dX,
+                                       uint16_t* dW, void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream);
 
 /* Cross-entropy on a logit tensor the caller already holds, the unfused
  * counterpart of the head ("Complete Guide to Liger Kernel", section
@@ -187,6 +192,14 @@ flce_status_t flce_forward_backward_noalloc(const uint16_t* X, const uint16_t* W
                                             int64_t N, int64_t H, int64_t V, int32_t ignore_index,
                                             float* loss, uint16_t* dX, uint16_t* dW,
                                             cudaStream_t stream);
+
+/* Failure-detection probe.  Launches one thread that waits, each time for at
+ * most timeout_ns, on an mbarrier phase that nobody completes and on a global
+ * counter that nobody increments, with the same bounded-wait code the
+ * kernels use.  d_status: DEVICE int32[3]; afterwards d_status[0] and
+ * d_status[1] hold FLCE_ERR_TIMEOUT (the waits gave up instead of hanging)
+ * and d_status[2] the untouched counter.  timeout_ns in (0, 1e10]. */
+flce_status_t flce_probe_bounded_wait(int64_t timeout_ns, int32_t* d_status, cudaStream_t stream);
 
 /* How a call of these sizes is split into launches (host-only query). */
 typedef struct {

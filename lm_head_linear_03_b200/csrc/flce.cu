@@ -288,6 +288,7 @@ struct Options {
   int reduction = RED_MEAN;
   const float* grad_row_scale = nullptr;
   float* row_loss = nullptr;
+  const int* mean_count = nullptr;
 };
 
 flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
@@ -400,6 +401,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     c.reduction = opt.reduction;
     c.grad_row_scale = opt.grad_row_scale;
     c.row_loss = opt.row_loss;
+    c.mean_count = opt.mean_count;
     const int grid = static_cast<int>((N + COMBINE_THREADS - 1) / COMBINE_THREADS);
     size_t slot;
     prof_begin(stream, KIND_COMBINE, &slot);
@@ -507,21 +509,23 @@ flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, 
 
 flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H,
                                        int64_t V, int32_t ignore_index, int32_t reduction,
-                                       const float* grad_row_scale, float* d_loss, float* d_row_loss,
-                                       int32_t* d_status, uint16_t* dX, uint16_t* dW, void* workspace,
-                                       size_t workspace_bytes, cudaStream_t stream) {
+                                       const float* grad_row_scale, const int32_t* d_mean_count, float* d_loss,
+                                       float* d_row_loss, int32_t* d_status, uint16_t* dX, uint16_t* dW,
+                                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!d_loss || !d_status) return FLCE_ERR_INVALID_ARGUMENT;
   if (reduction != FLCE_REDUCTION_MEAN && reduction != FLCE_REDUCTION_SUM && reduction != FLCE_REDUCTION_NONE)
     return FLCE_ERR_INVALID_ARGUMENT;
   const flce_status_t s = check_args(X, W, y, N, H, V, dX, dW, workspace, true);
   if (s != FLCE_OK) return s;
-  if (!aligned(d_status, 4) || !aligned(d_loss, 4) || !aligned(d_row_loss, 4) || !aligned(grad_row_scale, 4))
+  if (!aligned(d_status, 4) || !aligned(d_loss, 4) || !aligned(d_row_loss, 4) || !aligned(grad_row_scale, 4) ||
+      !aligned(d_mean_count, 4))
     return FLCE_ERR_UNSUPPORTED;
   if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   Options opt;
   opt.reduction = reduction;
   opt.grad_row_scale = reduction == FLCE_REDUCTION_NONE ? grad_row_scale : nullptr;
   opt.row_loss = d_row_loss;
+  opt.mean_count = reduction == FLCE_REDUCTION_MEAN ? d_mean_count : nullptr;
   return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, stream, opt);
 }
 
@@ -584,6 +588,19 @@ flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64
   prof_end(stream, slot);
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   return FLCE_OK;
+}
+
+flce_status_t flce_probe_bounded_wait(int64_t timeout_ns, int32_t* d_status, cudaStream_t stream) {
+  if (!d_status || timeout_ns <= 0 || timeout_ns > 10000000000ll) return FLCE_ERR_INVALID_ARGUMENT;
+  if (!aligned(d_status, 4)) return FLCE_ERR_UNSUPPORTED;
+  DevInfo di;
+  int dev;
+  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
+  // d_status[0], d_status[1]: the two waits' results; d_status[2]: the counter nobody sets
+  if (cudaMemsetAsync(d_status, 0, 3 * sizeof(int32_t), stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  flce_wait_probe_kernel<<<1, 32, 0, stream>>>(d_status, d_status + 2, static_cast<unsigned long long>(timeout_ns));
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
 flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_W, const int32_t* h_y, int64_t N,

@@ -1059,6 +1059,7 @@ struct CombineArgs {
   int reduction;
   const float* grad_row_scale;
   float* row_loss;  // optional per-row losses
+  const int* mean_count;  // optional: divide the mean by this count instead of n_valid
   const int32_t* y;
   const float* part_m;
   const float* part_l;
@@ -1142,13 +1143,32 @@ __global__ void __launch_bounds__(COMBINE_THREADS) flce_combine_kernel(const Com
       cnt += bc[b];
     }
     *a.n_valid = static_cast<int>(cnt);
-    *a.inv_n = cnt ? static_cast<float>(1.0 / static_cast<double>(cnt)) : 0.f;
+    // a data-parallel caller divides by the count over every rank's tokens
+    const long long den = a.mean_count ? static_cast<long long>(*a.mean_count) : cnt;
+    *a.inv_n = den > 0 ? static_cast<float>(1.0 / static_cast<double>(den)) : 0.f;
     if (a.reduction == RED_MEAN)
-      *a.loss = cnt ? static_cast<float>(tot / static_cast<double>(cnt)) : 0.f;
+      *a.loss = den > 0 ? static_cast<float>(tot / static_cast<double>(den)) : 0.f;
     else
       *a.loss = static_cast<float>(tot);
     *a.ticket = 0u;
   }
+}
+
+// ================================================== bounded-wait probe ==
+//
+// Exercises the two bounded waits every kernel above relies on, on things that
+// never happen: an mbarrier phase nobody arrives on and a global counter
+// nobody increments.  Each wait must give up after `timeout_ns` and report
+// ST_TIMEOUT in its own status slot, leaving the context usable.
+__global__ void flce_wait_probe_kernel(int* status, const int* never, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(smem_u32(&bar), 1);
+  fence_mbar_init();
+  if (!mbar_wait(smem_u32(&bar), 0, &abort_flag, timeout_ns)) status[0] = ST_TIMEOUT;
+  if (!wait_counter(never, 1, &abort_flag, timeout_ns)) status[1] = ST_TIMEOUT;
 }
 
 // ======================================== cross-entropy on given logits ==

@@ -41,6 +41,7 @@ EXPORTED = (
     "flce_forward_backward_ex",
     "flce_ce_workspace_size",
     "flce_cross_entropy",
+    "flce_probe_bounded_wait",
 )
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -95,12 +96,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_profile_enable.restype = ctypes.c_int
     lib.flce_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)]
     lib.flce_profile_read.restype = ctypes.c_int
-    lib.flce_forward_backward_ex.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.flce_forward_backward_ex.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                             vp]
     lib.flce_forward_backward_ex.restype = ctypes.c_int
     lib.flce_ce_workspace_size.argtypes = [i64, i64]
     lib.flce_ce_workspace_size.restype = sz
     lib.flce_cross_entropy.argtypes = [vp, vp, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.flce_cross_entropy.restype = ctypes.c_int
+    lib.flce_probe_bounded_wait.argtypes = [i64, vp, vp]
+    lib.flce_probe_bounded_wait.restype = ctypes.c_int
     lib.flce_forward_backward_noalloc.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp, vp]
     lib.flce_forward_backward_noalloc.restype = ctypes.c_int
     _lib = lib
@@ -189,12 +193,14 @@ def forward_backward_async(X, W, y, ignore_index: int = -100, *, out=None, works
 
 
 def forward_backward_ex(X, W, y, ignore_index: int = -100, *, reduction: str = "mean", grad_row_scale=None,
-                        row_loss: bool = False, grads: bool = True, workspace=None, stream=None):
+                        mean_count=None, row_loss: bool = False, grads: bool = True, workspace=None, stream=None):
     """Asynchronous call with every option; returns device tensors
     (loss[1], status[1], row_loss[N] or None, dX or None, dW or None).
 
     reduction 'mean' | 'sum' | 'none'; grad_row_scale: fp32[N] upstream
-    gradient of each row's loss for 'none'; grads=False skips the gradient pass.
+    gradient of each row's loss for 'none'; mean_count: int32[1] device count
+    the mean divides by instead of this call's n_valid; grads=False skips the
+    gradient pass.
     """
     lib = load_library()
     _check_inputs(X, W, y)
@@ -211,9 +217,11 @@ def forward_backward_ex(X, W, y, ignore_index: int = -100, *, reduction: str = "
     dW = torch.empty_like(W) if grads else None
     workspace = alloc_workspace(N, H, V, dev) if workspace is None else workspace
     vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
+    if mean_count is not None and (mean_count.dtype != torch.int32 or not mean_count.is_cuda):
+        raise ValueError("mean_count must be a CUDA int32 tensor")
     st = lib.flce_forward_backward_ex(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, REDUCTIONS[reduction],
-                                      vp(grad_row_scale), _ptr(loss), vp(rl), _ptr(status), vp(dX), vp(dW),
-                                      _ptr(workspace), workspace.numel(), _stream_handle(stream))
+                                      vp(grad_row_scale), vp(mean_count), _ptr(loss), vp(rl), _ptr(status), vp(dX),
+                                      vp(dW), _ptr(workspace), workspace.numel(), _stream_handle(stream))
     _check(st, "flce_forward_backward_ex")
     return loss, status, rl, dX, dW
 
@@ -298,3 +306,11 @@ def forward_backward_noalloc(X, W, y, ignore_index: int = -100, *, dX=None, dW=N
                                            ctypes.byref(loss), _ptr(dX), _ptr(dW), _stream_handle(stream))
     _check(st, "flce_forward_backward_noalloc")
     return loss.value, dX, dW
+
+
+def probe_bounded_wait(timeout_ns: int = 1_000_000, stream=None):
+    """Runs the bounded-wait probe and returns its device status tensor int32[3]."""
+    lib = load_library()
+    st = torch.empty(3, dtype=torch.int32, device="cuda")
+    _check(lib.flce_probe_bounded_wait(timeout_ns, _ptr(st), _stream_handle(stream)), "flce_probe_bounded_wait")
+    return st

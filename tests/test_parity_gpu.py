@@ -275,3 +275,35 @@ def test_whole_ignored_token_tiles_are_skipped(N, H, V, ignored):
     y[ignored] = -100
     loss, dX, dW = run_full_oracle_case(X, W, y)
     assert torch.count_nonzero(dX[ignored]).item() == 0
+
+
+def test_bounded_waits_give_up_and_report_timeout():
+    """Failure detection without a fault: waits on an event that never comes
+    end after their limit with FLCE_ERR_TIMEOUT, and the device stays usable."""
+    F = _lib()
+    from lm_head_linear_03_b200 import flce
+    import time
+    t0 = time.perf_counter()
+    st = flce.probe_bounded_wait(2_000_000)  # 2 ms per wait
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert st.tolist() == [5, 5, 0]
+    run_full_oracle_case(*make_inputs(WORKLOADS["tiny"]))
+
+
+def test_mean_over_external_count():
+    """The data-parallel hook: the mean divides by a count from outside the call
+    (all ranks' valid targets); equals the oracle with weights 1/count."""
+    F = _lib()
+    w = custom("mean_count", N=300, H=136, V=5000, ignore_frac=0.1)
+    X, W, y = make_inputs(w)
+    count = 1000
+    loss, status, _, dX, dW = F.forward_backward_ex(X.cuda(), W.cuda(), y.cuda(),
+                                                    mean_count=torch.tensor([count], dtype=torch.int32).cuda())
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    valid = (y != -100).numpy()
+    ref, rdX, rdW, _, _ = O.flce_reference(X, W, y, reduction="none", grad_row_scale=np.where(valid, 1.0 / count, 0.0))
+    assert_loss_close(loss.item(), ref)
+    assert_grad_close(_np(dX), rdX, "dX")
+    assert_grad_close(_np(dW), rdW, "dW")
