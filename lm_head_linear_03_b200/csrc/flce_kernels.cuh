@@ -819,7 +819,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
           give_up();
           break;
         }
-        fence_proxy_async_global();  // G written by other CTAs' TMA stores, read by TMA below
+        // G written by other CTAs' TMA stores is read below by TMA: order the
+        // acquire above before those reads (G tiles read only X and W)
+        if (it.kind != ITEM_GRAD) fence_proxy_async_global();
         const int m0 = it.a * CM + rank * BM;
         const int n0 = it.b * BN + rank * BNH;
         for (int kb = 0; kb < kblocks; ++kb) {

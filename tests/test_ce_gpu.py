@@ -46,7 +46,9 @@ def _check(Z, y, reduction="mean", grad_row_scale=None, grad="new"):
     return dz
 
 
-@pytest.mark.parametrize("N,V", [(256, 4096), (300, 5000), (1, 300), (129, 100), (64, 1001), (17, 3)])
+# Widths with V % 8 == 0 take the 16-byte vector path, others the scalar one.
+@pytest.mark.parametrize("N,V", [(256, 4096), (300, 5000), (1, 300), (129, 100), (64, 1001), (17, 3),
+                                 (9, 40000), (5, 200000), (3, 300000)])
 def test_ce_small(N, V):
     Z, y = _case(N, V)
     _check(Z, y)
