@@ -36,7 +36,7 @@
  *
  * Ownership.  All device pointers belong to the caller.  The library never
  * allocates device memory: scratch space is the caller's `workspace`, at least
- * flce_workspace_size(N, H, V) bytes, whose size depends on N and H only.  dX
+ * flce_workspace_size(N, H, V) bytes (at least the base size, see there).  dX
  * and dW are overwritten, not accumulated into.  The library keeps only
  * read-only host caches (device properties, a driver entry point).
  *
@@ -45,6 +45,16 @@
  * bounded wait inside a kernel that ran out) are written to a device status
  * word; the synchronous entry points read it back and return it.  Nothing
  * traps or asserts on the device.
+ *
+ * Ignored rows.  The work runs in 256-row token tiles, and a tile whose
+ * targets are all ignored is skipped.  When ignored rows are scattered, so
+ * that packing the valid rows first would fill fewer tiles than the tiles
+ * holding any valid row, and the workspace holds the packed-X area (see
+ * flce_workspace_size), the library reorders the token rows on the device (a
+ * stable partition, valid rows first): it packs those rows of X into the
+ * workspace, runs both passes on them, and writes dX and the per-row losses
+ * back in the caller's row order.  The choice changes only the order of
+ * floating-point sums, not the result's definition.
  */
 #ifndef FLCE_H_
 #define FLCE_H_
@@ -62,7 +72,7 @@ typedef enum {
   FLCE_OK = 0,
   FLCE_ERR_INVALID_ARGUMENT = 1,    /* NULL pointer, non-positive size, size too large */
   FLCE_ERR_UNSUPPORTED = 2,         /* H % 8 != 0, misaligned pointer, device is not sm_100 */
-  FLCE_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < flce_workspace_size(N, H, V) */
+  FLCE_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < flce_workspace_size(N, H, 1) */
   FLCE_ERR_TARGET_OUT_OF_RANGE = 4, /* some y_i != ignore_index lies outside [0, V) */
   FLCE_ERR_TIMEOUT = 5,             /* a bounded wait inside a kernel gave up */
   FLCE_ERR_CUDA = 6                 /* a CUDA runtime call failed */
@@ -71,9 +81,15 @@ typedef enum {
 /* Human-readable name of a status code (static storage). */
 const char* flce_status_string(int status);
 
-/* Bytes of device workspace one call needs.  Depends on N and H only (V is
- * accepted for symmetry and ignored): the logits are processed one vocabulary
- * chunk of fixed width at a time.  Returns 0 for invalid sizes. */
+/* Bytes of device workspace one call asks for.  The logits are processed one
+ * vocabulary chunk of fixed width at a time, so the base size depends on N
+ * and H only; it is flce_workspace_size(N, H, 1).  On top of it comes an
+ * N x H bf16 area (its byte size rounded up to a multiple of 256) for a
+ * packed copy of X, which reordered token rows need
+ * (see "Ignored rows"), whenever the whole stays within 5% of the N x V bf16
+ * logits the head never stores.  Every entry accepts any workspace of at
+ * least the base size and reorders rows only when the area fits in it.
+ * Returns 0 for invalid sizes. */
 size_t flce_workspace_size(int64_t N, int64_t H, int64_t V);
 
 /* Synchronous forward + backward.
@@ -92,7 +108,7 @@ flce_status_t flce_forward_backward(const uint16_t* X, const uint16_t* W, const 
 /* Asynchronous twin: enqueues the whole computation on `stream` and returns.
  *   d_loss:   DEVICE float*, receives the loss when the stream gets there
  *   d_status: DEVICE int32_t*, receives 0 or a device-side flce_status_t
- *   workspace_bytes: size of `workspace`, checked against flce_workspace_size
+ *   workspace_bytes: size of `workspace`, at least flce_workspace_size(N, H, 1)
  * Host-side argument errors are returned immediately; device-side errors only
  * appear in *d_status. */
 flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, const int32_t* y,
@@ -201,6 +217,17 @@ flce_status_t flce_forward_backward_noalloc(const uint16_t* X, const uint16_t* W
  * and d_status[2] the untouched counter.  timeout_ns in (0, 1e10]. */
 flce_status_t flce_probe_bounded_wait(int64_t timeout_ns, int32_t* d_status, cudaStream_t stream);
 
+/* Token-row order chosen by the last call that used `workspace` (see
+ * "Ignored rows" above), read back once `stream` has finished that call:
+ *   *reordered = 1 when the rows were reordered (valid rows first, X packed
+ *                in that order, dX scattered back), 0 otherwise
+ *   *n_valid   = the number of rows whose target is not ignore_index
+ * Synchronises `stream`.  The workspace must be the 256-B aligned buffer the
+ * call used; FLCE_ERR_INVALID_ARGUMENT for NULL or misaligned pointers.  The
+ * pages describe no such query; it exposes the library's own choice. */
+flce_status_t flce_row_order_info(const void* workspace, int32_t* reordered, int32_t* n_valid,
+                                  cudaStream_t stream);
+
 /* How a call of these sizes is split into launches (host-only query). */
 typedef struct {
   int64_t workspace_bytes; /* same as flce_workspace_size */
@@ -219,8 +246,10 @@ flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out);
  * online log-sum-exp, 1 combine, 2 pass 2 (logit recompute + G, dW and dX
  * contractions of every vocabulary chunk, one persistent launch), 3 prep
  * (valid rows per 256-row token tile), 4 cross-entropy on given logits (rows
- * pass; its final sum is counted under kind 1). */
-#define FLCE_NUM_KERNEL_KINDS 5
+ * pass; its final sum is counted under kind 1), 5 token-row order (see
+ * "Ignored rows"), 6 dX row scatter and 7 X row packing (both only do work
+ * when the rows were reordered). */
+#define FLCE_NUM_KERNEL_KINDS 8
 const char* flce_kernel_name(int kind);
 flce_status_t flce_profile_enable(int on);
 flce_status_t flce_profile_read(int32_t* launches, double* total_ms);

@@ -17,5 +17,6 @@ from .flce import (  # noqa: F401
     plan,
     profile_enable,
     profile_read,
+    row_order_info,
     workspace_size,
 )

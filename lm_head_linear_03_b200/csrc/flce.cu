@@ -27,19 +27,25 @@ constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per bou
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t ctrl, counters, counters_bytes, tile_valid, lse2, zy, part_m, part_l, blk_loss, blk_cnt, G, lo, total;
+  size_t ctrl, counters, counters_bytes, tile_cnt, tile_valid, perm, y_perm, g_perm, lse2, zy, part_m, part_l,
+      blk_loss, blk_cnt, G, lo, xc, total;
+  bool packed;  // holds xc, the packed copy of X that reordered rows need
 };
 
-// ctrl block: [0] status, [4] ticket, [8] n_valid, [12] inv_n, [16] loss
+// ctrl block: [0] status, [4] ticket, [8] n_valid, [12] inv_n, [16] loss,
+// [20] reordered (1 when the token rows are reordered), [24] valid rows
 struct Ctrl {
   int32_t status;
   uint32_t ticket;
   int32_t n_valid;
   float inv_n;
   float loss;
+  int32_t reordered;
+  int32_t n_rows;
 };
 
-WsLayout ws_layout(int64_t N, int64_t H) {
+// `packed`: with the N x H area for the packed copy of X (reordered rows).
+WsLayout ws_layout(int64_t N, int64_t H, bool packed = false) {
   WsLayout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -54,7 +60,11 @@ WsLayout ws_layout(int64_t N, int64_t H) {
   const size_t tm = (n + CM - 1) / CM;
   L.counters_bytes = (2 * tm + 2 * (VC / BN)) * 4;
   L.counters = take(L.counters_bytes);
+  L.tile_cnt = take(tm * 4);
   L.tile_valid = take(tm * 4);
+  L.perm = take(tm * CM * 4);
+  L.y_perm = take(n * 4);
+  L.g_perm = take(n * 4);
   L.lse2 = take(n * 4);
   L.zy = take(n * 4);
   L.part_m = take(static_cast<size_t>(MAX_SPLITS) * n * 4);
@@ -63,8 +73,18 @@ WsLayout ws_layout(int64_t N, int64_t H) {
   L.blk_cnt = take(nblk * 4);
   L.G = take(n * VC * 2);
   L.lo = take(n * static_cast<size_t>(H) * 2);
+  L.packed = packed;
+  L.xc = packed ? take(n * static_cast<size_t>(H) * 2) : 0;
   L.total = off;
   return L;
+}
+
+// The workspace a call is asked for: the packed-X area is included when the
+// whole stays within 5% of the N x V bf16 logits the head never stores.
+size_t ws_total(int64_t N, int64_t H, int64_t V) {
+  const size_t with = ws_layout(N, H, true).total;
+  const double logits = 2.0 * static_cast<double>(N) * static_cast<double>(V);
+  return static_cast<double>(with) <= 0.05 * logits ? with : ws_layout(N, H).total;
 }
 
 // Workspace of the cross-entropy-on-logits entry: depends on N only.
@@ -234,7 +254,8 @@ Plan make_plan(int64_t N, int64_t H, int64_t V, int clusters) {
   p.lse_clusters =
       static_cast<int>(std::min<long long>(static_cast<long long>(p.tiles_m) * p.splits, clusters));
   p.num_chunks = static_cast<int>((V + VC - 1) / VC);
-  p.launches = 4;  // prep, pass 1, combine, pass 2
+  // prep, row order, pass 1, combine, pass 2, dX scatter; X pack with the packed-X area
+  p.launches = ws_total(N, H, V) == ws_layout(N, H, true).total ? 7 : 6;
   return p;
 }
 
@@ -293,7 +314,7 @@ struct Options {
 
 flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
                       int32_t ignore_index, float* d_loss, int32_t* d_status, uint16_t* dX, uint16_t* dW,
-                      void* workspace, cudaStream_t stream, const Options& opt = Options()) {
+                      void* workspace, size_t ws_bytes, cudaStream_t stream, const Options& opt = Options()) {
   DevInfo di;
   int dev;
   if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
@@ -302,7 +323,8 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   if (!get_encode()) return FLCE_ERR_CUDA;
 
   if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;  // now with max_clusters
-  const WsLayout L = ws_layout(N, H);
+  // reordered rows need the packed-X area: only a large enough workspace has it
+  const WsLayout L = ws_layout(N, H, ws_bytes >= ws_layout(N, H, true).total);
   const Plan P = make_plan(N, H, V, di.max_clusters);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
@@ -312,12 +334,19 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   float* part_l = reinterpret_cast<float*>(ws + L.part_l);
   uint16_t* G = reinterpret_cast<uint16_t*>(ws + L.G);
   uint16_t* lo = reinterpret_cast<uint16_t*>(ws + L.lo);
+  int* perm = reinterpret_cast<int*>(ws + L.perm);
+  int32_t* y_perm = reinterpret_cast<int32_t*>(ws + L.y_perm);
+  float* g_perm = reinterpret_cast<float*>(ws + L.g_perm);
+  const float* g_rows = opt.grad_row_scale ? g_perm : nullptr;  // upstream weights in the rows' order
+  uint16_t* Xc = L.packed ? reinterpret_cast<uint16_t*>(ws + L.xc) : nullptr;
 
-  CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn, mHi, mLo;
+  CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn, mHi, mLo, mXc_k, mXc_mn;
   const uint64_t n = static_cast<uint64_t>(N), h = static_cast<uint64_t>(H), v = static_cast<uint64_t>(V);
   bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BNH) &&
             make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
             make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK) &&
+            // the packed copy of X (the caller's X stands in when there is none: never read then)
+            make_map(&mXc_k, Xc ? Xc : X, h, n, h * 2, BK, BM) && make_map(&mXc_mn, Xc ? Xc : X, h, n, h * 2, 64, BK) &&
             (dX == nullptr || (make_map(&mHi, dX, h, n, h * 2, BN, BM, Swz::none) &&
                                make_map(&mLo, lo, h, n, h * 2, BN, BM, Swz::none)));
   // 32 x 32 output boxes of the epilogues (64-byte swizzle)
@@ -339,7 +368,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   a.V = static_cast<int>(V);
   a.ignore_index = ignore_index;
   a.Vc = VC;
-  a.y = y;
+  a.y = y_perm;
   a.part_m = part_m;
   a.part_l = part_l;
   a.zy = zy;
@@ -352,17 +381,34 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   a.status = d_status;
   a.timeout_ns = DEFAULT_TIMEOUT_NS;
   a.reduction = opt.reduction;
-  a.grad_row_scale = opt.grad_row_scale;
+  a.grad_row_scale = g_rows;
   a.tile_valid = reinterpret_cast<const int*>(ws + L.tile_valid);
+  a.perm = perm;
+  a.reordered = &ctrl->reordered;
 
-  // Valid rows per 256-row token tile.
+  // Valid rows per 256-row token tile, then the token-row order of both passes.
   {
     size_t slot;
     prof_begin(stream, KIND_PREP, &slot);
     flce_prep_kernel<<<P.tiles_m, CM, 0, stream>>>(y, static_cast<int>(N), ignore_index,
-                                                   reinterpret_cast<int*>(ws + L.tile_valid));
+                                                   reinterpret_cast<int*>(ws + L.tile_cnt));
     prof_end(stream, slot);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    prof_begin(stream, KIND_ORDER, &slot);
+    flce_row_order_kernel<<<P.tiles_m, CM, 0, stream>>>(
+        y, opt.grad_row_scale, static_cast<int>(N), P.tiles_m, ignore_index,
+        reinterpret_cast<const int*>(ws + L.tile_cnt), L.packed ? 1 : 0, reinterpret_cast<int*>(ws + L.tile_valid),
+        perm, y_perm, g_perm, &ctrl->reordered, &ctrl->n_rows);
+    prof_end(stream, slot);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    if (L.packed) {  // X rows in the new order (returns at once when the order was kept)
+      const int pgrid = static_cast<int>(std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(di.num_sms) * 8));
+      prof_begin(stream, KIND_PACK, &slot);
+      flce_pack_rows_kernel<<<pgrid, 256, 0, stream>>>(X, Xc, perm, &ctrl->reordered, &ctrl->n_rows,
+                                                        static_cast<int>(N), static_cast<int>(H));
+      prof_end(stream, slot);
+      if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    }
   }
 
   // Pass 1: logits tile by tile, online log-sum-exp per (row, split).
@@ -375,7 +421,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     p1.num_units = P.tiles_m * P.splits;
     size_t slot;
     prof_begin(stream, KIND_LSE, &slot);
-    flce_pass1_kernel<<<CLUSTER * P.lse_clusters, NUM_THREADS, P1_SMEM_BYTES, stream>>>(mX_k, mW_k, p1);
+    flce_pass1_kernel<<<CLUSTER * P.lse_clusters, NUM_THREADS, P1_SMEM_BYTES, stream>>>(mX_k, mXc_k, mW_k, p1);
     prof_end(stream, slot);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
@@ -386,7 +432,8 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     c.V = static_cast<int>(V);
     c.ignore_index = ignore_index;
     c.splits = P.splits;
-    c.y = y;
+    c.y = y_perm;
+    c.perm = perm;
     c.part_m = part_m;
     c.part_l = part_l;
     c.zy = zy;
@@ -399,7 +446,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     c.loss = d_loss;
     c.status = d_status;
     c.reduction = opt.reduction;
-    c.grad_row_scale = opt.grad_row_scale;
+    c.grad_row_scale = g_rows;
     c.row_loss = opt.row_loss;
     c.mean_count = opt.mean_count;
     const int grid = static_cast<int>((N + COMBINE_THREADS - 1) / COMBINE_THREADS);
@@ -444,14 +491,42 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     pm.Loo = mLoo;
     pm.Hipf = mHi;
     pm.Lopf = mLo;
+    pm.Xck = mXc_k;
+    pm.Xcmn = mXc_mn;
     const int grid = static_cast<int>(std::min<long long>(total, P.clusters));
     size_t slot;
     prof_begin(stream, KIND_PASS2, &slot);
     flce_pass2_kernel<<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, stream>>>(pm, b);
     prof_end(stream, slot);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    // reordered rows: the final dX rows go back in place (no-op otherwise)
+    const int sgrid = static_cast<int>(std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(di.num_sms) * 8));
+    prof_begin(stream, KIND_SCATTER, &slot);
+    flce_dx_scatter_kernel<<<sgrid, 256, 0, stream>>>(lo, dX, perm, &ctrl->reordered, &ctrl->n_rows,
+                                                      static_cast<int>(N), static_cast<int>(H));
+    prof_end(stream, slot);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
   return FLCE_OK;
+}
+
+// Synchronous call on a workspace of `ws_bytes` bytes: enqueue, then read the
+// loss and the device status back.
+flce_status_t sync_call(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
+                        int32_t ignore_index, float* loss, uint16_t* dX, uint16_t* dW, void* workspace,
+                        size_t ws_bytes, cudaStream_t stream) {
+  if (!loss) return FLCE_ERR_INVALID_ARGUMENT;
+  flce_status_t s = check_args(X, W, y, N, H, V, dX, dW, workspace);
+  if (s != FLCE_OK) return s;
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(workspace);  // the control block opens every layout
+  s = enqueue(X, W, y, N, H, V, ignore_index, &ctrl->loss, &ctrl->status, dX, dW, workspace, ws_bytes, stream);
+  if (s != FLCE_OK) return s;
+  Ctrl host{};
+  if (cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  *loss = host.loss;
+  return static_cast<flce_status_t>(host.status);
 }
 
 }  // namespace
@@ -474,25 +549,14 @@ const char* flce_status_string(int s) {
 
 size_t flce_workspace_size(int64_t N, int64_t H, int64_t V) {
   if (check_sizes(N, H, V == 0 ? 1 : V) != FLCE_OK) return 0;
-  return ws_layout(N, H).total;
+  return ws_total(N, H, V == 0 ? 1 : V);
 }
 
 flce_status_t flce_forward_backward(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H,
                                     int64_t V, int32_t ignore_index, float* loss, uint16_t* dX, uint16_t* dW,
                                     void* workspace, cudaStream_t stream) {
-  if (!loss) return FLCE_ERR_INVALID_ARGUMENT;
-  flce_status_t s = check_args(X, W, y, N, H, V, dX, dW, workspace);
-  if (s != FLCE_OK) return s;
-  const WsLayout L = ws_layout(N, H);
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(static_cast<uint8_t*>(workspace) + L.ctrl);
-  s = enqueue(X, W, y, N, H, V, ignore_index, &ctrl->loss, &ctrl->status, dX, dW, workspace, stream);
-  if (s != FLCE_OK) return s;
-  Ctrl host{};
-  if (cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-    return FLCE_ERR_CUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
-  *loss = host.loss;
-  return static_cast<flce_status_t>(host.status);
+  if (check_sizes(N, H, V) != FLCE_OK) return check_sizes(N, H, V);
+  return sync_call(X, W, y, N, H, V, ignore_index, loss, dX, dW, workspace, ws_total(N, H, V), stream);
 }
 
 flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N,
@@ -504,7 +568,7 @@ flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, 
   if (s != FLCE_OK) return s;
   if (!aligned(d_status, 4) || !aligned(d_loss, 4)) return FLCE_ERR_UNSUPPORTED;
   if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
-  return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, stream);
+  return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, workspace_bytes, stream);
 }
 
 flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H,
@@ -526,7 +590,8 @@ flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, con
   opt.grad_row_scale = reduction == FLCE_REDUCTION_NONE ? grad_row_scale : nullptr;
   opt.row_loss = d_row_loss;
   opt.mean_count = reduction == FLCE_REDUCTION_MEAN ? d_mean_count : nullptr;
-  return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, stream, opt);
+  return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, workspace_bytes, stream,
+                 opt);
 }
 
 size_t flce_ce_workspace_size(int64_t N, int64_t V) {
@@ -619,7 +684,8 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
       cudaMemcpyAsync(d_y, h_y, yb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return FLCE_ERR_CUDA;
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(static_cast<uint8_t*>(workspace) + L.ctrl);
-  s = enqueue(d_X, d_W, d_y, N, H, V, ignore_index, &ctrl->loss, &ctrl->status, d_dX, d_dW, workspace, stream);
+  s = enqueue(d_X, d_W, d_y, N, H, V, ignore_index, &ctrl->loss, &ctrl->status, d_dX, d_dW, workspace,
+              workspace_bytes, stream);
   if (s != FLCE_OK) return s;
   Ctrl host{};
   if (cudaMemcpyAsync(h_dX, d_dX, xb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
@@ -646,7 +712,7 @@ flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out) {
       clusters = sms / CLUSTER;
   }
   const Plan P = make_plan(N, H, V, clusters);
-  out->workspace_bytes = static_cast<int64_t>(ws_layout(N, H).total);
+  out->workspace_bytes = static_cast<int64_t>(ws_total(N, H, V));
   out->vocab_chunk = VC;
   out->num_chunks = P.num_chunks;
   out->lse_splits = P.splits;
@@ -662,6 +728,9 @@ const char* flce_kernel_name(int kind) {
     case KIND_PASS2: return "pass2_grad_dw_dx";
     case KIND_PREP: return "prep_tile_valid";
     case KIND_CE: return "ce_on_logits_rows";
+    case KIND_ORDER: return "prep_row_order";
+    case KIND_SCATTER: return "dx_row_scatter";
+    case KIND_PACK: return "prep_pack_rows";
     default: return "unknown";
   }
 }
@@ -675,6 +744,18 @@ flce_status_t flce_profile_enable(int on) {
   }
   g_prof.on = on != 0;
   g_prof.used = 0;
+  return FLCE_OK;
+}
+
+flce_status_t flce_row_order_info(const void* workspace, int32_t* reordered, int32_t* n_valid,
+                                  cudaStream_t stream) {
+  if (!workspace || !reordered || !n_valid || !aligned(workspace, 256)) return FLCE_ERR_INVALID_ARGUMENT;
+  Ctrl host{};
+  if (cudaMemcpyAsync(&host, workspace, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  *reordered = host.reordered;
+  *n_valid = host.n_rows;
   return FLCE_OK;
 }
 
@@ -735,5 +816,5 @@ extern "C" flce_status_t flce_forward_backward_noalloc(const uint16_t* X, const 
   if (ws_layout(N, H).total > static_cast<size_t>(FLCE_NOALLOC_SCRATCH_BYTES)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   if (noalloc_scratch(&scratch) != cudaSuccess) return FLCE_ERR_CUDA;
-  return flce_forward_backward(X, W, y, N, H, V, ignore_index, loss, dX, dW, scratch, stream);
+  return sync_call(X, W, y, N, H, V, ignore_index, loss, dX, dW, scratch, FLCE_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -85,7 +85,10 @@ __device__ __forceinline__ float row_weight(int reduction, const float* inv_n, c
 }
 
 // Kinds of launch, as the profiler reports them.
-enum : int { KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_PREP = 3, KIND_CE = 4 };
+enum : int {
+  KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_PREP = 3, KIND_CE = 4, KIND_ORDER = 5, KIND_SCATTER = 6,
+  KIND_PACK = 7
+};
 enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
 
 struct GemmArgs {
@@ -110,6 +113,13 @@ struct GemmArgs {
   int reduction;                 // RED_MEAN, RED_SUM, RED_NONE
   const float* grad_row_scale;   // RED_NONE: per-row upstream gradient, or null for 1
   const int* tile_valid;         // [ceil(N/256)] valid rows per 256-row token tile (prep kernel)
+  // Token-row order.  When the rows of ignored targets are scattered, the rows
+  // are reordered so that every valid row comes first (a stable partition);
+  // then perm[r] is the row of X behind row r, the GEMMs read a packed copy of
+  // X in that order (same TMA tiles), and y, the upstream weights and every
+  // output row of the workspace follow the new order.
+  const int* perm;               // [ceil(N/256)*256] row of X behind each row
+  const int* reordered;          // device word: 1 when the rows are reordered
   // pass 2 (one persistent launch over every chunk)
   int TM, HN;             // 256-row token tiles, 256-column hidden tiles
   int C;                  // vocabulary chunks
@@ -322,9 +332,12 @@ __device__ __forceinline__ void epi_zero_tile(uint32_t taddr, int row0, int nb, 
 // fp32-grade sum over the chunks, at the memory cost of one bf16 copy of dX.
 // Each 32-column slice of the warp's rows is read back (hi and lo boxes by TMA,
 // one slice ahead), combined with the accumulator and written back by TMA.
+// The last chunk writes the rounded sum through `mapFinal` (dX itself, or the
+// workspace when the rows are reordered and a scatter puts them in place).
 __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk, bool last_chunk, uint32_t taddr,
                                             int row0, int nb, int row_local, EpiStage& es, const CUtensorMap* mapHi,
-                                            const CUtensorMap* mapLo, volatile int* abort_flag, bool& ok) {
+                                            const CUtensorMap* mapLo, const CUtensorMap* mapFinal,
+                                            volatile int* abort_flag, bool& ok) {
   const int lane = row_local & 31;
   const int wrow0 = row0 + (row_local & ~31);
   const bool accumulate = !first_chunk;
@@ -390,7 +403,7 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk,
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(mapHi, es.addr + b * EPI_BUF_BYTES, nb * BN + c * 32, wrow0, stream);
+      tma_store_2d(last_chunk ? mapFinal : mapHi, es.addr + b * EPI_BUF_BYTES, nb * BN + c * 32, wrow0, stream);
       if (!last_chunk)
         tma_store_2d(mapLo, es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, nb * BN + c * 32, wrow0, stream);
       bulk_commit();
@@ -405,8 +418,8 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk,
 // into a running (max, sum of exponentials) over the vocabulary split of the
 // unit, and picks out the target logit.  No logit leaves the chip.
 __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1)
-    flce_pass1_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
-                      const GemmArgs a) {
+    flce_pass1_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapXc,
+                      const __grid_constant__ CUtensorMap mapW, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   // Same dynamic-smem base in both CTAs, so every offset below matches across the pair.
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -445,8 +458,10 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // X rows in the token-row order: the caller's X, or its packed copy
+  const CUtensorMap* mX = *a.reordered != 0 ? &mapXc : &mapX;
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&mapX);
+    prefetch_tmap(mX);
     prefetch_tmap(&mapW);
   }
   if (warp == 1) {
@@ -482,8 +497,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
               break;
             }
             if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * STAGE_BYTES);
-            load_stage_pass1(&mapX, &mapW, sA(stage), sB(stage), mapa_shared(full_bar(stage), 0), mb, nb, kb,
-                             rank, keep, stream);
+            load_stage_pass1(mX, &mapW, sA(stage), sB(stage), mapa_shared(full_bar(stage), 0), mb, nb, kb, rank,
+                             keep, stream);
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -717,6 +732,7 @@ struct Pass2Maps {
   CUtensorMap Go, DWo;     // epilogue output boxes of G and dW
   CUtensorMap Hio, Loo;    // epilogue boxes of the dX running sum (hi = dX, lo)
   CUtensorMap Hipf, Lopf;  // whole-tile L2 prefetch of the running sum
+  CUtensorMap Xck, Xcmn;   // the packed copy of X (reordered rows), K- and MN-major
 };
 
 __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1)
@@ -758,11 +774,15 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // X rows in the token-row order: the caller's X, or its packed copy
+  const bool reordered = *a.reordered != 0;
+  const CUtensorMap* mXk = reordered ? &m.Xck : &m.Xk;
+  const CUtensorMap* mXmn = reordered ? &m.Xcmn : &m.Xmn;
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&m.Xk);
+    prefetch_tmap(mXk);
     prefetch_tmap(&m.Wk);
     prefetch_tmap(&m.Gmn);
-    prefetch_tmap(&m.Xmn);
+    prefetch_tmap(mXmn);
     prefetch_tmap(&m.Gk);
     prefetch_tmap(&m.Wmn);
   }
@@ -836,7 +856,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
           const uint32_t bar = mapa_shared(full_bar(stage), 0);
           const int k0 = kb * BK;
           if (it.kind == ITEM_GRAD) {
-            tma_load_2d_pair(sA(stage), &m.Xk, bar, k0, m0, keep);
+            tma_load_2d_pair(sA(stage), mXk, bar, k0, m0, keep);
             tma_load_2d_pair(sB(stage), &m.Wk, bar, k0, vbase + n0, normal);
           } else if (it.kind == ITEM_DW) {
 #pragma unroll
@@ -844,7 +864,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
               tma_load_2d_pair(sA(stage) + i * MN_BOX_BYTES, &m.Gmn, bar, m0 + i * 64, k0, normal);
 #pragma unroll
             for (int i = 0; i < BNH / 64; ++i)
-              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, &m.Xmn, bar, n0 + i * 64, k0, keep);
+              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, mXmn, bar, n0 + i * 64, k0, keep);
           } else {
             tma_load_2d_pair(sA(stage), &m.Gk, bar, k0, m0, normal);
 #pragma unroll
@@ -949,6 +969,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     es.addr = smem_u32(es.ptr);
     es.bar = smem_u32(bars + 2 * STAGES + 5 + 2 * q);
     es.k = 0;
+    // the rounded dX goes to the workspace when the rows are reordered
+    const CUtensorMap* dx_final = reordered ? &m.Loo : &m.Hio;
     // with every token ignored the dW contraction has no k-block at all
     bool any_valid = false;
     for (int t = 0; t < a.TM && !any_valid; ++t) any_valid = a.tile_valid[t] != 0;
@@ -995,8 +1017,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         else
           epi_zero_tile(taddr, vbase + row0, it.b, row_local, es, &m.DWo);
       } else {
-        epi_dx_tile(a, it.c == 0, it.c == a.C - 1, taddr, row0, it.b, row_local, es, &m.Hio, &m.Loo, abort_flag,
-                    ok);
+        epi_dx_tile(a, it.c == 0, it.c == a.C - 1, taddr, row0, it.b, row_local, es, &m.Hio, &m.Loo, dx_final,
+                    abort_flag, ok);
         if (!ok) {
           give_up();
           break;
@@ -1054,13 +1076,126 @@ __global__ void __launch_bounds__(CM) flce_prep_kernel(const int32_t* y, int N, 
   if (threadIdx.x == 0) tile_valid[blockIdx.x] = cnt;
 }
 
+// Token-row order for the two passes (one CTA per 256-row tile of y).
+// Ignored rows cost as much as valid ones unless a whole 256-row tile is
+// ignored.  When the valid rows, packed first, fill fewer tiles than the
+// tiles that hold any valid row, the rows are reordered: a stable partition
+// with every valid row first, in their original order, then the ignored rows.
+// Writes the row map `perm`, y and the upstream weights in that order, the
+// per-tile valid counts of the new order, and the decision (`reordered_out`).
+// `allow` = 0 keeps the caller's order (no room for the packed copy of X).
+// Every CTA computes the same totals from `tile_cnt`, so they all decide alike.
+__global__ void __launch_bounds__(CM)
+    flce_row_order_kernel(const int32_t* y, const float* g, int N, int TM, int ignore_index, const int* tile_cnt,
+                          int allow, int* tile_valid, int* perm, int32_t* y_perm, float* g_perm, int* reordered_out,
+                          int* n_rows_out) {
+  const int t = blockIdx.x;
+  int total = 0, nonempty = 0, before = 0;
+  for (int i = threadIdx.x; i < TM; i += CM) {
+    const int c = tile_cnt[i];
+    total += c;
+    nonempty += c > 0 ? 1 : 0;
+    before += i < t ? c : 0;
+  }
+  __shared__ int red[3][CM / 32];
+  __shared__ int wrank[CM / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    total += __shfl_down_sync(0xffffffffu, total, o);
+    nonempty += __shfl_down_sync(0xffffffffu, nonempty, o);
+    before += __shfl_down_sync(0xffffffffu, before, o);
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) {
+    red[0][w] = total;
+    red[1][w] = nonempty;
+    red[2][w] = before;
+  }
+  const int r = t * CM + threadIdx.x;
+  const bool in = r < N;
+  const int yr = in ? y[r] : ignore_index;
+  const bool v = in && yr != ignore_index;
+  const unsigned bal = __ballot_sync(0xffffffffu, v);
+  if (lane == 0) wrank[w] = __popc(bal);
+  __syncthreads();
+  total = nonempty = before = 0;
+  int rank_v = __popc(bal & ((1u << lane) - 1u));
+  for (int i = 0; i < CM / 32; ++i) {
+    total += red[0][i];
+    nonempty += red[1][i];
+    before += red[2][i];
+    rank_v += i < w ? wrank[i] : 0;
+  }
+  const bool reorder = allow != 0 && (total + CM - 1) / CM < nonempty;
+  if (in) {
+    int dest = r;
+    if (reorder) {
+      // ignored rows ahead of this one: those of the (full) earlier tiles plus
+      // those earlier in this tile
+      dest = v ? before + rank_v : total + (t * CM - before) + (static_cast<int>(threadIdx.x) - rank_v);
+    }
+    perm[dest] = r;
+    y_perm[dest] = yr;
+    if (g) g_perm[dest] = g[r];
+  } else {
+    perm[r] = 0;  // padding of the last tile: any in-range row (its outputs are never kept)
+  }
+  if (threadIdx.x == 0) tile_valid[t] = reorder ? max(0, min(CM, total - t * CM)) : tile_cnt[t];
+  if (t == 0 && threadIdx.x == 0) {
+    *reordered_out = reorder ? 1 : 0;
+    *n_rows_out = total;
+  }
+}
+
+// With reordered rows the GEMMs read X through a packed copy in the new order,
+// Xc[r] = X[perm[r]], for every row of the 256-row tiles that hold a valid row
+// (the ignored rows sharing the last such tile included, so that every row the
+// tensor cores read is finite).  One warp per row, 16-byte accesses.
+__global__ void __launch_bounds__(256)
+    flce_pack_rows_kernel(const uint16_t* X, uint16_t* Xc, const int* perm, const int* reordered,
+                          const int* n_rows, int N, int H) {
+  if (*reordered == 0) return;
+  const int rows = min(N, (*n_rows + CM - 1) / CM * CM);
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int h8 = H / 8;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < rows; r += gridDim.x * wpb) {
+    const uint4* sr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(perm[r]) * H);
+    uint4* d = reinterpret_cast<uint4*>(Xc + static_cast<size_t>(r) * H);
+    for (int j = lane; j < h8; j += 32) d[j] = sr[j];
+  }
+}
+
+// With reordered rows the rounded dX sits in the workspace in the new order:
+// put each row back in place and write zeros for the rows of ignored targets
+// (one warp per row, 16-byte accesses; H is a multiple of 8).
+__global__ void __launch_bounds__(256)
+    flce_dx_scatter_kernel(const uint16_t* src, uint16_t* dX, const int* perm, const int* reordered,
+                           const int* n_rows, int N, int H) {
+  if (*reordered == 0) return;
+  const int nr = *n_rows;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int h8 = H / 8;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < N; r += gridDim.x * wpb) {
+    uint4* d = reinterpret_cast<uint4*>(dX + static_cast<size_t>(perm[r]) * H);
+    if (r < nr) {
+      const uint4* sr = reinterpret_cast<const uint4*>(src + static_cast<size_t>(r) * H);
+      for (int j = lane; j < h8; j += 32) d[j] = sr[j];
+    } else {
+      for (int j = lane; j < h8; j += 32) d[j] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
 // ------------------------------------------------------------ combine --
 
 struct CombineArgs {
   int N, V, ignore_index, splits;
   int reduction;
   const float* grad_row_scale;
-  float* row_loss;  // optional per-row losses
+  float* row_loss;  // optional per-row losses, in the caller's row order
+  const int* perm;  // row of the caller behind each row of y, part_m, ... (token-row order)
   const int* mean_count;  // optional: divide the mean by this count instead of n_valid
   const int32_t* y;
   const float* part_m;
@@ -1106,7 +1241,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS) flce_combine_kernel(const Com
         li = a.reduction == RED_NONE && a.grad_row_scale ? row * static_cast<double>(a.grad_row_scale[i]) : row;
       }
     }
-    if (a.row_loss) a.row_loss[i] = static_cast<float>(row);
+    if (a.row_loss) a.row_loss[a.perm[i]] = static_cast<float>(row);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {

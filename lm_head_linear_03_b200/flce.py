@@ -25,7 +25,7 @@ STATUS_NAMES = {
     5: "FLCE_ERR_TIMEOUT",
     6: "FLCE_ERR_CUDA",
 }
-NUM_KERNEL_KINDS = 5
+NUM_KERNEL_KINDS = 8
 
 EXPORTED = (
     "flce_status_string",
@@ -42,6 +42,7 @@ EXPORTED = (
     "flce_ce_workspace_size",
     "flce_cross_entropy",
     "flce_probe_bounded_wait",
+    "flce_row_order_info",
 )
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -107,6 +108,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_probe_bounded_wait.restype = ctypes.c_int
     lib.flce_forward_backward_noalloc.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp, vp]
     lib.flce_forward_backward_noalloc.restype = ctypes.c_int
+    lib.flce_row_order_info.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), vp]
+    lib.flce_row_order_info.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -149,10 +152,32 @@ def plan(N: int, H: int, V: int) -> PlanT:
     return p
 
 
-def alloc_workspace(N: int, H: int, V: int, device=None) -> torch.Tensor:
-    """A uint8 device buffer of flce_workspace_size bytes (torch's allocator
-    hands out 512-B aligned blocks)."""
-    return torch.empty(workspace_size(N, H, V), dtype=torch.uint8, device=device or "cuda")
+def packed_x_bytes(N: int, H: int) -> int:
+    """Size of the workspace area for the packed copy of X: N x H bf16, rounded
+    up to 256 bytes."""
+    return (N * H * 2 + 255) // 256 * 256
+
+
+def alloc_workspace(N: int, H: int, V: int, device=None, reorder: bool | None = None) -> torch.Tensor:
+    """A uint8 device buffer for one call (torch's allocator hands out 512-B
+    aligned blocks): flce_workspace_size bytes by default; with ``reorder`` True
+    the base size plus the N x H bf16 packed-X area whatever V is (so that
+    scattered ignored rows can always be skipped), with False the base size."""
+    if reorder is None:
+        nbytes = workspace_size(N, H, V)
+    else:
+        nbytes = workspace_size(N, H, 1) + (packed_x_bytes(N, H) if reorder else 0)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def row_order_info(workspace: torch.Tensor, stream=None):
+    """(reordered, n_valid) of the last call that used ``workspace``: whether its
+    token rows were reordered (valid rows first, X packed in that order) and
+    how many rows had a non-ignored target.  Waits for ``stream``."""
+    r, n = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load_library().flce_row_order_info(_ptr(workspace), ctypes.byref(r), ctypes.byref(n),
+                                              _stream_handle(stream)), "flce_row_order_info")
+    return bool(r.value), int(n.value)
 
 
 def forward_backward(X, W, y, ignore_index: int = -100, *, dX=None, dW=None, workspace=None, stream=None):

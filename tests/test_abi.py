@@ -51,10 +51,16 @@ def test_status_strings(lib):
     assert lib.flce_status_string(99) == b"FLCE_UNKNOWN_STATUS"
 
 
-def test_workspace_size_independent_of_vocab(lib):
+def test_workspace_size_by_vocab(lib):
     from lm_head_linear_03_b200 import flce
-    sizes = {flce.workspace_size(8192, 4096, v) for v in (1, 2, 4096, 32064, 128256, 256000, 1 << 24)}
-    assert len(sizes) == 1
+    # the base size depends on N and H only; a vocabulary large enough that the
+    # packed-X area (N x H bf16) keeps the whole within 5% of the logits adds it
+    base = flce.workspace_size(8192, 4096, 1)
+    area = 8192 * 4096 * 2
+    for v in (1, 2, 4096, 32064, 128256, 256000, 1 << 24):
+        want = base + area if (base + area) <= 0.05 * 8192 * v * 2 else base
+        assert flce.workspace_size(8192, 4096, v) == want, v
+    assert flce.workspace_size(4096, 2304, 256000) == flce.workspace_size(4096, 2304, 1) + 4096 * 2304 * 2
     # the Llama-3-8B head workload stays within 5% of its N x V x 2-byte logits
     assert flce.workspace_size(8192, 4096, 128256) <= 0.05 * 8192 * 128256 * 2
     assert flce.workspace_size(0, 4096, 10) == 0
@@ -66,7 +72,8 @@ def test_plan_is_host_only(lib):
     p = flce.plan(8192, 4096, 128256)
     assert p.vocab_chunk == 2048 and p.num_chunks == 63
     assert 1 <= p.lse_splits <= 64
-    assert p.launches == 4
+    assert p.launches == 6  # prep, row order, pass 1, combine, pass 2, dX scatter
+    assert flce.plan(4096, 2304, 256000).launches == 7  # and the X pack (packed-X area fits)
 
 
 def test_argument_errors_before_any_launch(lib):
@@ -84,3 +91,30 @@ def test_argument_errors_before_any_launch(lib):
     odd = ctypes.c_void_p((1 << 20) + 8)
     assert lib.flce_forward_backward(odd, fake, fake, i64(8), i64(8), i64(8), -100, ctypes.byref(f),
                                      fake, fake, fake, None) == 2  # misaligned X
+    r, n = ctypes.c_int32(0), ctypes.c_int32(0)
+    assert lib.flce_row_order_info(None, ctypes.byref(r), ctypes.byref(n), None) == 1
+    assert lib.flce_row_order_info(odd, ctypes.byref(r), ctypes.byref(n), None) == 1  # misaligned workspace
+
+
+def _reorder_rule(valid):
+    """The row-order rule as the header states it: reorder when the valid rows,
+    packed first, fill fewer 256-row tiles than the tiles holding a valid row."""
+    import math
+    tiles = [sum(valid[i:i + 256]) for i in range(0, len(valid), 256)]
+    return math.ceil(sum(valid) / 256) < sum(1 for t in tiles if t)
+
+
+def test_row_order_rule_on_the_workloads(lib):
+    """Which of the named workloads take the reordered path with the default
+    workspace: the rule must say so and the packed-X area must fit the 5%
+    budget (host mirror of the device rule; the GPU tests check the device)."""
+    import torch
+    from lm_head_linear_03_b200 import flce
+    from lm_head_linear_03_b200.inputs import WORKLOADS, make_targets
+    expect = {"tiny": False, "llama3_8b_head": False, "long_context": False,
+              "gemma2_large_vocab": True, "phi3_mini_small_vocab": False}
+    for name, want in expect.items():
+        w = WORKLOADS[name]
+        y = make_targets(w, torch.Generator().manual_seed(w.seed))
+        has_area = flce.workspace_size(w.N, w.H, w.V) > flce.workspace_size(w.N, w.H, 1)
+        assert (_reorder_rule((y != -100).tolist()) and has_area) == want, name
