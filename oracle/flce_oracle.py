@@ -45,6 +45,14 @@ weighted sum over valid rows, ``loss = sum_valid s_i l_i`` with
 ``g_i`` ('none', default 1), and ``G_ij = s_i (exp(z_ij - lse_i) - [j == y_i])``
 for valid rows, so that dX and dW are the gradients of that loss.
 
+Vocabulary shards.  Because the loss is computed chunk by chunk over the
+vocabulary (second page above), the chunks may live on different devices: a
+shard of W rows ``[v0, v0 + V_s)`` yields, per row, the log-sum-exp of its own
+logits and the target logit when the target falls inside it
+(:func:`shard_stats`); the log-sum-exp of the shards' values is ``lse_i`` and
+the sum of their target logits is ``z_{i, y_i}`` (:func:`merge_shard_stats`).
+Each shard's columns of G then give its rows of dW in full and its share of dX.
+
 Inputs are converted exactly to fp64 (bf16 -> fp64 is exact).  A matrix product
 (numpy/BLAS in fp64) serves as a step; nothing is blocked, fused or reordered
 beyond what the definition states, except that the functions meant for full-size
@@ -235,3 +243,29 @@ def ce_reference(Z, y, ignore_index: int = IGNORE_INDEX, reduction: str = "mean"
     G[rows, yv] -= 1.0
     G *= s[:, None]
     return loss, G, lse, n, row_loss
+
+
+def shard_stats(X, W_shard, y, v0: int, ignore_index: int = IGNORE_INDEX):
+    """Statistics of one vocabulary shard, W rows ``v0 .. v0 + V_s - 1`` given as
+    ``W_shard``: returns ``(lse_s, zy_s)`` with ``lse_s[i]`` the log-sum-exp of
+    row i's logits over the shard and ``zy_s[i]`` its target logit when
+    ``v0 <= y_i < v0 + V_s`` (0 otherwise, and for ignored rows).  The global
+    range of the targets is the caller's to check."""
+    X = _f64(X)
+    Ws = _f64(W_shard)
+    y = _i64(y)
+    Z = X @ Ws.T                                   # this shard's logits
+    lse_s = log_sum_exp(Z)
+    local = y - v0
+    inside = (y != ignore_index) & (local >= 0) & (local < Ws.shape[0])
+    zy_s = np.where(inside, Z[np.arange(len(y)), np.where(inside, local, 0)], 0.0)
+    return lse_s, zy_s
+
+
+def merge_shard_stats(all_lse, all_zy):
+    """Merges the shards' statistics, arrays ``[shards][N]``: ``lse_i`` is the
+    log-sum-exp over shards of their log-sum-exps (exact: the exponential sums
+    add), and ``z_{i, y_i}`` the sum of their target logits (one shard holds
+    the target).  Returns ``(lse, zy)``."""
+    L = _f64(all_lse)
+    return log_sum_exp(L.T), _f64(all_zy).sum(axis=0)

@@ -293,9 +293,42 @@ def pin_ce_on_logits(orc):
     _close(G.T @ X, dW, 1e-12, atol=1e-16, what="G^T X vs fused dW")
 
 
+def pin_vocab_shards(orc):
+    """Shard statistics and their merge: for a split of the vocabulary into
+    uneven shards (one of a single entry, one holding no target), the merged
+    log-sum-exp equals torch's logsumexp of the explicit fp64 logits, the merged
+    target logit equals z[i, y_i], each shard's own log-sum-exp equals torch's
+    over its columns, and ignored rows or targets outside a shard give 0."""
+    X, W, y = _case(110, 11, 7, 37, n_ign=2)
+    y[3] = 36  # the last vocabulary entry
+    y[5] = 10  # the single-entry shard
+    bounds = [0, 10, 11, 20, 37]
+    y[(y >= 11) & (y < 20)] = 21  # shard [11, 20) holds no target
+    Z = torch.tensor(X) @ torch.tensor(W).T
+    lses, zys = [], []
+    for v0, v1 in zip(bounds[:-1], bounds[1:]):
+        lse_s, zy_s = orc.shard_stats(X, W[v0:v1], y, v0)
+        _close(lse_s, torch.logsumexp(Z[:, v0:v1], dim=1).numpy(), 1e-13, what=f"shard lse [{v0},{v1})")
+        inside = (y != IGN) & (y >= v0) & (y < v1)
+        want = np.where(inside, Z.numpy()[np.arange(len(y)), np.where(inside, y, 0)], 0.0)
+        assert np.array_equal(zy_s, want), f"shard target logits [{v0},{v1})"
+        if v0 == 11:
+            assert not np.any(zy_s), "a shard without targets reports none"
+        lses.append(lse_s)
+        zys.append(zy_s)
+    lse, zy = orc.merge_shard_stats(np.stack(lses), np.stack(zys))
+    _close(lse, torch.logsumexp(Z, dim=1).numpy(), 1e-13, what="merged lse")
+    valid = y != IGN
+    _close(zy[valid], Z.numpy()[np.arange(len(y))[valid], y[valid]], 1e-14, what="merged target logit")
+    assert np.all(zy[~valid] == 0.0)
+    per = torch.nn.functional.cross_entropy(Z, torch.tensor(y), ignore_index=IGN, reduction="none").numpy()
+    _close(np.where(valid, lse - zy, 0.0), per, 1e-12, what="row losses from merged statistics")
+
+
 ALL_PINS = [
     pin_zero_weight, pin_zero_input, pin_two_class, pin_large_logits,
     pin_torch_autograd, pin_finite_difference, pin_rows_of_g_sum_to_zero,
     pin_shift_invariance, pin_ignored_rows, pin_no_valid_rows, pin_target_range,
     pin_permutations, pin_equal_logits, pin_row_functions, pin_reductions, pin_ce_on_logits,
+    pin_vocab_shards,
 ]

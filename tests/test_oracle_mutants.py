@@ -38,6 +38,12 @@ MUTATIONS = [
     ("logit CE: row loss without the target logit", "    row_loss = np.where(valid, lse - Z[rows, yv], 0.0)\n    loss = float((s * row_loss).sum())\n    G = np.exp(Z - lse[:, None])\n    G[rows, yv] -= 1.0\n    G *= s[:, None]\n    return loss, G",
      "    row_loss = np.where(valid, lse, 0.0)\n    loss = float((s * row_loss).sum())\n    G = np.exp(Z - lse[:, None])\n    G[rows, yv] -= 1.0\n    G *= s[:, None]\n    return loss, G"),
     ("target range not checked", "bad = valid & ((y < 0) | (y >= V))", "bad = valid & (y < -10**9)"),
+    ("shard target not shifted by the shard start", "    local = y - v0\n", "    local = y\n"),
+    ("shard target past the shard's end accepted", "(local < Ws.shape[0])", "(local <= Ws.shape[0])"),
+    ("shards merged by max instead of log-sum-exp", "return log_sum_exp(L.T), _f64(all_zy).sum(axis=0)",
+     "return L.max(axis=0), _f64(all_zy).sum(axis=0)"),
+    ("shard target logits averaged", "return log_sum_exp(L.T), _f64(all_zy).sum(axis=0)",
+     "return log_sum_exp(L.T), _f64(all_zy).mean(axis=0)"),
 ]
 
 
