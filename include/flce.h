@@ -166,6 +166,37 @@ flce_status_t flce_forward_backward_ex(const uint16_t* X, const uint16_t* W, con
                                        uint16_t* dW, void* workspace, size_t workspace_bytes,
                                        cudaStream_t stream);
 
+/* Vocabulary-parallel head.  The loss and its gradient are computed in chunks
+ * over the vocabulary ("Liger Kernel explained", section on the cross-entropy
+ * head), so the chunks can live on different devices: rank r holds W rows
+ * [v0, v0 + V_shard) of a V-entry vocabulary as W_shard [V_shard][H], and
+ * every rank holds the same X [N][H] and y [N] (whole-vocabulary ids).  A step
+ * runs as
+ *   1. flce_vp_shard_stats: pass 1 on the shard.  Per row i it writes
+ *      d_shard_lse[i] = log sum_{j in shard} exp(z_ij) and d_shard_zy[i] =
+ *      z_{i,y_i} when v0 <= y_i < v0 + V_shard, else 0 (device fp32 [N]).
+ *   2. the exchange, by the caller (e.g. NCCL all-gather): every rank's two
+ *      vectors, stacked as d_all_lse, d_all_zy [shards][N] (shard order free).
+ *   3. flce_vp_backward: lse_i = log sum_s exp(all_lse[s][i]) and z_{i,y_i} =
+ *      sum_s all_zy[s][i] give the token-mean loss (d_loss, the same on every
+ *      rank) and this shard's G; it writes dW_shard [V_shard][H] complete and
+ *      this shard's part of dX, dX_part [N][H] = G_shard W_shard.
+ *   4. the caller sums dX_part over the ranks (e.g. NCCL all-reduce).
+ * Targets are checked against [0, V); out-of-range ones set
+ * FLCE_ERR_TARGET_OUT_OF_RANGE in d_status.  d_mean_count works as in
+ * flce_forward_backward_ex (mean only).  dX_part and dW_shard may both be NULL
+ * in step 3 for the loss alone.  Rows keep the caller's order (no
+ * reordering); the workspace needs flce_workspace_size(N, H, 1) bytes. */
+flce_status_t flce_vp_shard_stats(const uint16_t* X, const uint16_t* W_shard, const int32_t* y, int64_t N,
+                                  int64_t H, int64_t V_shard, int64_t v0, int64_t V, int32_t ignore_index,
+                                  float* d_shard_lse, float* d_shard_zy, int32_t* d_status, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
+flce_status_t flce_vp_backward(const uint16_t* X, const uint16_t* W_shard, const int32_t* y, int64_t N, int64_t H,
+                               int64_t V_shard, int64_t v0, int64_t V, int32_t ignore_index, int32_t shards,
+                               const float* d_all_lse, const float* d_all_zy, const int32_t* d_mean_count,
+                               float* d_loss, int32_t* d_status, uint16_t* dX_part, uint16_t* dW_shard,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Cross-entropy on a logit tensor the caller already holds, the unfused
  * counterpart of the head ("Complete Guide to Liger Kernel", section
  * LigerCrossEntropyLoss): the same loss, reductions and row losses as

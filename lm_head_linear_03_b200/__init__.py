@@ -18,5 +18,7 @@ from .flce import (  # noqa: F401
     profile_enable,
     profile_read,
     row_order_info,
+    vp_backward,
+    vp_shard_stats,
     workspace_size,
 )

@@ -310,6 +310,17 @@ struct Options {
   const float* grad_row_scale = nullptr;
   float* row_loss = nullptr;
   const int* mean_count = nullptr;
+  // Vocabulary shard: this call's W holds rows [v0, v0 + V) of a vocabulary of
+  // V_total entries (0 = V).  COMBINE_SHARD calls stop after writing the rows'
+  // shard statistics; COMBINE_SHARDS_IN calls take every shard's statistics
+  // instead of running pass 1.
+  int combine = COMBINE_FULL;
+  int64_t v0 = 0, V_total = 0;
+  float* shard_lse = nullptr;
+  float* shard_zy = nullptr;
+  int shards = 0;
+  const float* all_lse = nullptr;
+  const float* all_zy = nullptr;
 };
 
 flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
@@ -324,7 +335,8 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
 
   if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;  // now with max_clusters
   // reordered rows need the packed-X area: only a large enough workspace has it
-  const WsLayout L = ws_layout(N, H, ws_bytes >= ws_layout(N, H, true).total);
+  // (vocabulary shards keep the caller's order: their statistics are per row)
+  const WsLayout L = ws_layout(N, H, opt.combine == COMBINE_FULL && ws_bytes >= ws_layout(N, H, true).total);
   const Plan P = make_plan(N, H, V, di.max_clusters);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
@@ -397,8 +409,9 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     prof_begin(stream, KIND_ORDER, &slot);
     flce_row_order_kernel<<<P.tiles_m, CM, 0, stream>>>(
         y, opt.grad_row_scale, static_cast<int>(N), P.tiles_m, ignore_index,
-        reinterpret_cast<const int*>(ws + L.tile_cnt), L.packed ? 1 : 0, reinterpret_cast<int*>(ws + L.tile_valid),
-        perm, y_perm, g_perm, &ctrl->reordered, &ctrl->n_rows);
+        reinterpret_cast<const int*>(ws + L.tile_cnt), L.packed ? 1 : 0, static_cast<int>(opt.v0),
+        static_cast<int>(V), static_cast<int>(opt.V_total ? opt.V_total : V),
+        reinterpret_cast<int*>(ws + L.tile_valid), perm, y_perm, g_perm, &ctrl->reordered, &ctrl->n_rows, d_status);
     prof_end(stream, slot);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
     if (L.packed) {  // X rows in the new order (returns at once when the order was kept)
@@ -411,8 +424,9 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     }
   }
 
-  // Pass 1: logits tile by tile, online log-sum-exp per (row, split).
-  {
+  // Pass 1: logits tile by tile, online log-sum-exp per (row, split); a call
+  // given every vocabulary shard's statistics has its lse already.
+  if (opt.combine != COMBINE_SHARDS_IN) {
     GemmArgs p1 = a;
     p1.tiles_m = P.tiles_m;
     p1.tiles_n = P.vtiles;
@@ -449,6 +463,12 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     c.grad_row_scale = g_rows;
     c.row_loss = opt.row_loss;
     c.mean_count = opt.mean_count;
+    c.mode = opt.combine;
+    c.shards = opt.shards;
+    c.all_lse = opt.all_lse;
+    c.all_zy = opt.all_zy;
+    c.shard_lse = opt.shard_lse;
+    c.shard_zy = opt.shard_zy;
     const int grid = static_cast<int>((N + COMBINE_THREADS - 1) / COMBINE_THREADS);
     size_t slot;
     prof_begin(stream, KIND_COMBINE, &slot);
@@ -457,8 +477,8 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
   // Pass 2: every chunk's logit recompute, dW and dX tiles in one persistent launch
-  // (skipped for a forward-only call).
-  if (dX != nullptr) {
+  // (skipped for a forward-only call and for a shard's statistics).
+  if (dX != nullptr && opt.combine != COMBINE_SHARD) {
     GemmArgs b = a;
     b.TM = P.tiles_m;
     b.HN = static_cast<int>((H + BN - 1) / BN);
@@ -653,6 +673,59 @@ flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64
   prof_end(stream, slot);
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   return FLCE_OK;
+}
+
+namespace {
+flce_status_t check_shard(int64_t V_shard, int64_t v0, int64_t V) {
+  if (v0 < 0 || V <= 0 || V > (1ll << 30) || v0 + V_shard > V) return FLCE_ERR_INVALID_ARGUMENT;
+  return FLCE_OK;
+}
+}  // namespace
+
+flce_status_t flce_vp_shard_stats(const uint16_t* X, const uint16_t* W_shard, const int32_t* y, int64_t N,
+                                  int64_t H, int64_t V_shard, int64_t v0, int64_t V, int32_t ignore_index,
+                                  float* d_shard_lse, float* d_shard_zy, int32_t* d_status, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream) {
+  if (!d_shard_lse || !d_shard_zy || !d_status) return FLCE_ERR_INVALID_ARGUMENT;
+  flce_status_t s = check_args(X, W_shard, y, N, H, V_shard, nullptr, nullptr, workspace, true);
+  if (s == FLCE_OK) s = check_shard(V_shard, v0, V);
+  if (s != FLCE_OK) return s;
+  if (!aligned(d_shard_lse, 4) || !aligned(d_shard_zy, 4) || !aligned(d_status, 4)) return FLCE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  Options opt;
+  opt.combine = COMBINE_SHARD;
+  opt.v0 = v0;
+  opt.V_total = V;
+  opt.shard_lse = d_shard_lse;
+  opt.shard_zy = d_shard_zy;
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(workspace);  // the loss slot is unused by this step
+  return enqueue(X, W_shard, y, N, H, V_shard, ignore_index, &ctrl->loss, d_status, nullptr, nullptr, workspace,
+                 workspace_bytes, stream, opt);
+}
+
+flce_status_t flce_vp_backward(const uint16_t* X, const uint16_t* W_shard, const int32_t* y, int64_t N, int64_t H,
+                               int64_t V_shard, int64_t v0, int64_t V, int32_t ignore_index, int32_t shards,
+                               const float* d_all_lse, const float* d_all_zy, const int32_t* d_mean_count,
+                               float* d_loss, int32_t* d_status, uint16_t* dX_part, uint16_t* dW_shard,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!d_all_lse || !d_all_zy || !d_loss || !d_status || shards < 1) return FLCE_ERR_INVALID_ARGUMENT;
+  flce_status_t s = check_args(X, W_shard, y, N, H, V_shard, dX_part, dW_shard, workspace, true);
+  if (s == FLCE_OK) s = check_shard(V_shard, v0, V);
+  if (s != FLCE_OK) return s;
+  if (!aligned(d_all_lse, 4) || !aligned(d_all_zy, 4) || !aligned(d_loss, 4) || !aligned(d_status, 4) ||
+      !aligned(d_mean_count, 4))
+    return FLCE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  Options opt;
+  opt.combine = COMBINE_SHARDS_IN;
+  opt.v0 = v0;
+  opt.V_total = V;
+  opt.shards = shards;
+  opt.all_lse = d_all_lse;
+  opt.all_zy = d_all_zy;
+  opt.mean_count = d_mean_count;
+  return enqueue(X, W_shard, y, N, H, V_shard, ignore_index, d_loss, d_status, dX_part, dW_shard, workspace,
+                 workspace_bytes, stream, opt);
 }
 
 flce_status_t flce_probe_bounded_wait(int64_t timeout_ns, int32_t* d_status, cudaStream_t stream) {

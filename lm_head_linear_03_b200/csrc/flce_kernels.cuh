@@ -84,6 +84,12 @@ __device__ __forceinline__ float row_weight(int reduction, const float* inv_n, c
   return grad_row_scale ? grad_row_scale[row] : 1.f;
 }
 
+// Target of a valid row whose vocabulary entry lies in another shard: far
+// above any column index, and never equal to ignore_index.
+__host__ __device__ __forceinline__ int target_elsewhere(int ignore_index) {
+  return ignore_index == 0x7fffffff ? 0x7ffffffe : 0x7fffffff;
+}
+
 // Kinds of launch, as the profiler reports them.
 enum : int {
   KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_PREP = 3, KIND_CE = 4, KIND_ORDER = 5, KIND_SCATTER = 6,
@@ -1085,10 +1091,13 @@ __global__ void __launch_bounds__(CM) flce_prep_kernel(const int32_t* y, int N, 
 // per-tile valid counts of the new order, and the decision (`reordered_out`).
 // `allow` = 0 keeps the caller's order (no room for the packed copy of X).
 // Every CTA computes the same totals from `tile_cnt`, so they all decide alike.
+// Targets are checked against the whole vocabulary [0, V_total) and stored
+// relative to this call's W rows [v0, v0 + V): a target outside them (held by
+// another vocabulary shard) becomes TARGET_ELSEWHERE, which no column matches.
 __global__ void __launch_bounds__(CM)
     flce_row_order_kernel(const int32_t* y, const float* g, int N, int TM, int ignore_index, const int* tile_cnt,
-                          int allow, int* tile_valid, int* perm, int32_t* y_perm, float* g_perm, int* reordered_out,
-                          int* n_rows_out) {
+                          int allow, int v0, int V, int V_total, int* tile_valid, int* perm, int32_t* y_perm,
+                          float* g_perm, int* reordered_out, int* n_rows_out, int* status) {
   const int t = blockIdx.x;
   int total = 0, nonempty = 0, before = 0;
   for (int i = threadIdx.x; i < TM; i += CM) {
@@ -1127,6 +1136,8 @@ __global__ void __launch_bounds__(CM)
     rank_v += i < w ? wrank[i] : 0;
   }
   const bool reorder = allow != 0 && (total + CM - 1) / CM < nonempty;
+  if (v && (yr < 0 || yr >= V_total)) raise_status(status, ST_TARGET_OUT_OF_RANGE);
+  const int yl = !v ? ignore_index : (yr >= v0 && yr - v0 < V) ? yr - v0 : target_elsewhere(ignore_index);
   if (in) {
     int dest = r;
     if (reorder) {
@@ -1135,7 +1146,7 @@ __global__ void __launch_bounds__(CM)
       dest = v ? before + rank_v : total + (t * CM - before) + (static_cast<int>(threadIdx.x) - rank_v);
     }
     perm[dest] = r;
-    y_perm[dest] = yr;
+    y_perm[dest] = yl;
     if (g) g_perm[dest] = g[r];
   } else {
     perm[r] = 0;  // padding of the last tile: any in-range row (its outputs are never kept)
@@ -1190,8 +1201,21 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------ combine --
 
+// What the combine kernel does with the rows' statistics.
+enum : int {
+  COMBINE_FULL = 0,      // merge the pass-1 splits: lse, loss, 1/n
+  COMBINE_SHARD = 1,     // merge the splits into this vocabulary shard's (lse, target logit) per row, no loss
+  COMBINE_SHARDS_IN = 2  // lse and target logit from every shard's statistics, then loss and 1/n
+};
+
 struct CombineArgs {
   int N, V, ignore_index, splits;
+  int mode;                // COMBINE_*
+  int shards;              // COMBINE_SHARDS_IN: number of shards in all_lse / all_zy
+  const float* all_lse;    // [shards][N] per-shard log-sum-exp (natural log)
+  const float* all_zy;     // [shards][N] per-shard target logit (0 outside the shard)
+  float* shard_lse;        // COMBINE_SHARD outputs, [N] each
+  float* shard_zy;
   int reduction;
   const float* grad_row_scale;
   float* row_loss;  // optional per-row losses, in the caller's row order
@@ -1216,32 +1240,56 @@ constexpr int COMBINE_THREADS = 256;
 // Merges the per-split (max, sum) pairs of each row into its log-sum-exp, forms
 // the row loss lse_i - z_{i,y_i} for valid rows and reduces the token mean.
 // Deterministic: a fixed tree inside each block, then the last block to finish
-// adds the block sums in block order, in fp64.
+// adds the block sums in block order, in fp64.  (The target range was checked
+// by the row-order kernel.)
+// A vocabulary shard's call (COMBINE_SHARD) stops after writing its rows'
+// (lse, target logit); the call after the exchange (COMBINE_SHARDS_IN) takes
+// lse_i as the log-sum-exp of every shard's lse and z_{i,y_i} as the sum of
+// their target logits, then goes on as the full head does.
 __global__ void __launch_bounds__(COMBINE_THREADS) flce_combine_kernel(const CombineArgs a) {
   const int i = blockIdx.x * COMBINE_THREADS + threadIdx.x;
   double li = 0.0;
   int vi = 0;
   if (i < a.N) {
-    float M = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_m[static_cast<size_t>(s) * a.N + i]);
-    float L = 0.f;
-    for (int s = 0; s < a.splits; ++s)
-      L += a.part_l[static_cast<size_t>(s) * a.N + i] * exp2f(a.part_m[static_cast<size_t>(s) * a.N + i] - M);
-    const float l2 = M + log2f(L);
-    a.lse2[i] = l2;
     const int yi = a.y[i];
-    double row = 0.0;
-    if (yi != a.ignore_index) {
-      if (yi < 0 || yi >= a.V) {
-        raise_status(a.status, ST_TARGET_OUT_OF_RANGE);
-      } else {
-        row = static_cast<double>(l2) * LN2 - static_cast<double>(a.zy[i]);
-        vi = 1;
-        // mean and sum add the plain row losses (the mean divides at the end)
-        li = a.reduction == RED_NONE && a.grad_row_scale ? row * static_cast<double>(a.grad_row_scale[i]) : row;
+    const bool valid = yi != a.ignore_index;
+    float l2, zyi;
+    if (a.mode == COMBINE_SHARDS_IN) {
+      float M = -INFINITY;
+      for (int s = 0; s < a.shards; ++s) M = fmaxf(M, a.all_lse[static_cast<size_t>(s) * a.N + i]);
+      float S = 0.f;
+      zyi = 0.f;
+      for (int s = 0; s < a.shards; ++s) {
+        S += expf(a.all_lse[static_cast<size_t>(s) * a.N + i] - M);
+        zyi += a.all_zy[static_cast<size_t>(s) * a.N + i];
       }
+      l2 = (M + logf(S)) * LOG2E;
+    } else {
+      float M = -INFINITY;
+      for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_m[static_cast<size_t>(s) * a.N + i]);
+      float L = 0.f;
+      for (int s = 0; s < a.splits; ++s)
+        L += a.part_l[static_cast<size_t>(s) * a.N + i] * exp2f(a.part_m[static_cast<size_t>(s) * a.N + i] - M);
+      l2 = M + log2f(L);
+      zyi = a.zy[i];
+    }
+    if (a.mode == COMBINE_SHARD) {
+      // zy holds a value only for rows whose target this shard holds
+      a.shard_lse[a.perm[i]] = static_cast<float>(static_cast<double>(l2) * LN2);
+      a.shard_zy[a.perm[i]] = valid && yi >= 0 && yi < a.V ? zyi : 0.f;
+      return;
+    }
+    a.lse2[i] = l2;
+    double row = 0.0;
+    if (valid) {
+      row = static_cast<double>(l2) * LN2 - static_cast<double>(zyi);
+      vi = 1;
+      // mean and sum add the plain row losses (the mean divides at the end)
+      li = a.reduction == RED_NONE && a.grad_row_scale ? row * static_cast<double>(a.grad_row_scale[i]) : row;
     }
     if (a.row_loss) a.row_loss[a.perm[i]] = static_cast<float>(row);
+  } else if (a.mode == COMBINE_SHARD) {
+    return;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {

@@ -43,6 +43,8 @@ EXPORTED = (
     "flce_cross_entropy",
     "flce_probe_bounded_wait",
     "flce_row_order_info",
+    "flce_vp_shard_stats",
+    "flce_vp_backward",
 )
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -110,6 +112,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_forward_backward_noalloc.restype = ctypes.c_int
     lib.flce_row_order_info.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), vp]
     lib.flce_row_order_info.restype = ctypes.c_int
+    lib.flce_vp_shard_stats.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i32, vp, vp, vp, vp, sz, vp]
+    lib.flce_vp_shard_stats.restype = ctypes.c_int
+    lib.flce_vp_backward.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                     vp, sz, vp]
+    lib.flce_vp_backward.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -249,6 +256,56 @@ def forward_backward_ex(X, W, y, ignore_index: int = -100, *, reduction: str = "
                                       vp(dW), _ptr(workspace), workspace.numel(), _stream_handle(stream))
     _check(st, "flce_forward_backward_ex")
     return loss, status, rl, dX, dW
+
+
+def vp_shard_stats(X, W_shard, y, v0: int, V: int, ignore_index: int = -100, *, workspace=None, stream=None):
+    """Step 1 of the vocabulary-parallel head on this rank's shard, W rows
+    ``[v0, v0 + W_shard.shape[0])`` of a ``V``-entry vocabulary.  Returns device
+    tensors (shard_lse[N], shard_zy[N], status[1]) without waiting."""
+    lib = load_library()
+    _check_inputs(X, W_shard, y)
+    N, H = X.shape
+    Vs = W_shard.shape[0]
+    dev = X.device
+    lse = torch.empty(N, dtype=torch.float32, device=dev)
+    zy = torch.empty(N, dtype=torch.float32, device=dev)
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    workspace = alloc_workspace(N, H, 1, dev) if workspace is None else workspace
+    st = lib.flce_vp_shard_stats(_ptr(X), _ptr(W_shard), _ptr(y), N, H, Vs, v0, V, ignore_index, _ptr(lse), _ptr(zy),
+                                 _ptr(status), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(st, "flce_vp_shard_stats")
+    return lse, zy, status
+
+
+def vp_backward(X, W_shard, y, v0: int, V: int, all_lse, all_zy, ignore_index: int = -100, *, mean_count=None,
+                grads: bool = True, workspace=None, stream=None):
+    """Step 3 of the vocabulary-parallel head: every shard's statistics
+    (``all_lse``, ``all_zy``: float32 [shards][N]) give the loss; returns device
+    tensors (loss[1], status[1], dX_part or None, dW_shard or None) without
+    waiting.  dX_part is this shard's share of dX (sum it over the ranks)."""
+    lib = load_library()
+    _check_inputs(X, W_shard, y)
+    N, H = X.shape
+    Vs = W_shard.shape[0]
+    dev = X.device
+    for t in (all_lse, all_zy):
+        if t.dtype != torch.float32 or not t.is_cuda or t.dim() != 2 or t.shape[1] != N or not t.is_contiguous():
+            raise ValueError("all_lse / all_zy must be contiguous CUDA float32 tensors of shape [shards, N]")
+    if all_lse.shape != all_zy.shape:
+        raise ValueError("all_lse and all_zy differ in shape")
+    if mean_count is not None and (mean_count.dtype != torch.int32 or not mean_count.is_cuda):
+        raise ValueError("mean_count must be a CUDA int32 tensor")
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    dX = torch.empty_like(X) if grads else None
+    dW = torch.empty_like(W_shard) if grads else None
+    workspace = alloc_workspace(N, H, 1, dev) if workspace is None else workspace
+    vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
+    st = lib.flce_vp_backward(_ptr(X), _ptr(W_shard), _ptr(y), N, H, Vs, v0, V, ignore_index, all_lse.shape[0],
+                              _ptr(all_lse), _ptr(all_zy), vp(mean_count), _ptr(loss), _ptr(status), vp(dX), vp(dW),
+                              _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(st, "flce_vp_backward")
+    return loss, status, dX, dW
 
 
 def cross_entropy(logits, y, ignore_index: int = -100, *, reduction: str = "mean", grad_row_scale=None,

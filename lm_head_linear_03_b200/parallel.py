@@ -1,4 +1,7 @@
-"""Data-parallel use of the head: token rows sharded over ranks, W replicated.
+"""Multi-device use of the head: data-parallel over tokens, or vocabulary-parallel.
+
+Data-parallel (:func:`dp_forward_backward`): token rows sharded over ranks, W
+replicated.
 
 Rows are independent once the mean's denominator is known, so each rank runs
 the fused head on its own tokens with the mean taken over the valid targets of
@@ -6,6 +9,13 @@ the fused head on its own tokens with the mean taken over the valid targets of
 the batch dW, while each rank's dX is already final for its rows.  The
 exchanges are one all-reduce of the count (before the call) and all-reduces of
 the loss and dW (after it), through torch.distributed (NCCL on GPUs).
+
+Vocabulary-parallel (:func:`vp_forward_backward`): W rows sharded over ranks in
+contiguous ranges, X and y replicated.  The loss is computed chunk by chunk
+over the vocabulary, so each rank reduces its own chunk to per-row statistics
+(log-sum-exp, target logit); one all-gather of those two N-vectors gives every
+rank the global log-sum-exp, after which its dW rows are complete and its dX is
+a share that one all-reduce sums.
 """
 from __future__ import annotations
 
@@ -37,4 +47,52 @@ def dp_forward_backward(X, W, y, ignore_index: int = -100, *, group=None, local_
         raise FlceError(int(bad.item()), "dp_forward_backward")
     dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=group)
     dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=group)
+    return loss, dX, dW
+
+
+def _vp_stats_call(X, W_shard, y, v0, V, ignore_index):
+    from .flce import vp_shard_stats
+    return vp_shard_stats(X, W_shard, y, v0, V, ignore_index)
+
+
+def _vp_backward_call(X, W_shard, y, v0, V, all_lse, all_zy, ignore_index):
+    from .flce import vp_backward
+    return vp_backward(X, W_shard, y, v0, V, all_lse, all_zy, ignore_index)
+
+
+def vocab_shard_range(V: int, world: int, rank: int):
+    """The contiguous W rows ``[v0, v1)`` rank ``rank`` of ``world`` holds: the
+    vocabulary split as evenly as possible, the first ``V % world`` shards one
+    row longer."""
+    base, extra = divmod(V, world)
+    v0 = rank * base + min(rank, extra)
+    return v0, v0 + base + (1 if rank < extra else 0)
+
+
+def vp_forward_backward(X, W_shard, y, v0: int, V: int, ignore_index: int = -100, *, group=None,
+                        stats_call=None, backward_call=None):
+    """Returns (loss, dX, dW_shard) on every rank of ``group`` for a vocabulary
+    split into contiguous shards; this rank holds W rows ``[v0, v0 + V_s)``.
+
+    ``stats_call(X, W_shard, y, v0, V, ignore_index) -> (lse[N], zy[N], status[1])``
+    and ``backward_call(X, W_shard, y, v0, V, all_lse, all_zy, ignore_index) ->
+    (loss[1], status[1], dX_part, dW_shard)`` default to the CUDA library.
+    """
+    stats = stats_call or _vp_stats_call
+    back = backward_call or _vp_backward_call
+    world = dist.get_world_size(group)
+    lse, zy, st1 = stats(X, W_shard, y, v0, V, ignore_index)
+    both = torch.stack([lse, zy])                                   # [2, N]
+    gathered = [torch.empty_like(both) for _ in range(world)]
+    dist.all_gather(gathered, both, group=group)
+    allst = torch.stack(gathered)                                   # [world, 2, N]
+    all_lse = allst[:, 0].contiguous()
+    all_zy = allst[:, 1].contiguous()
+    loss, st2, dX, dW = back(X, W_shard, y, v0, V, all_lse, all_zy, ignore_index)
+    bad = torch.maximum(st1.to(torch.int32).reshape(1), st2.to(torch.int32).reshape(1)).clone()
+    dist.all_reduce(bad, op=dist.ReduceOp.MAX, group=group)
+    if int(bad.item()) != 0:
+        from .flce import FlceError
+        raise FlceError(int(bad.item()), "vp_forward_backward")
+    dist.all_reduce(dX, op=dist.ReduceOp.SUM, group=group)
     return loss, dX, dW

@@ -93,6 +93,12 @@ def test_argument_errors_before_any_launch(lib):
                                      fake, fake, fake, None) == 2  # misaligned X
     r, n = ctypes.c_int32(0), ctypes.c_int32(0)
     assert lib.flce_row_order_info(None, ctypes.byref(r), ctypes.byref(n), None) == 1
+    # vocabulary shards: a shard reaching past the vocabulary, or no statistics
+    lib.flce_vp_shard_stats.restype = ctypes.c_int
+    assert lib.flce_vp_shard_stats(fake, fake, fake, i64(8), i64(8), i64(8), i64(5), i64(10), -100, fake, fake, fake,
+                                   fake, ctypes.c_size_t(1 << 30), None) == 1
+    assert lib.flce_vp_backward(fake, fake, fake, i64(8), i64(8), i64(8), i64(0), i64(10), -100, 2, None, fake,
+                                None, fake, fake, fake, fake, fake, ctypes.c_size_t(1 << 30), None) == 1
     assert lib.flce_row_order_info(odd, ctypes.byref(r), ctypes.byref(n), None) == 1  # misaligned workspace
 
 
