@@ -1418,8 +1418,11 @@ __global__ void __launch_bounds__(CE_THREADS) flce_ce_rows_kernel(const CeArgs a
     if (tid == 0 && yi != a.ignore_index && !in_range) raise_status(a.status, ST_TARGET_OUT_OF_RANGE);
     if (tid == 0) s_zy = 0.f;
     __syncthreads();
-    // ---- online max and sum of 2^(z log2 e) over the row
+    // ---- online max and sum of 2^(z log2 e) over the row.  The row is read
+    // again for the gradient: keep it in L2 (evict_last) until then; the
+    // second read and the gradient stores are its last touch (evict_first).
     float m = -1e30f, l = 0.f;
+    const uint64_t keep = l2_evict_last(), last = l2_evict_first();
     if (vec) {
       const uint4* zv = reinterpret_cast<const uint4*>(z);
       const int nv = a.V >> 3;
@@ -1429,7 +1432,7 @@ __global__ void __launch_bounds__(CE_THREADS) flce_ce_rows_kernel(const CeArgs a
 #pragma unroll
         for (int u = 0; u < CE_UNROLL; ++u) {
           const int j = base + u * CE_THREADS;
-          buf[u] = j < nv ? zv[j] : make_uint4(0, 0, 0, 0);
+          buf[u] = j < nv ? ld_l2hint_v4(zv + j, keep) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < CE_UNROLL; ++u) {
@@ -1503,7 +1506,7 @@ __global__ void __launch_bounds__(CE_THREADS) flce_ce_rows_kernel(const CeArgs a
 #pragma unroll
           for (int u = 0; u < CE_UNROLL; ++u) {
             const int j = base + u * CE_THREADS;
-            buf[u] = (j < nv && valid) ? zv[j] : make_uint4(0, 0, 0, 0);
+            buf[u] = (j < nv && valid) ? ld_l2hint_v4(zv + j, last) : make_uint4(0, 0, 0, 0);
           }
 #pragma unroll
           for (int u = 0; u < CE_UNROLL; ++u) {
@@ -1516,8 +1519,10 @@ __global__ void __launch_bounds__(CE_THREADS) flce_ce_rows_kernel(const CeArgs a
               for (int e = 0; e < 8; ++e)
                 o[e] = valid ? ex2_approx(fmaf(f[e], LOG2E, -l2r)) * sc : 0.f;
               if (valid && static_cast<unsigned>(yi - 8 * j) < 8u) o[yi - 8 * j] -= sc;
-              gv[j] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                                 pack_bf16x2(o[6], o[7]));
+              st_l2hint_v4(gv + j,
+                           make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                      pack_bf16x2(o[6], o[7])),
+                           last);
             }
           }
         }

@@ -120,6 +120,22 @@ __device__ __forceinline__ uint64_t l2_evict_normal() {
   return p;
 }
 
+// 16-byte global load / store that bypasses L1 and carries an L2 residency
+// policy (createpolicy): lets a streaming kernel keep what it reads again and
+// push out what it touches for the last time.
+__device__ __forceinline__ uint4 ld_l2hint_v4(const uint4* p, uint64_t policy) {
+  uint4 v;
+  asm volatile("ld.global.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
+__device__ __forceinline__ void st_l2hint_v4(uint4* p, uint4 v, uint64_t policy) {
+  asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy)
+               : "memory");
+}
+
 // Tile load issued by either CTA of an SM pair; the bytes are counted on the
 // mbarrier at `bar_cluster`, which may be the pair leader's.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
