@@ -38,7 +38,8 @@
  * allocates device memory: scratch space is the caller's `workspace`, at least
  * flce_workspace_size(N, H, V) bytes (at least the base size, see there).  dX
  * and dW are overwritten, not accumulated into.  The library keeps only
- * read-only host caches (device properties, a driver entry point).
+ * read-only host caches (device properties, a driver entry point) and, for
+ * the host-buffer entry, one copy stream with a few events per device.
  *
  * Errors.  Argument errors are found on the host and returned before anything
  * is launched.  Errors found on the device (a valid target outside [0, V), a
@@ -123,7 +124,14 @@ flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, 
  *   d_X, d_W, d_y, d_dX, d_dW, workspace: caller-owned device buffers of the
  *   same shapes (workspace >= flce_workspace_size bytes)
  * Copies the inputs to the device, runs the computation, copies loss, dX and
- * dW back, and waits for the stream.  No allocation happens inside. */
+ * dW back, and waits for the stream.  No allocation happens inside.  The
+ * copies overlap the kernels: W goes over in pieces on an internal copy stream
+ * and pass 1 runs piece by piece as they land; pass 2 runs in sections of
+ * whole vocabulary chunks and each section's finished dW rows come back while
+ * the next one computes.  Results agree with flce_forward_backward's to
+ * rounding (the log-sum-exp partials are merged in another order).  The copy
+ * stream and its events are made on first use, one set per device, and kept;
+ * host-buffer calls on one device run one at a time. */
 flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_W,
                                          const int32_t* h_y, int64_t N, int64_t H, int64_t V,
                                          int32_t ignore_index, float* h_loss, uint16_t* h_dX,

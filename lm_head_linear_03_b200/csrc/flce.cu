@@ -305,6 +305,50 @@ flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N,
 }
 
 // --------------------------------------------------------------- enqueue --
+// Host-buffer calls overlap the PCIe copies with the kernels: W arrives in
+// pieces on a copy stream and pass 1 runs piece by piece as they land; pass 2
+// runs as a few launches over consecutive chunk sections of its item queue,
+// and each section's finished dW rows go back on the copy stream while the
+// next section computes.
+constexpr int MAX_PIECES = 8;
+struct PipeCtx {
+  cudaStream_t copy = nullptr;
+  int pieces = 0;                      // W pieces = pass-1 launches
+  int64_t piece_v[MAX_PIECES + 1] = {};  // vocabulary rows [piece_v[i], piece_v[i+1]), multiples of BN
+  cudaEvent_t w_ready[MAX_PIECES] = {};  // recorded on `copy` after piece i's copy
+  int groups = 0;                      // pass-2 launches
+  cudaEvent_t p2_done[MAX_PIECES] = {};
+  uint16_t* h_dW = nullptr;            // host dW, filled group by group on `copy`
+};
+
+// Per-device copy stream and events of the host-buffer entry, made on first
+// use and kept (like the device-property cache) for the life of the process.
+struct PipeRes {
+  std::mutex mu;
+  cudaStream_t copy = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t ev[2 * MAX_PIECES] = {};
+};
+PipeRes g_pipe[64];
+
+cudaError_t pipe_resources(PipeRes** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  PipeRes& r = g_pipe[dev];
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (r.copy == nullptr) {
+    if ((e = cudaStreamCreateWithFlags(&r.copy, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.start, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.done, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (auto& ev : r.ev)
+      if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  *out = &r;
+  return cudaSuccess;
+}
+
 struct Options {
   int reduction = RED_MEAN;
   const float* grad_row_scale = nullptr;
@@ -321,6 +365,7 @@ struct Options {
   int shards = 0;
   const float* all_lse = nullptr;
   const float* all_zy = nullptr;
+  const PipeCtx* pipe = nullptr;  // host-buffer call: pieces of pass 1, sections of pass 2
 };
 
 flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
@@ -426,7 +471,8 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
 
   // Pass 1: logits tile by tile, online log-sum-exp per (row, split); a call
   // given every vocabulary shard's statistics has its lse already.
-  if (opt.combine != COMBINE_SHARDS_IN) {
+  int total_splits = P.splits;
+  if (opt.combine != COMBINE_SHARDS_IN && opt.pipe == nullptr) {
     GemmArgs p1 = a;
     p1.tiles_m = P.tiles_m;
     p1.tiles_n = P.vtiles;
@@ -438,6 +484,32 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     flce_pass1_kernel<<<CLUSTER * P.lse_clusters, NUM_THREADS, P1_SMEM_BYTES, stream>>>(mX_k, mXc_k, mW_k, p1);
     prof_end(stream, slot);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  } else if (opt.combine != COMBINE_SHARDS_IN) {
+    // one launch per W piece, after its copy; its splits fill the next partial slots
+    const PipeCtx& pp = *opt.pipe;
+    total_splits = 0;
+    for (int i = 0; i < pp.pieces; ++i) {
+      const int64_t v0 = pp.piece_v[i], vp = pp.piece_v[i + 1] - pp.piece_v[i];
+      CUtensorMap mWp;
+      if (!make_map(&mWp, W + v0 * H, h, static_cast<uint64_t>(vp), h * 2, BK, BNH)) return FLCE_ERR_CUDA;
+      GemmArgs p1 = a;
+      p1.V = static_cast<int>(vp);
+      p1.v_off = static_cast<int>(v0);
+      p1.split_off = total_splits;
+      p1.tiles_m = P.tiles_m;
+      p1.tiles_n = static_cast<int>((vp + BN - 1) / BN);
+      p1.k_blocks = static_cast<int>((H + BK - 1) / BK);
+      p1.splits = std::min(choose_splits(P.tiles_m, p1.tiles_n, P.clusters), MAX_SPLITS / pp.pieces);
+      p1.num_units = P.tiles_m * p1.splits;
+      total_splits += p1.splits;
+      const int grid = static_cast<int>(std::min<long long>(p1.num_units, P.clusters));
+      if (cudaStreamWaitEvent(stream, pp.w_ready[i], 0) != cudaSuccess) return FLCE_ERR_CUDA;
+      size_t slot;
+      prof_begin(stream, KIND_LSE, &slot);
+      flce_pass1_kernel<<<CLUSTER * grid, NUM_THREADS, P1_SMEM_BYTES, stream>>>(mX_k, mXc_k, mWp, p1);
+      prof_end(stream, slot);
+      if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    }
   }
   // Combine the splits: lse, loss, n_valid, 1/n.
   {
@@ -445,7 +517,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     c.N = static_cast<int>(N);
     c.V = static_cast<int>(V);
     c.ignore_index = ignore_index;
-    c.splits = P.splits;
+    c.splits = total_splits;
     c.y = y_perm;
     c.perm = perm;
     c.part_m = part_m;
@@ -486,11 +558,14 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     b.VTf = VC / BN;
     b.VT_last = static_cast<int>((V - static_cast<int64_t>(P.num_chunks - 1) * VC + BN - 1) / BN);
     if (b.C == 1) b.VTf = b.VT_last;
+    // section_end[c]: end of the queue's section c (dX(c) dW(c) G(c+1)), after G(0)
+    std::vector<long long> section_end(b.C);
     long long total = static_cast<long long>(b.C == 1 ? b.VT_last : b.VTf) * b.TM;  // G(0)
     for (int c = 0; c < b.C; ++c) {
       const long long vt = c == b.C - 1 ? b.VT_last : b.VTf;
       total += static_cast<long long>(b.TM) * b.HN + vt * b.HN;
       if (c + 1 < b.C) total += static_cast<long long>(c + 1 == b.C - 1 ? b.VT_last : b.VTf) * b.TM;
+      section_end[c] = total;
     }
     b.total_items = total;
     int* ctr = reinterpret_cast<int*>(ws + L.counters);
@@ -513,12 +588,30 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     pm.Lopf = mLo;
     pm.Xck = mXc_k;
     pm.Xcmn = mXc_mn;
-    const int grid = static_cast<int>(std::min<long long>(total, P.clusters));
+    // one launch over the whole queue; a host-buffer call splits it into
+    // sections of whole chunks and sends each section's dW rows back
+    const int groups = opt.pipe ? std::max(1, std::min(opt.pipe->groups, b.C)) : 1;
     size_t slot;
-    prof_begin(stream, KIND_PASS2, &slot);
-    flce_pass2_kernel<<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, stream>>>(pm, b);
-    prof_end(stream, slot);
-    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    for (int k = 0; k < groups; ++k) {
+      const int c0 = static_cast<int>(static_cast<long long>(k) * b.C / groups);
+      const int c1 = static_cast<int>(static_cast<long long>(k + 1) * b.C / groups);
+      b.item_begin = k == 0 ? 0 : section_end[c0 - 1];
+      b.item_end = section_end[c1 - 1];
+      const int grid = static_cast<int>(std::min<long long>(b.item_end - b.item_begin, P.clusters));
+      prof_begin(stream, KIND_PASS2, &slot);
+      flce_pass2_kernel<<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, stream>>>(pm, b);
+      prof_end(stream, slot);
+      if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+      if (opt.pipe) {  // dW rows of chunks c0 .. c1-1 are final
+        const PipeCtx& pp = *opt.pipe;
+        const int64_t r0 = static_cast<int64_t>(c0) * VC, r1 = std::min<int64_t>(V, static_cast<int64_t>(c1) * VC);
+        if (cudaEventRecord(pp.p2_done[k], stream) != cudaSuccess ||
+            cudaStreamWaitEvent(pp.copy, pp.p2_done[k], 0) != cudaSuccess ||
+            cudaMemcpyAsync(pp.h_dW + r0 * H, dW + r0 * H, static_cast<size_t>(r1 - r0) * H * 2,
+                            cudaMemcpyDeviceToHost, pp.copy) != cudaSuccess)
+          return FLCE_ERR_CUDA;
+      }
+    }
     // reordered rows: the final dX rows go back in place (no-op otherwise)
     const int sgrid = static_cast<int>(std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(di.num_sms) * 8));
     prof_begin(stream, KIND_SCATTER, &slot);
@@ -749,21 +842,49 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
   if (!h_X || !h_W || !h_y || !h_loss || !h_dX || !h_dW) return FLCE_ERR_INVALID_ARGUMENT;
   flce_status_t s = check_args(d_X, d_W, d_y, N, H, V, d_dX, d_dW, workspace);
   if (s != FLCE_OK) return s;
-  const WsLayout L = ws_layout(N, H);
-  if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
-  const size_t xb = static_cast<size_t>(N) * H * 2, wb = static_cast<size_t>(V) * H * 2, yb = N * 4;
+  if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  PipeRes* pr = nullptr;
+  if (pipe_resources(&pr) != cudaSuccess) return FLCE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(pr->mu);  // one host-buffer call per device at a time: shared copy stream
+  const size_t xb = static_cast<size_t>(N) * H * 2, yb = N * 4;
+  // X and y first, on the caller's stream: every kernel needs them
   if (cudaMemcpyAsync(d_X, h_X, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(d_W, h_W, wb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
       cudaMemcpyAsync(d_y, h_y, yb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return FLCE_ERR_CUDA;
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(static_cast<uint8_t*>(workspace) + L.ctrl);
+  // W in pieces on the copy stream, which starts after the caller's earlier work
+  PipeCtx pp;
+  pp.copy = pr->copy;
+  const int64_t vt = (V + BN - 1) / BN;
+  pp.pieces = static_cast<int>(std::min<int64_t>(MAX_PIECES, vt));
+  for (int i = 0; i <= pp.pieces; ++i) pp.piece_v[i] = std::min<int64_t>(V, (vt * i / pp.pieces) * BN);
+  pp.groups = MAX_PIECES;
+  pp.h_dW = h_dW;
+  if (cudaEventRecord(pr->start, stream) != cudaSuccess || cudaStreamWaitEvent(pr->copy, pr->start, 0) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  for (int i = 0; i < pp.pieces; ++i) {
+    const int64_t v0 = pp.piece_v[i], v1 = pp.piece_v[i + 1];
+    pp.w_ready[i] = pr->ev[i];
+    pp.p2_done[i] = pr->ev[MAX_PIECES + i];
+    if (cudaMemcpyAsync(d_W + v0 * H, h_W + v0 * H, static_cast<size_t>(v1 - v0) * H * 2, cudaMemcpyHostToDevice,
+                        pr->copy) != cudaSuccess ||
+        cudaEventRecord(pp.w_ready[i], pr->copy) != cudaSuccess)
+      return FLCE_ERR_CUDA;
+  }
+  for (int i = pp.pieces; i < MAX_PIECES; ++i) pp.p2_done[i] = pr->ev[MAX_PIECES + i];
+  Options opt;
+  opt.pipe = &pp;
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(workspace);  // the control block opens every layout
   s = enqueue(d_X, d_W, d_y, N, H, V, ignore_index, &ctrl->loss, &ctrl->status, d_dX, d_dW, workspace,
-              workspace_bytes, stream);
-  if (s != FLCE_OK) return s;
+              workspace_bytes, stream, opt);
+  if (s != FLCE_OK) {
+    cudaStreamSynchronize(pr->copy);
+    return s;
+  }
+  // dX and the control block on the caller's stream; dW went back section by section
   Ctrl host{};
   if (cudaMemcpyAsync(h_dX, d_dX, xb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-      cudaMemcpyAsync(h_dW, d_dW, wb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-      cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+      cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaEventRecord(pr->done, pr->copy) != cudaSuccess || cudaStreamWaitEvent(stream, pr->done, 0) != cudaSuccess)
     return FLCE_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
   *h_loss = host.loss;

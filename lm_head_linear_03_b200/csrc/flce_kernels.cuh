@@ -103,6 +103,8 @@ struct GemmArgs {
   int k_blocks;           // pass 1: BK-wide steps along K = H
   int num_units;          // pass 1: tiles_m * splits
   int splits;             // pass 1: vocabulary splits
+  int v_off;              // pass 1: vocabulary id of W's row 0 (a launch over a range of the vocabulary)
+  int split_off;          // pass 1: first partial slot of this launch's splits
   int Vc;                 // pass 2: chunk width = row stride of the G buffer
   const int32_t* y;
   float* part_m;          // [splits][N] running max, log2 units
@@ -131,6 +133,7 @@ struct GemmArgs {
   int C;                  // vocabulary chunks
   int VTf, VT_last;       // 256-wide vocabulary tiles in a full / the last chunk
   long long total_items;
+  long long item_begin, item_end;  // the items of the queue this launch runs
   int* g_row;             // [TM]  G tiles finished per token tile    (x EPI_WARPS*CLUSTER)
   int* g_col;             // [VTf] G tiles finished per chunk column  (x EPI_WARPS*CLUSTER)
   int* x_row;             // [TM]  dX tiles finished per token tile   (x EPI_WARPS*CLUSTER)
@@ -601,7 +604,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       if (a.tile_valid[mb] == 0) continue;  // every row of the tile is ignored
       LseState st;
       st.row = mb * CM + rank * BM + row_local;
-      st.yr = st.row < a.N ? a.y[st.row] : a.ignore_index;
+      // the target's column in this launch's vocabulary range (-1: none; only the pick reads it)
+      const int yrow = st.row < a.N ? a.y[st.row] : a.ignore_index;
+      st.yr = yrow != a.ignore_index && yrow >= a.v_off ? yrow - a.v_off : -1;
       st.run_m = -1e30f;
       st.run_l = 0.f;
       st.zy_val = 0.f;
@@ -623,8 +628,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         if (acc == 0) acc_phase ^= 1u;
       }
       if (ok && st.row < a.N) {
-        a.part_m[static_cast<size_t>(split) * a.N + st.row] = st.run_m;
-        a.part_l[static_cast<size_t>(split) * a.N + st.row] = st.run_l;
+        a.part_m[static_cast<size_t>(split + a.split_off) * a.N + st.row] = st.run_m;
+        a.part_l[static_cast<size_t>(split + a.split_off) * a.N + st.row] = st.run_l;
         if (st.has_zy) a.zy[st.row] = st.zy_val;
       }
     }
@@ -817,7 +822,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (long long u = cid; ok && u < a.total_items; u += ncl) {
+      for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
         const Item it = decode_item(a, u);
         const int vbase = it.c * a.Vc;
         const int vcount = min(a.Vc, a.V - vbase);
@@ -910,7 +915,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (long long u = cid; ok && u < a.total_items; u += ncl) {
+      for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
         const Item it = decode_item(a, u);
         const int vcount = min(a.Vc, a.V - it.c * a.Vc);
         const bool skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
@@ -983,7 +988,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (long long u = cid; ok && u < a.total_items; u += ncl) {
+    for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
       const Item it = decode_item(a, u);
       const int vbase = it.c * a.Vc;
       const int row0 = it.a * CM + rank * BM;
