@@ -168,3 +168,25 @@ def test_default_workspace_reorders_the_large_vocab_shape():
     reordered, n_valid = F.row_order_info(ws)
     assert reordered and n_valid == int((y != -100).sum())
     assert torch.count_nonzero(dX[y == -100]).item() == 0
+
+
+def test_host_entry_with_reordered_rows():
+    """The host-buffer entry (W in pieces, pass 2 in sections) on reordered rows:
+    packed X, dX scattered back, both copied out; checked against the oracle."""
+    F = _lib()
+    w = custom("host_reorder", N=1300, H=256, V=7000, ignore_frac=0.4)
+    X, W, y = make_inputs(w)
+    assert expect_reorder(y)
+    hX, hW, hy = X.pin_memory(), W.pin_memory(), y.pin_memory()
+    ws = F.alloc_workspace(w.N, w.H, w.V, reorder=True)
+    dev = (torch.empty_like(X, device="cuda"), torch.empty_like(W, device="cuda"),
+           torch.empty_like(y, device="cuda"), torch.empty_like(X, device="cuda"),
+           torch.empty_like(W, device="cuda"), ws)
+    loss, hdX, hdW = F.forward_backward_host(hX, hW, hy, dev)
+    reordered, _ = F.row_order_info(ws)
+    assert reordered
+    rl, rdX, rdW, _, _ = O.flce_reference(X, W, y)
+    assert_loss_close(loss, rl)
+    assert_grad_close(_np(hdX), rdX, "dX")
+    assert_grad_close(_np(hdW), rdW, "dW")
+    assert torch.count_nonzero(hdX[y == -100]).item() == 0
