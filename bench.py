@@ -48,8 +48,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--op", choices=["flce", "ce"], default="flce",
-                    help="flce: the fused head (default); ce: cross-entropy on given logits of the same workload")
+    ap.add_argument("--op", choices=["flce", "ce", "unfused"], default="flce",
+                    help="flce: the fused head (default); ce: cross-entropy on given logits of the same workload; "
+                         "unfused: PyTorch eager linear + cross_entropy + autograd, a context row (not this library)")
     return ap.parse_args()
 
 
@@ -491,6 +492,62 @@ def run_ce(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_unfused(args, world, rank, local):
+    """Context row: the unfused head in PyTorch eager mode (cuBLAS bf16 logits,
+    fp32 cross_entropy, autograd for dX and dW) on the same inputs.  It keeps
+    the N x V logits and their gradient; the fused head exists to avoid that."""
+    from lm_head_linear_03_b200.inputs import make_inputs
+    w = workload(args)
+    dev = torch.device("cuda", local)
+    X, W, y = make_inputs(w, dev)
+    N, H, V = w.N, w.H, w.V
+    Xp = X.clone().requires_grad_(True)
+    Wp = W.clone().requires_grad_(True)
+    yl = y.long()
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        Xp.grad = None
+        Wp.grad = None
+        logits = Xp @ Wp.T
+        loss = torch.nn.functional.cross_entropy(logits.float(), yl, ignore_index=-100)
+        loss.backward()
+        return loss
+
+    torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    peak = torch.cuda.max_memory_allocated(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC + " (context: unfused PyTorch eager head)", "impl": "torch_unfused_context",
+        "value": world * N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "H": H, "V": V},
+        "peak_device_bytes_above_inputs": int(peak - base),
+        "logits_bytes": N * V * 2,
+        "note": "cuBLAS bf16 X @ W^T, fp32 cross_entropy, autograd; 6*N*H*V matmul FLOPs, no recompute",
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -499,6 +556,8 @@ def main():
             run_reference(args, world, rank)
         elif args.op == "ce":
             run_ce(args, world, rank, local)
+        elif args.op == "unfused":
+            run_unfused(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
