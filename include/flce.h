@@ -273,7 +273,9 @@ typedef struct {
   int32_t vocab_chunk;     /* vocabulary entries per pass-2 chunk */
   int32_t num_chunks;      /* pass-2 chunks */
   int32_t lse_splits;      /* vocabulary splits of the pass-1 log-sum-exp */
-  int32_t launches;        /* kernels launched by one call */
+  int32_t launches;        /* kernels launched by one device-buffer call (the
+                              host-buffer entry splits pass 1 per W piece and
+                              pass 2 per section of chunks) */
   int32_t num_sms;         /* SMs the persistent kernels are sized for */
 } flce_plan_t;
 flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out);
