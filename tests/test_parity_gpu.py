@@ -84,6 +84,15 @@ def test_small_against_full_oracle(w):
     run_full_oracle_case(X, W, y)
 
 
+@pytest.mark.parametrize("N,H,V,frac", [(70000, 64, 600, 0.3), (70000, 32, 300, 0.0), (8, 64, 300000, 0.25)])
+def test_many_tiles_or_wide_vocab(N, H, V, frac):
+    """More than 256 token tiles (the row-order kernel's loops over tiles take
+    several passes), and a vocabulary of 300000 with a handful of rows."""
+    w = custom(f"extent_{N}_{H}_{V}", N=N, H=H, V=V, ignore_frac=frac)
+    X, W, y = make_inputs(w)
+    run_full_oracle_case(X, W, y)
+
+
 def test_all_rows_ignored_gives_zero():
     w = custom("all_ignored", N=200, H=64, V=1000)
     X, W, y = make_inputs(w)

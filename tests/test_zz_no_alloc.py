@@ -52,3 +52,22 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert flce.workspace_size(N, H, V) > flce.NOALLOC_SCRATCH_BYTES
     st = lib.flce_forward_backward_noalloc(fake, fake, fake, N, H, V, -100, ctypes.byref(loss), fake, fake, None)
     assert st == 3  # FLCE_ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.gpu
+def test_noalloc_reorders_rows_when_its_scratch_has_room():
+    """The fixed scratch holds the packed-X area for small problems, so scattered
+    ignored rows are reordered there too; results against the oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from lm_head_linear_03_b200 import flce
+    from oracle import flce_oracle as O
+    w = custom("noalloc_reorder", N=1100, H=256, V=5000, ignore_frac=0.5)
+    assert flce.workspace_size(w.N, w.H, 1) + flce.packed_x_bytes(w.N, w.H) <= flce.NOALLOC_SCRATCH_BYTES
+    X, W, y = make_inputs(w)
+    loss, dX, dW = flce.forward_backward_noalloc(X.cuda(), W.cuda(), y.cuda())
+    rl, rdX, rdW, _, _ = O.flce_reference(X, W, y)
+    assert_loss_close(loss, rl)
+    assert_grad_close(dX.float().cpu().numpy().astype("float64"), rdX, "dX")
+    assert_grad_close(dW.float().cpu().numpy().astype("float64"), rdW, "dW")
+    assert torch.count_nonzero(dX[(y == -100).cuda()]).item() == 0
