@@ -111,7 +111,12 @@ flce_status_t flce_forward_backward(const uint16_t* X, const uint16_t* W, const 
  *   d_status: DEVICE int32_t*, receives 0 or a device-side flce_status_t
  *   workspace_bytes: size of `workspace`, at least flce_workspace_size(N, H, 1)
  * Host-side argument errors are returned immediately; device-side errors only
- * appear in *d_status. */
+ * appear in *d_status.
+ * CUDA graphs: the call enqueues only memsets and kernel launches, so it may
+ * be captured on `stream` once one call outside a capture has set up the
+ * library on this device.  Decisions that depend on the data (skipped token
+ * tiles, reordered rows, the mean's count) are taken on the device, so a
+ * replay computes the head on whatever the captured buffers hold then. */
 flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, const int32_t* y,
                                           int64_t N, int64_t H, int64_t V, int32_t ignore_index,
                                           float* d_loss, int32_t* d_status, uint16_t* dX,
