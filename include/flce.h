@@ -261,6 +261,20 @@ flce_status_t flce_forward_backward_noalloc(const uint16_t* X, const uint16_t* W
  * and d_status[2] the untouched counter.  timeout_ns in (0, 1e10]. */
 flce_status_t flce_probe_bounded_wait(int64_t timeout_ns, int32_t* d_status, cudaStream_t stream);
 
+/* Failure-detection probe of the GEMM kernels' own waits.  Enqueues one call
+ * with the arguments of flce_forward_backward_async, except that every dW
+ * item of pass 2 waits for one more finished logit-gradient tile than the
+ * queue produces, and every wait inside the kernels is bounded by timeout_ns
+ * instead of 2 s.  The starved waits give up, the SM pairs wind down (both
+ * CTAs of a pair together) and *d_status receives FLCE_ERR_TIMEOUT; the
+ * loss, dX and dW are then undefined.  The device stays usable.
+ * timeout_ns in (0, 1e10]. */
+flce_status_t flce_probe_pass2_timeout(const uint16_t* X, const uint16_t* W, const int32_t* y,
+                                       int64_t N, int64_t H, int64_t V, int32_t ignore_index,
+                                       float* d_loss, int32_t* d_status, uint16_t* dX, uint16_t* dW,
+                                       void* workspace, size_t workspace_bytes, int64_t timeout_ns,
+                                       cudaStream_t stream);
+
 /* Token-row order chosen by the last call that used `workspace` (see
  * "Ignored rows" above), read back once `stream` has finished that call:
  *   *reordered = 1 when the rows were reordered (valid rows first, X packed

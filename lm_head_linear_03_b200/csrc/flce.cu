@@ -366,6 +366,10 @@ struct Options {
   const float* all_lse = nullptr;
   const float* all_zy = nullptr;
   const PipeCtx* pipe = nullptr;  // host-buffer call: pieces of pass 1, sections of pass 2
+  // failure probe only: a shorter wait limit, and dW mainloops that wait for
+  // one G tile more than the queue produces
+  unsigned long long timeout_ns = DEFAULT_TIMEOUT_NS;
+  int starve_dw = 0;
 };
 
 flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H, int64_t V,
@@ -436,7 +440,8 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   a.dX = dX;
   a.lo = lo;
   a.status = d_status;
-  a.timeout_ns = DEFAULT_TIMEOUT_NS;
+  a.timeout_ns = opt.timeout_ns;
+  a.starve_dw = opt.starve_dw;
   a.reduction = opt.reduction;
   a.grad_row_scale = g_rows;
   a.tile_valid = reinterpret_cast<const int*>(ws + L.tile_valid);
@@ -832,6 +837,21 @@ flce_status_t flce_probe_bounded_wait(int64_t timeout_ns, int32_t* d_status, cud
   if (cudaMemsetAsync(d_status, 0, 3 * sizeof(int32_t), stream) != cudaSuccess) return FLCE_ERR_CUDA;
   flce_wait_probe_kernel<<<1, 32, 0, stream>>>(d_status, d_status + 2, static_cast<unsigned long long>(timeout_ns));
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+flce_status_t flce_probe_pass2_timeout(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H,
+                                       int64_t V, int32_t ignore_index, float* d_loss, int32_t* d_status,
+                                       uint16_t* dX, uint16_t* dW, void* workspace, size_t workspace_bytes,
+                                       int64_t timeout_ns, cudaStream_t stream) {
+  if (!d_loss || !d_status || timeout_ns <= 0 || timeout_ns > 10000000000ll) return FLCE_ERR_INVALID_ARGUMENT;
+  const flce_status_t s = check_args(X, W, y, N, H, V, dX, dW, workspace);
+  if (s != FLCE_OK) return s;
+  if (!aligned(d_status, 4) || !aligned(d_loss, 4)) return FLCE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  Options opt;
+  opt.timeout_ns = static_cast<unsigned long long>(timeout_ns);
+  opt.starve_dw = 1;
+  return enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace, workspace_bytes, stream, opt);
 }
 
 flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_W, const int32_t* h_y, int64_t N,

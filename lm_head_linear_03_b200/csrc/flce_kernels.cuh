@@ -118,6 +118,7 @@ struct GemmArgs {
   uint16_t* lo;           // [N][H] bf16, low half of the dX accumulator
   int* status;
   unsigned long long timeout_ns;
+  int starve_dw;          // failure probe only: dW mainloops wait for one G tile more than exist
   int reduction;                 // RED_MEAN, RED_SUM, RED_NONE
   const float* grad_row_scale;   // RED_NONE: per-row upstream gradient, or null for 1
   const int* tile_valid;         // [ceil(N/256)] valid rows per 256-row token tile (prep kernel)
@@ -142,6 +143,19 @@ struct GemmArgs {
 
 __device__ __forceinline__ void raise_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// A wait of one CTA of an SM pair gave up: both CTAs wind down at once (the
+// peer's roles see the flag in their next wait), so the pair reaches the
+// end-of-kernel handshake together and neither CTA leaves while the other may
+// still reach into its shared memory.  The handshake allows END_WAIT_LIMITS
+// wait limits, more than the one wait a CTA can still be in when the other
+// arrives.
+constexpr unsigned long long END_WAIT_LIMITS = 4;
+__device__ __forceinline__ void give_up_pair(volatile int* abort_flag, int rank, int* status) {
+  *abort_flag = 1;
+  st_cluster_u32(mapa_shared(smem_u32(const_cast<int*>(abort_flag)), static_cast<uint32_t>(rank ^ 1)), 1u);
+  raise_status(status, ST_TIMEOUT);
 }
 
 // Pass-1 work unit u -> token tile mb, vocabulary split `split` and the range
@@ -482,10 +496,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  auto give_up = [&]() {
-    *abort_flag = 1;
-    raise_status(a.status, ST_TIMEOUT);
-  };
+  auto give_up = [&]() { give_up_pair(abort_flag, rank, a.status); };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -643,7 +654,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     mbar_arrive_cluster(mapa_shared(fin_bar, static_cast<uint32_t>(rank ^ 1)));
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_cluster(fin_bar, 0)) {
-      if (globaltimer_ns() - t0 > a.timeout_ns) {
+      if (globaltimer_ns() - t0 > END_WAIT_LIMITS * a.timeout_ns) {
         raise_status(a.status, ST_TIMEOUT);
         break;
       }
@@ -806,10 +817,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  auto give_up = [&]() {
-    *abort_flag = 1;
-    raise_status(a.status, ST_TIMEOUT);
-  };
+  auto give_up = [&]() { give_up_pair(abort_flag, rank, a.status); };
   // cumulative G tiles of token tile tm after chunk c
   auto g_row_target = [&](int c) {
     return SIGNALS_PER_ITEM * (c < a.C - 1 ? (c + 1) * a.VTf : (a.C - 1) * a.VTf + a.VT_last);
@@ -835,7 +843,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
           kblocks = (a.H + BK - 1) / BK;
         } else if (it.kind == ITEM_DW) {
           kblocks = (a.N + BK - 1) / BK;
-          ok = wait_counter(a.g_col + it.a, SIGNALS_PER_ITEM * a.TM * (it.c + 1), abort_flag, a.timeout_ns);
+          ok = wait_counter(a.g_col + it.a, SIGNALS_PER_ITEM * a.TM * (it.c + 1) + a.starve_dw, abort_flag,
+                            a.timeout_ns);
         } else {
           kblocks = (vcount + BK - 1) / BK;
           ok = wait_counter(a.g_row + it.a, g_row_target(it.c), abort_flag, a.timeout_ns);
@@ -1063,7 +1072,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     mbar_arrive_cluster(mapa_shared(fin_bar, static_cast<uint32_t>(rank ^ 1)));
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_cluster(fin_bar, 0)) {
-      if (globaltimer_ns() - t0 > a.timeout_ns) {
+      if (globaltimer_ns() - t0 > END_WAIT_LIMITS * a.timeout_ns) {
         raise_status(a.status, ST_TIMEOUT);
         break;
       }

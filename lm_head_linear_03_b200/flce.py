@@ -42,6 +42,7 @@ EXPORTED = (
     "flce_ce_workspace_size",
     "flce_cross_entropy",
     "flce_probe_bounded_wait",
+    "flce_probe_pass2_timeout",
     "flce_row_order_info",
     "flce_vp_shard_stats",
     "flce_vp_backward",
@@ -108,6 +109,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_cross_entropy.restype = ctypes.c_int
     lib.flce_probe_bounded_wait.argtypes = [i64, vp, vp]
     lib.flce_probe_bounded_wait.restype = ctypes.c_int
+    lib.flce_probe_pass2_timeout.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, sz, i64, vp]
+    lib.flce_probe_pass2_timeout.restype = ctypes.c_int
     lib.flce_forward_backward_noalloc.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp, vp]
     lib.flce_forward_backward_noalloc.restype = ctypes.c_int
     lib.flce_row_order_info.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), vp]
@@ -388,6 +391,25 @@ def forward_backward_noalloc(X, W, y, ignore_index: int = -100, *, dX=None, dW=N
                                            ctypes.byref(loss), _ptr(dX), _ptr(dW), _stream_handle(stream))
     _check(st, "flce_forward_backward_noalloc")
     return loss.value, dX, dW
+
+
+def probe_pass2_timeout(X, W, y, ignore_index: int = -100, *, timeout_ns: int = 5_000_000, workspace=None,
+                        stream=None):
+    """Enqueues one call whose pass-2 dW items wait for a tile that never
+    comes, every wait bounded by ``timeout_ns``; returns the device status
+    tensor int32[1] (FLCE_ERR_TIMEOUT once the stream gets there)."""
+    lib = load_library()
+    _check_inputs(X, W, y)
+    N, H = X.shape
+    V = W.shape[0]
+    loss = torch.empty(1, dtype=torch.float32, device=X.device)
+    status = torch.empty(1, dtype=torch.int32, device=X.device)
+    dX, dW = torch.empty_like(X), torch.empty_like(W)
+    workspace = alloc_workspace(N, H, V, X.device) if workspace is None else workspace
+    _check(lib.flce_probe_pass2_timeout(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, _ptr(loss), _ptr(status),
+                                        _ptr(dX), _ptr(dW), _ptr(workspace), workspace.numel(), timeout_ns,
+                                        _stream_handle(stream)), "flce_probe_pass2_timeout")
+    return status
 
 
 def probe_bounded_wait(timeout_ns: int = 1_000_000, stream=None):

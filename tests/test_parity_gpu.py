@@ -312,6 +312,26 @@ def test_bounded_waits_give_up_and_report_timeout():
     run_full_oracle_case(*make_inputs(WORKLOADS["tiny"]))
 
 
+def test_pass2_starved_waits_give_up_and_report_timeout():
+    """The GEMM kernels' own waits: a call whose dW items wait for one more
+    G tile than the queue produces ends with FLCE_ERR_TIMEOUT within seconds
+    (each SM pair winds down, both CTAs together), and the next call on the
+    device matches the oracle."""
+    _lib()
+    from lm_head_linear_03_b200 import flce
+    import time
+    w = custom("starved_dw", N=700, H=256, V=5000, ignore_frac=0.1)
+    X, W, y = make_inputs(w)
+    Xd, Wd, yd = X.cuda(), W.cuda(), y.cuda()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    st = flce.probe_pass2_timeout(Xd, Wd, yd, timeout_ns=5_000_000)  # 5 ms per wait
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 10.0
+    assert st.item() == 5
+    run_full_oracle_case(X, W, y)
+
+
 def test_mean_over_external_count():
     """The data-parallel hook: the mean divides by a count from outside the call
     (all ranks' valid targets); equals the oracle with weights 1/count."""
