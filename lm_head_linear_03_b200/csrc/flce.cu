@@ -573,6 +573,9 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       section_end[c] = total;
     }
     b.total_items = total;
+    // G tiles column by column when a chunk holds more than three rounds of
+    // them for the SM pairs, else row by row (see the queue's description)
+    b.g_cols_first = static_cast<long long>(b.TM) * b.VTf > 3ll * P.clusters ? b.VTf : 0;
     int* ctr = reinterpret_cast<int*>(ws + L.counters);
     b.g_row = ctr;
     b.x_row = ctr + b.TM;

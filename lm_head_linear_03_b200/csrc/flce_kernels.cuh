@@ -119,6 +119,7 @@ struct GemmArgs {
   int* status;
   unsigned long long timeout_ns;
   int starve_dw;          // failure probe only: dW mainloops wait for one G tile more than exist
+  int g_cols_first;       // G(c): this many vocabulary tiles first, column by column; the rest row by row
   int reduction;                 // RED_MEAN, RED_SUM, RED_NONE
   const float* grad_row_scale;   // RED_NONE: per-row upstream gradient, or null for 1
   const int* tile_valid;         // [ceil(N/256)] valid rows per 256-row token tile (prep kernel)
@@ -674,8 +675,14 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
 //
 //   G(0)  |  dX(0) dW(0) G(1)  |  dX(1) dW(1) G(2)  | ... |  dX(C-1) dW(C-1)
 //
-// where G(c) are the logit-recompute tiles of chunk c (column-major), dX(c) the
-// dX += G_c W_c tiles and dW(c) the dW rows of chunk c.  There is one G buffer,
+// where G(c) are the logit-recompute tiles of chunk c, dX(c) the
+// dX += G_c W_c tiles and dW(c) the dW rows of chunk c.  The G tiles of a
+// chunk go column by column (all token tiles of one vocabulary tile, then the
+// next) when a chunk holds more than three rounds of them for the SM pairs:
+// the dW(c) items that their epilogues wait for finish column by column.  With
+// fewer rounds they go row by row, so that each token tile's G row is complete
+// early and the dX(c) items that wait for it are not all held up by the last
+// column.  There is one G buffer,
 // so items wait for what they read and for the readers of what they overwrite:
 //   dX(c) mainloop  after G(c) of its token tile (all its columns),
 //   dX(c) epilogue  after dX(c-1) of its token tile (running sum),
@@ -700,14 +707,31 @@ __device__ __forceinline__ long long section_size(const GemmArgs& p, int c) {
   return n;
 }
 
+// Tile of the r-th G item of chunk c: the first g_cols_first vocabulary tiles
+// column by column (every token tile of one column, then the next column),
+// the remaining ones row by row.
+__device__ __forceinline__ void grad_tile(const GemmArgs& p, int c, long long r, Item& it) {
+  const int vt = chunk_vtiles(p, c);
+  const int k = min(p.g_cols_first, vt);
+  const long long head = static_cast<long long>(k) * p.TM;
+  if (r < head) {
+    it.b = static_cast<int>(r / p.TM);
+    it.a = static_cast<int>(r - static_cast<long long>(it.b) * p.TM);
+  } else {
+    const long long r2 = r - head;
+    const int w = vt - k;
+    it.a = static_cast<int>(r2 / w);
+    it.b = k + static_cast<int>(r2 - static_cast<long long>(it.a) * w);
+  }
+}
+
 __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
   Item it;
   const long long g0 = static_cast<long long>(chunk_vtiles(p, 0)) * p.TM;
   if (i < g0) {
     it.kind = ITEM_GRAD;
     it.c = 0;
-    it.b = static_cast<int>(i / p.TM);
-    it.a = static_cast<int>(i - static_cast<long long>(it.b) * p.TM);
+    grad_tile(p, 0, i, it);
     return it;
   }
   // sections 0 .. C-3 all have the size of section 0; the last two may be shorter
@@ -738,8 +762,7 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
     r -= nx + nw;
     it.kind = ITEM_GRAD;
     it.c = c + 1;
-    it.b = static_cast<int>(r / p.TM);
-    it.a = static_cast<int>(r - static_cast<long long>(it.b) * p.TM);
+    grad_tile(p, c + 1, r, it);
   }
   return it;
 }
