@@ -77,3 +77,46 @@ def test_reference_arm_two_ranks_rank0_only():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1 and json.loads(lines[0])["n_gpus"] == 2
+
+
+def _remeasure_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    w, r, _ = bench.dist_setup(None)
+    # rank 0 saw a thermal slowdown, rank 1 only the power cap
+    clocks = ({"sm_mhz": 900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_thermal_slowdown"]} if r == 0 else
+              {"sm_mhz": 1400.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]})
+    got = bench.remeasure_needed(clocks, w)
+    bench.dist_teardown(w)
+    q.put((rank, got))
+
+
+def test_remeasure_decision_is_the_same_on_every_rank():
+    """A timed region rejected on one rank is measured again on all of them."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_remeasure_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=10) for _ in range(2))
+    assert got == {0: True, 1: True}
+
+
+def test_clock_records_rejected_or_kept():
+    sys.path.insert(0, ROOT)
+    import bench
+    keep = [{"sm_mhz": 1400.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]},
+            {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+            {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}]
+    reject = [{"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["hw_slowdown"]},
+              {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0, "reasons": ["hw_thermal_slowdown", "sw_power_cap"]},
+              {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": ["sw_thermal_slowdown"]},
+              {"sm_mhz": 1100.0, "sm_max_mhz": 1965.0, "reasons": []}]   # held low with no reason: a clock lock
+    assert not any(bench.clocks_rejected(c) for c in keep)
+    assert all(bench.clocks_rejected(c) for c in reject)
