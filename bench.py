@@ -342,6 +342,19 @@ def run_ours(args, world, rank, local):
     ms_max, clocks = timed_region(dev, stream, world, args.steps, step)
     ms_per_step = ms_max / args.steps
 
+    # --- step-time spread: the same K steps, each between its own events ----
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    torch.cuda.synchronize(dev)
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    step_ms = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps))
+    step_stats = {"median": statistics.median(step_ms), "min": step_ms[0],
+                  "p90": step_ms[min(len(step_ms) - 1, int(0.9 * len(step_ms)))], "n": len(step_ms),
+                  "note": "one step per event pair, outside the timed region; this rank"}
+
     # --- per-kernel durations: the same K steps with every launch bracketed --
     F.profile_enable(True)
     barrier(world)
@@ -449,6 +462,7 @@ def run_ours(args, world, rank, local):
             "algorithmic_flops_per_launch": algo_flops_per_launch, "avg_launch_ms": avg_ms,
             "launches_per_step": per_step_launches,
         },
+        "step_ms": step_stats,
         "kernels": {k: {"launches_per_step": v[0] / args.steps, "ms_per_step": v[1] / args.steps,
                         "share": v[1] / total_prof_ms} for k, v in kinds.items()},
         "profiled_ms_per_step": prof_ms_per_step,
