@@ -48,9 +48,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--op", choices=["flce", "ce", "unfused"], default="flce",
+    ap.add_argument("--op", choices=["flce", "ce", "unfused", "vp"], default="flce",
                     help="flce: the fused head (default); ce: cross-entropy on given logits of the same workload; "
-                         "unfused: PyTorch eager linear + cross_entropy + autograd, a context row (not this library)")
+                         "unfused: PyTorch eager linear + cross_entropy + autograd, a context row (not this library); "
+                         "vp: the vocabulary-parallel head's shards run one after another on this GPU")
+    ap.add_argument("--shards", type=int, default=8, help="vocabulary shards of --op vp")
     return ap.parse_args()
 
 
@@ -531,6 +533,83 @@ def run_ce(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_vp(args, world, rank, local):
+    """The vocabulary-parallel head's compute, measured on one GPU: the S
+    shards of the vocabulary run one after another (each shard's statistics,
+    then each shard's backward), with the all-gather of the statistics as a
+    stack and the dX all-reduce as a sum on this device.  One step is the work
+    S ranks would share, collectives excluded; the fused head on the whole
+    vocabulary is timed beside it."""
+    import lm_head_linear_03_b200 as F
+    from lm_head_linear_03_b200.inputs import make_inputs
+    from lm_head_linear_03_b200.parallel import vocab_shard_range
+    F.load_library()
+    w = workload(args)
+    dev = torch.device("cuda", local)
+    X, W, y = make_inputs(w, dev)
+    N, H, V = w.N, w.H, w.V
+    S = args.shards
+    bounds = [vocab_shard_range(V, S, r) for r in range(S)]
+    shards = [W[v0:v1].contiguous() for v0, v1 in bounds]
+    stream = torch.cuda.current_stream(dev)
+    ws = F.alloc_workspace(N, H, 1, dev)
+    dX = torch.empty(N, H, dtype=torch.float32, device=dev)
+    status = []
+
+    def step():
+        stats = [F.vp_shard_stats(X, Ws, y, v0, V, workspace=ws, stream=stream)
+                 for (v0, _), Ws in zip(bounds, shards)]
+        all_lse = torch.stack([st[0] for st in stats])
+        all_zy = torch.stack([st[1] for st in stats])
+        dX.zero_()
+        status.clear()
+        for (v0, _), Ws in zip(bounds, shards):
+            loss, st, dXp, _dWs = F.vp_backward(X, Ws, y, v0, V, all_lse, all_zy, workspace=ws, stream=stream)
+            dX.add_(dXp)
+            status.append(st)
+        status.extend(st[2] for st in stats)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert all(int(t.item()) == 0 for t in status), "device status"
+    ms, clocks = timed_region(dev, stream, world, args.steps, step)
+    ms /= args.steps
+
+    fws = F.alloc_workspace(N, H, V, dev)
+    out = (torch.empty(1, dtype=torch.float32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
+           torch.empty_like(X), torch.empty_like(W))
+
+    def fused():
+        F.forward_backward_async(X, W, y, out=out, workspace=fws, stream=stream)
+
+    for _ in range(3):
+        fused()
+    fused_ms, _ = timed_region(dev, stream, world, args.steps, fused)
+    fused_ms /= args.steps
+    if rank != 0:
+        return
+    pk, pk_src = peaks()
+    flops = 8.0 * N * H * V
+    line = {
+        "metric": "vocabulary-parallel head, shards in sequence on one GPU, tokens/s (collectives excluded)",
+        "value": world * N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "H": H, "V": V, "shards": S,
+                   "shard_rows": [v1 - v0 for v0, v1 in bounds]},
+        "tflops": flops / (ms * 1e-3) / 1e12,
+        "pct_of_measured_bf16_sustained": 100.0 * flops / (ms * 1e-3) / 1e12 / pk["bf16_tflops_sustained"],
+        "fused_whole_vocabulary_ms": fused_ms,
+        "shards_over_fused": ms / fused_ms,
+        "gpu_launches": 9 * S * args.steps,
+        "clocks": clocks,
+        "note": f"peaks: {pk_src}; this library's launches per shard: prep, row order, pass 1, combine; then prep, "
+                "row order, combine, pass 2, scatter (torch's stack and dX sum not counted)",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_unfused(args, world, rank, local):
     """Context row: the unfused head in PyTorch eager mode (cuBLAS bf16 logits,
     fp32 cross_entropy, autograd for dX and dW) on the same inputs.  It keeps
@@ -597,6 +676,8 @@ def main():
             run_ce(args, world, rank, local)
         elif args.op == "unfused":
             run_unfused(args, world, rank, local)
+        elif args.op == "vp":
+            run_vp(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
