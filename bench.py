@@ -48,10 +48,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--op", choices=["flce", "ce", "unfused", "vp"], default="flce",
+    ap.add_argument("--op", choices=["flce", "ce", "unfused", "vp", "pref"], default="flce",
                     help="flce: the fused head (default); ce: cross-entropy on given logits of the same workload; "
                          "unfused: PyTorch eager linear + cross_entropy + autograd, a context row (not this library); "
-                         "vp: the vocabulary-parallel head's shards run one after another on this GPU")
+                         "vp: the vocabulary-parallel head's shards run one after another on this GPU; "
+                         "pref: the pairwise logistic preference loss on the head")
     ap.add_argument("--shards", type=int, default=8, help="vocabulary shards of --op vp")
     return ap.parse_args()
 
@@ -610,6 +611,71 @@ def run_vp(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_pref(args, world, rank, local):
+    """The pairwise logistic (DPO-form) preference loss on the head, measured:
+    the workload's token rows packed as sequences of 1024 rows whose first
+    quarter is the prompt (ignored), consecutive sequences forming (chosen,
+    rejected) pairs.  One step is a forward-only head call for the per-row
+    log-probabilities, the pair loss, and a full head call with the pairs'
+    upstream weights; the fused mean cross-entropy on the same rows is timed
+    beside it."""
+    import lm_head_linear_03_b200 as F
+    from lm_head_linear_03_b200.inputs import make_inputs
+    from lm_head_linear_03_b200.preference import preference_forward_backward
+    F.load_library()
+    w = workload(args)
+    dev = torch.device("cuda", local)
+    X, W, y = make_inputs(w, dev)
+    N, H, V = w.N, w.H, w.V
+    seq_len = 1024 if N >= 2048 else max(2, N // 2)
+    rows = torch.arange(N, device=dev)
+    seq = rows // seq_len
+    y = torch.where(rows % seq_len < seq_len // 4, torch.full_like(y, -100), y).contiguous()
+    S = int(seq.max().item()) + 1
+    chosen = torch.arange(0, S - 1, 2, device=dev)
+    rejected = chosen + 1
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        preference_forward_backward(X, W, y, seq, chosen, rejected, beta=0.1)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    ms, clocks = timed_region(dev, stream, world, args.steps, step)
+    ms /= args.steps
+
+    fws = F.alloc_workspace(N, H, V, dev)
+    out = (torch.empty(1, dtype=torch.float32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
+           torch.empty_like(X), torch.empty_like(W))
+
+    def fused():
+        F.forward_backward_async(X, W, y, out=out, workspace=fws, stream=stream)
+
+    for _ in range(3):
+        fused()
+    fused_ms, _ = timed_region(dev, stream, world, args.steps, fused)
+    fused_ms /= args.steps
+    if rank != 0:
+        return
+    line = {
+        "metric": "pairwise logistic preference loss on the fused head fwd+bwd tokens/s",
+        "value": world * N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "H": H, "V": V, "sequences": S, "pairs": int(chosen.numel()),
+                   "seq_len": seq_len, "prompt_rows_per_sequence": seq_len // 4},
+        "fused_mean_ce_ms": fused_ms,
+        "pref_over_fused": ms / fused_ms,
+        "gpu_launches": 10 * args.steps,
+        "clocks": clocks,
+        "note": "this library's launches per step: forward-only head call (prep, row order, pass 1, combine) and "
+                "full head call (prep, row order, pass 1, combine, pass 2, scatter); host syncs for the "
+                "sequence count and the status checks fall inside the step",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_unfused(args, world, rank, local):
     """Context row: the unfused head in PyTorch eager mode (cuBLAS bf16 logits,
     fp32 cross_entropy, autograd for dX and dW) on the same inputs.  It keeps
@@ -678,6 +744,8 @@ def main():
             run_unfused(args, world, rank, local)
         elif args.op == "vp":
             run_vp(args, world, rank, local)
+        elif args.op == "pref":
+            run_pref(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
