@@ -44,6 +44,14 @@ MUTATIONS = [
      "return L.max(axis=0), _f64(all_zy).sum(axis=0)"),
     ("shard target logits averaged", "return log_sum_exp(L.T), _f64(all_zy).sum(axis=0)",
      "return log_sum_exp(L.T), _f64(all_zy).mean(axis=0)"),
+    ("blocked lse drops the ragged last block", "    for b in range(0, X.shape[0], block):",
+     "    out[:] = 0.0\n    for b in range(0, X.shape[0] - X.shape[0] % block, block):"),
+    ("blocked loss divides by all rows", "loss = float(row_loss.sum() / n) if n else 0.0",
+     "loss = float(row_loss.sum() / len(y)) if n else 0.0"),
+    ("dX rows take another row's log-sum-exp", "G = np.exp(Z - np.asarray(lse_rows, dtype=np.float64)[:, None])",
+     "G = np.exp(Z - np.asarray(lse_rows, dtype=np.float64)[::-1][:, None])"),
+    ("dW rows keep ignored rows", "    G *= valid[:, None]\n    G *= (1.0 / n) if n else 0.0\n    return G.T @ X64",
+     "    G *= (1.0 / n) if n else 0.0\n    return G.T @ X64"),
 ]
 
 
