@@ -36,7 +36,7 @@
  *
  * Ownership.  All device pointers belong to the caller.  The library never
  * allocates device memory: scratch space is the caller's `workspace`, at least
- * flce_workspace_size(N, H, V) bytes (at least the base size, see there).  dX
+ * flce_workspace_size(N, H, V) bytes, a size that does not depend on V.  dX
  * and dW are overwritten, not accumulated into.  The library keeps only
  * read-only host caches (device properties, a driver entry point) and, for
  * the host-buffer entry, one copy stream with a few events per device.
@@ -51,10 +51,10 @@
  * targets are all ignored is skipped.  When ignored rows are scattered, so
  * that packing the valid rows first would fill fewer tiles than the tiles
  * holding any valid row, and the workspace holds the packed-X area (see
- * flce_workspace_size), the library reorders the token rows on the device (a
- * stable partition, valid rows first): it packs those rows of X into the
- * workspace, runs both passes on them, and writes dX and the per-row losses
- * back in the caller's row order.  The choice changes only the order of
+ * flce_workspace_size_reorder), the library reorders the token rows on the
+ * device (a stable partition, valid rows first): it packs those rows of X
+ * into the workspace, runs both passes on them, and writes dX and the per-row
+ * losses back in the caller's row order.  The choice changes only the order of
  * floating-point sums, not the result's definition.
  */
 #ifndef FLCE_H_
@@ -73,7 +73,7 @@ typedef enum {
   FLCE_OK = 0,
   FLCE_ERR_INVALID_ARGUMENT = 1,    /* NULL pointer, non-positive size, size too large */
   FLCE_ERR_UNSUPPORTED = 2,         /* H % 8 != 0, misaligned pointer, device is not sm_100 */
-  FLCE_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < flce_workspace_size(N, H, 1) */
+  FLCE_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < flce_workspace_size(N, H, V) */
   FLCE_ERR_TARGET_OUT_OF_RANGE = 4, /* some y_i != ignore_index lies outside [0, V) */
   FLCE_ERR_TIMEOUT = 5,             /* a bounded wait inside a kernel gave up */
   FLCE_ERR_CUDA = 6                 /* a CUDA runtime call failed */
@@ -82,22 +82,28 @@ typedef enum {
 /* Human-readable name of a status code (static storage). */
 const char* flce_status_string(int status);
 
-/* Bytes of device workspace one call asks for.  The logits are processed one
- * vocabulary chunk of fixed width at a time, so the base size depends on N
- * and H only; it is flce_workspace_size(N, H, 1).  On top of it comes an
- * N x H bf16 area (its byte size rounded up to a multiple of 256) for a
- * packed copy of X, which reordered token rows need
- * (see "Ignored rows"), whenever the whole stays within 5% of the N x V bf16
- * logits the head never stores.  Every entry accepts any workspace of at
- * least the base size and reorders rows only when the area fits in it.
- * Returns 0 for invalid sizes. */
+/* Bytes of device workspace one call needs.  The logits are processed one
+ * vocabulary chunk of fixed width at a time, so the size depends on N and H
+ * only: V is accepted for the caller's convenience and does not change the
+ * value.  Returns 0 for invalid sizes. */
 size_t flce_workspace_size(int64_t N, int64_t H, int64_t V);
+
+/* Bytes of a workspace that also holds the N x H bf16 area (its byte size
+ * rounded up to a multiple of 256) for a packed copy of X, which reordered
+ * token rows need (see "Ignored rows"): flce_workspace_size(N, H, V) plus that
+ * area, again independent of V.  Entries that take a workspace_bytes argument
+ * reorder rows only when given at least this many bytes; with less (but at
+ * least flce_workspace_size) they keep the caller's order.  Returns 0 for
+ * invalid sizes.  The pages describe no such query; it sizes the library's
+ * own row gather. */
+size_t flce_workspace_size_reorder(int64_t N, int64_t H);
 
 /* Synchronous forward + backward.
  *   X  [N,H] bf16, device      W  [V,H] bf16, device      y [N] int32, device
  *   loss: HOST float*, receives the token-mean loss
  *   dX [N,H] bf16, device (out)   dW [V,H] bf16, device (out)
  *   workspace: device, >= flce_workspace_size(N, H, V) bytes, 256-B aligned
+ *              (this entry never reorders token rows: it has no size argument)
  *   stream: the CUDA stream to run on (0 = legacy default stream)
  * Blocks the calling host thread until the stream has finished the call, then
  * returns FLCE_OK or the first error seen, including device-side errors. */
@@ -109,7 +115,9 @@ flce_status_t flce_forward_backward(const uint16_t* X, const uint16_t* W, const 
 /* Asynchronous twin: enqueues the whole computation on `stream` and returns.
  *   d_loss:   DEVICE float*, receives the loss when the stream gets there
  *   d_status: DEVICE int32_t*, receives 0 or a device-side flce_status_t
- *   workspace_bytes: size of `workspace`, at least flce_workspace_size(N, H, 1)
+ *   workspace_bytes: size of `workspace`, at least flce_workspace_size(N, H, V);
+ *                    flce_workspace_size_reorder(N, H) or more lets the call
+ *                    reorder token rows
  * Host-side argument errors are returned immediately; device-side errors only
  * appear in *d_status.
  * CUDA graphs: the call enqueues only memsets and kernel launches, so it may
@@ -239,7 +247,8 @@ flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64
  * fixed array of FLCE_NOALLOC_SCRATCH_BYTES in the library's device module,
  * held on every GPU that loads the library until the process exits.  Sizes
  * whose flce_workspace_size exceeds it are rejected with
- * FLCE_ERR_WORKSPACE_TOO_SMALL before anything runs.
+ * FLCE_ERR_WORKSPACE_TOO_SMALL before anything runs; token rows are reordered
+ * only when flce_workspace_size_reorder fits in it too.
  *
  * The first call on a device looks the array's device address up (a
  * cudaGetSymbolAddress, no allocation); make that first call before any stream
@@ -289,10 +298,13 @@ flce_status_t flce_row_order_info(const void* workspace, int32_t* reordered, int
 /* How a call of these sizes is split into launches (host-only query). */
 typedef struct {
   int64_t workspace_bytes; /* same as flce_workspace_size */
+  int64_t workspace_reorder_bytes; /* same as flce_workspace_size_reorder */
   int32_t vocab_chunk;     /* vocabulary entries per pass-2 chunk */
   int32_t num_chunks;      /* pass-2 chunks */
   int32_t lse_splits;      /* vocabulary splits of the pass-1 log-sum-exp */
-  int32_t launches;        /* kernels launched by one device-buffer call (the
+  int32_t launches;        /* kernels launched by one device-buffer call on a
+                              workspace of workspace_bytes (one more, the X row
+                              packing, on one of workspace_reorder_bytes; the
                               host-buffer entry splits pass 1 per W piece and
                               pass 2 per section of chunks) */
   int32_t num_sms;         /* SMs the persistent kernels are sized for */

@@ -17,8 +17,10 @@ from .flce import (  # noqa: F401
     plan,
     profile_enable,
     profile_read,
+    reorder_fits,
     row_order_info,
     vp_backward,
     vp_shard_stats,
     workspace_size,
+    workspace_size_reorder,
 )

@@ -79,14 +79,6 @@ WsLayout ws_layout(int64_t N, int64_t H, bool packed = false) {
   return L;
 }
 
-// The workspace a call is asked for: the packed-X area is included when the
-// whole stays within 5% of the N x V bf16 logits the head never stores.
-size_t ws_total(int64_t N, int64_t H, int64_t V) {
-  const size_t with = ws_layout(N, H, true).total;
-  const double logits = 2.0 * static_cast<double>(N) * static_cast<double>(V);
-  return static_cast<double>(with) <= 0.05 * logits ? with : ws_layout(N, H).total;
-}
-
 // Workspace of the cross-entropy-on-logits entry: depends on N only.
 struct CeLayout {
   size_t ctrl, tile_valid, row_acc, blk_sum, total;
@@ -254,8 +246,9 @@ Plan make_plan(int64_t N, int64_t H, int64_t V, int clusters) {
   p.lse_clusters =
       static_cast<int>(std::min<long long>(static_cast<long long>(p.tiles_m) * p.splits, clusters));
   p.num_chunks = static_cast<int>((V + VC - 1) / VC);
-  // prep, row order, pass 1, combine, pass 2, dX scatter; X pack with the packed-X area
-  p.launches = ws_total(N, H, V) == ws_layout(N, H, true).total ? 7 : 6;
+  // prep, row order, pass 1, combine, pass 2, dX scatter (plus the X row
+  // packing on a workspace with the packed-X area)
+  p.launches = 6;
   return p;
 }
 
@@ -670,14 +663,19 @@ const char* flce_status_string(int s) {
 
 size_t flce_workspace_size(int64_t N, int64_t H, int64_t V) {
   if (check_sizes(N, H, V == 0 ? 1 : V) != FLCE_OK) return 0;
-  return ws_total(N, H, V == 0 ? 1 : V);
+  return ws_layout(N, H).total;
+}
+
+size_t flce_workspace_size_reorder(int64_t N, int64_t H) {
+  if (check_sizes(N, H, 1) != FLCE_OK) return 0;
+  return ws_layout(N, H, true).total;
 }
 
 flce_status_t flce_forward_backward(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H,
                                     int64_t V, int32_t ignore_index, float* loss, uint16_t* dX, uint16_t* dW,
                                     void* workspace, cudaStream_t stream) {
   if (check_sizes(N, H, V) != FLCE_OK) return check_sizes(N, H, V);
-  return sync_call(X, W, y, N, H, V, ignore_index, loss, dX, dW, workspace, ws_total(N, H, V), stream);
+  return sync_call(X, W, y, N, H, V, ignore_index, loss, dX, dW, workspace, ws_layout(N, H).total, stream);
 }
 
 flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N,
@@ -929,7 +927,8 @@ flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out) {
       clusters = sms / CLUSTER;
   }
   const Plan P = make_plan(N, H, V, clusters);
-  out->workspace_bytes = static_cast<int64_t>(ws_total(N, H, V));
+  out->workspace_bytes = static_cast<int64_t>(ws_layout(N, H).total);
+  out->workspace_reorder_bytes = static_cast<int64_t>(ws_layout(N, H, true).total);
   out->vocab_chunk = VC;
   out->num_chunks = P.num_chunks;
   out->lse_splits = P.splits;

@@ -30,6 +30,7 @@ NUM_KERNEL_KINDS = 8
 EXPORTED = (
     "flce_status_string",
     "flce_workspace_size",
+    "flce_workspace_size_reorder",
     "flce_forward_backward",
     "flce_forward_backward_async",
     "flce_forward_backward_host",
@@ -60,6 +61,7 @@ class FlceError(RuntimeError):
 class PlanT(ctypes.Structure):
     _fields_ = [
         ("workspace_bytes", ctypes.c_int64),
+        ("workspace_reorder_bytes", ctypes.c_int64),
         ("vocab_chunk", ctypes.c_int32),
         ("num_chunks", ctypes.c_int32),
         ("lse_splits", ctypes.c_int32),
@@ -85,6 +87,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_status_string.restype = ctypes.c_char_p
     lib.flce_workspace_size.argtypes = [i64, i64, i64]
     lib.flce_workspace_size.restype = sz
+    lib.flce_workspace_size_reorder.argtypes = [i64, i64]
+    lib.flce_workspace_size_reorder.restype = sz
     lib.flce_forward_backward.argtypes = [vp, vp, vp, i64, i64, i64, i32, fp, vp, vp, vp, vp]
     lib.flce_forward_backward.restype = ctypes.c_int
     lib.flce_forward_backward_async.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
@@ -129,9 +133,10 @@ def _check(status: int, where: str):
         raise FlceError(status, where)
 
 
-def _stream_handle(stream) -> int:
+def _stream_handle(stream, device=None):
+    """The raw handle of ``stream``, or of the current stream of ``device``."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -139,9 +144,10 @@ def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _check_inputs(X, W, y):
-    if not (X.is_cuda and W.is_cuda and y.is_cuda):
-        raise ValueError("X, W and y must be CUDA tensors")
+def _check_tensors(X, W, y, dX=None, dW=None, workspace=None, require_cuda=True):
+    """X bf16 [N,H], W bf16 [V,H], y int32 [N], optional outputs dX bf16 [N,H]
+    and dW bf16 [V,H] and a uint8 workspace: all contiguous and on one device,
+    a CUDA device unless ``require_cuda`` is False.  Raises ValueError."""
     if X.dtype != torch.bfloat16 or W.dtype != torch.bfloat16 or y.dtype != torch.int32:
         raise ValueError("expected X, W bf16 and y int32")
     if X.dim() != 2 or W.dim() != 2 or y.dim() != 1:
@@ -150,10 +156,35 @@ def _check_inputs(X, W, y):
         raise ValueError(f"shape mismatch: X{tuple(X.shape)} W{tuple(W.shape)} y{tuple(y.shape)}")
     if not (X.is_contiguous() and W.is_contiguous() and y.is_contiguous()):
         raise ValueError("X, W and y must be contiguous")
+    for name, t, like in (("dX", dX, X), ("dW", dW, W)):
+        if t is None:
+            continue
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != tuple(like.shape) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor of shape {tuple(like.shape)}, "
+                             f"got {t.dtype} {tuple(t.shape)}")
+    if workspace is not None and (workspace.dtype != torch.uint8 or workspace.dim() != 1
+                                  or not workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous 1-D uint8 tensor")
+    devices = {t.device for t in (X, W, y, dX, dW, workspace) if t is not None}
+    if len(devices) != 1:
+        raise ValueError(f"all tensors of a call must be on one device, got {sorted(map(str, devices))}")
+    if require_cuda and X.device.type != "cuda":
+        raise ValueError("X, W and y must be CUDA tensors")
 
 
-def workspace_size(N: int, H: int, V: int) -> int:
+def _check_inputs(X, W, y):
+    _check_tensors(X, W, y)
+
+
+def workspace_size(N: int, H: int, V: int = 1) -> int:
+    """flce_workspace_size: bytes one call needs; independent of V."""
     return int(load_library().flce_workspace_size(N, H, V))
+
+
+def workspace_size_reorder(N: int, H: int) -> int:
+    """flce_workspace_size_reorder: bytes of a workspace that also holds the
+    packed copy of X, so that scattered ignored rows can be skipped."""
+    return int(load_library().flce_workspace_size_reorder(N, H))
 
 
 def plan(N: int, H: int, V: int) -> PlanT:
@@ -168,16 +199,30 @@ def packed_x_bytes(N: int, H: int) -> int:
     return (N * H * 2 + 255) // 256 * 256
 
 
-def alloc_workspace(N: int, H: int, V: int, device=None, reorder: bool | None = None) -> torch.Tensor:
+def reorder_fits(N: int, H: int, V: int, budget: float = 0.05) -> bool:
+    """Whether a workspace with the packed-X area stays within ``budget`` of the
+    N x V bf16 logit tensor that the head never stores (5% is the bound the
+    workload specification sets).  The benchmark and the full-size tests use it
+    to choose the workspace; the library itself takes whatever it is given."""
+    return workspace_size_reorder(N, H) <= budget * 2.0 * N * V
+
+
+def alloc_workspace(N: int, H: int, V: int = 1, device=None, reorder: bool = False) -> torch.Tensor:
     """A uint8 device buffer for one call (torch's allocator hands out 512-B
-    aligned blocks): flce_workspace_size bytes by default; with ``reorder`` True
-    the base size plus the N x H bf16 packed-X area whatever V is (so that
-    scattered ignored rows can always be skipped), with False the base size."""
-    if reorder is None:
-        nbytes = workspace_size(N, H, V)
-    else:
-        nbytes = workspace_size(N, H, 1) + (packed_x_bytes(N, H) if reorder else 0)
+    aligned blocks): flce_workspace_size bytes, or flce_workspace_size_reorder
+    bytes with ``reorder`` (then scattered ignored rows can be skipped).  V does
+    not change the size."""
+    nbytes = workspace_size_reorder(N, H) if reorder else workspace_size(N, H, V)
     return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def _check_aux(t, dtype, numel, device, name):
+    """A small device buffer of the call (loss, status, per-row vectors):
+    contiguous, of ``dtype`` and at least ``numel`` elements, on ``device``."""
+    if t is None:
+        return
+    if t.dtype != dtype or not t.is_contiguous() or t.numel() < numel or t.device != device:
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of {numel} elements on {device}")
 
 
 def row_order_info(workspace: torch.Tensor, stream=None):
@@ -185,8 +230,9 @@ def row_order_info(workspace: torch.Tensor, stream=None):
     token rows were reordered (valid rows first, X packed in that order) and
     how many rows had a non-ignored target.  Waits for ``stream``."""
     r, n = ctypes.c_int32(0), ctypes.c_int32(0)
-    _check(load_library().flce_row_order_info(_ptr(workspace), ctypes.byref(r), ctypes.byref(n),
-                                              _stream_handle(stream)), "flce_row_order_info")
+    with torch.cuda.device(workspace.device):
+        _check(load_library().flce_row_order_info(_ptr(workspace), ctypes.byref(r), ctypes.byref(n),
+                                                  _stream_handle(stream, workspace.device)), "flce_row_order_info")
     return bool(r.value), int(n.value)
 
 
@@ -194,15 +240,18 @@ def forward_backward(X, W, y, ignore_index: int = -100, *, dX=None, dW=None, wor
     """Synchronous call: returns (loss: float, dX, dW).  Raises FlceError on any
     host- or device-detected error."""
     lib = load_library()
-    _check_inputs(X, W, y)
+    _check_tensors(X, W, y, dX, dW, workspace)
     N, H = X.shape
     V = W.shape[0]
     dX = torch.empty_like(X) if dX is None else dX
     dW = torch.empty_like(W) if dW is None else dW
     workspace = alloc_workspace(N, H, V, X.device) if workspace is None else workspace
+    if workspace.numel() < workspace_size(N, H, V):
+        raise ValueError("workspace smaller than flce_workspace_size")
     loss = ctypes.c_float(0.0)
-    st = lib.flce_forward_backward(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, ctypes.byref(loss),
-                                   _ptr(dX), _ptr(dW), _ptr(workspace), _stream_handle(stream))
+    with torch.cuda.device(X.device):
+        st = lib.flce_forward_backward(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, ctypes.byref(loss),
+                                       _ptr(dX), _ptr(dW), _ptr(workspace), _stream_handle(stream, X.device))
     _check(st, "flce_forward_backward")
     return loss.value, dX, dW
 
@@ -211,7 +260,6 @@ def forward_backward_async(X, W, y, ignore_index: int = -100, *, out=None, works
     """Enqueues the call and returns device tensors (loss[1] f32, status[1] i32, dX, dW)
     without waiting.  ``out`` may pass preallocated (loss, status, dX, dW)."""
     lib = load_library()
-    _check_inputs(X, W, y)
     N, H = X.shape
     V = W.shape[0]
     if out is None:
@@ -219,10 +267,14 @@ def forward_backward_async(X, W, y, ignore_index: int = -100, *, out=None, works
                torch.empty(1, dtype=torch.int32, device=X.device),
                torch.empty_like(X), torch.empty_like(W))
     loss, status, dX, dW = out
+    _check_tensors(X, W, y, dX, dW, workspace)
+    _check_aux(loss, torch.float32, 1, X.device, "loss")
+    _check_aux(status, torch.int32, 1, X.device, "status")
     workspace = alloc_workspace(N, H, V, X.device) if workspace is None else workspace
-    st = lib.flce_forward_backward_async(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, _ptr(loss),
-                                         _ptr(status), _ptr(dX), _ptr(dW), _ptr(workspace),
-                                         workspace.numel(), _stream_handle(stream))
+    with torch.cuda.device(X.device):
+        st = lib.flce_forward_backward_async(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, _ptr(loss),
+                                             _ptr(status), _ptr(dX), _ptr(dW), _ptr(workspace),
+                                             workspace.numel(), _stream_handle(stream, X.device))
     _check(st, "flce_forward_backward_async")
     return loss, status, dX, dW
 
@@ -238,13 +290,12 @@ def forward_backward_ex(X, W, y, ignore_index: int = -100, *, reduction: str = "
     gradient pass.
     """
     lib = load_library()
-    _check_inputs(X, W, y)
+    _check_tensors(X, W, y, workspace=workspace)
     N, H = X.shape
     V = W.shape[0]
     dev = X.device
-    if grad_row_scale is not None and (grad_row_scale.dtype != torch.float32 or not grad_row_scale.is_cuda
-                                       or grad_row_scale.shape != (N,) or not grad_row_scale.is_contiguous()):
-        raise ValueError("grad_row_scale must be a contiguous CUDA float32 tensor of shape [N]")
+    _check_aux(grad_row_scale, torch.float32, N, dev, "grad_row_scale")
+    _check_aux(mean_count, torch.int32, 1, dev, "mean_count")
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     status = torch.empty(1, dtype=torch.int32, device=dev)
     rl = torch.empty(N, dtype=torch.float32, device=dev) if row_loss else None
@@ -252,11 +303,11 @@ def forward_backward_ex(X, W, y, ignore_index: int = -100, *, reduction: str = "
     dW = torch.empty_like(W) if grads else None
     workspace = alloc_workspace(N, H, V, dev) if workspace is None else workspace
     vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
-    if mean_count is not None and (mean_count.dtype != torch.int32 or not mean_count.is_cuda):
-        raise ValueError("mean_count must be a CUDA int32 tensor")
-    st = lib.flce_forward_backward_ex(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, REDUCTIONS[reduction],
-                                      vp(grad_row_scale), vp(mean_count), _ptr(loss), vp(rl), _ptr(status), vp(dX),
-                                      vp(dW), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    with torch.cuda.device(dev):
+        st = lib.flce_forward_backward_ex(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, REDUCTIONS[reduction],
+                                          vp(grad_row_scale), vp(mean_count), _ptr(loss), vp(rl), _ptr(status),
+                                          vp(dX), vp(dW), _ptr(workspace), workspace.numel(),
+                                          _stream_handle(stream, dev))
     _check(st, "flce_forward_backward_ex")
     return loss, status, rl, dX, dW
 
@@ -266,7 +317,7 @@ def vp_shard_stats(X, W_shard, y, v0: int, V: int, ignore_index: int = -100, *, 
     ``[v0, v0 + W_shard.shape[0])`` of a ``V``-entry vocabulary.  Returns device
     tensors (shard_lse[N], shard_zy[N], status[1]) without waiting."""
     lib = load_library()
-    _check_inputs(X, W_shard, y)
+    _check_tensors(X, W_shard, y, workspace=workspace)
     N, H = X.shape
     Vs = W_shard.shape[0]
     dev = X.device
@@ -274,8 +325,10 @@ def vp_shard_stats(X, W_shard, y, v0: int, V: int, ignore_index: int = -100, *, 
     zy = torch.empty(N, dtype=torch.float32, device=dev)
     status = torch.empty(1, dtype=torch.int32, device=dev)
     workspace = alloc_workspace(N, H, 1, dev) if workspace is None else workspace
-    st = lib.flce_vp_shard_stats(_ptr(X), _ptr(W_shard), _ptr(y), N, H, Vs, v0, V, ignore_index, _ptr(lse), _ptr(zy),
-                                 _ptr(status), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    with torch.cuda.device(dev):
+        st = lib.flce_vp_shard_stats(_ptr(X), _ptr(W_shard), _ptr(y), N, H, Vs, v0, V, ignore_index, _ptr(lse),
+                                     _ptr(zy), _ptr(status), _ptr(workspace), workspace.numel(),
+                                     _stream_handle(stream, dev))
     _check(st, "flce_vp_shard_stats")
     return lse, zy, status
 
@@ -287,26 +340,26 @@ def vp_backward(X, W_shard, y, v0: int, V: int, all_lse, all_zy, ignore_index: i
     tensors (loss[1], status[1], dX_part or None, dW_shard or None) without
     waiting.  dX_part is this shard's share of dX (sum it over the ranks)."""
     lib = load_library()
-    _check_inputs(X, W_shard, y)
+    _check_tensors(X, W_shard, y, workspace=workspace)
     N, H = X.shape
     Vs = W_shard.shape[0]
     dev = X.device
     for t in (all_lse, all_zy):
-        if t.dtype != torch.float32 or not t.is_cuda or t.dim() != 2 or t.shape[1] != N or not t.is_contiguous():
-            raise ValueError("all_lse / all_zy must be contiguous CUDA float32 tensors of shape [shards, N]")
+        if t.dtype != torch.float32 or t.device != dev or t.dim() != 2 or t.shape[1] != N or not t.is_contiguous():
+            raise ValueError(f"all_lse / all_zy must be contiguous float32 tensors of shape [shards, N] on {dev}")
     if all_lse.shape != all_zy.shape:
         raise ValueError("all_lse and all_zy differ in shape")
-    if mean_count is not None and (mean_count.dtype != torch.int32 or not mean_count.is_cuda):
-        raise ValueError("mean_count must be a CUDA int32 tensor")
+    _check_aux(mean_count, torch.int32, 1, dev, "mean_count")
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     status = torch.empty(1, dtype=torch.int32, device=dev)
     dX = torch.empty_like(X) if grads else None
     dW = torch.empty_like(W_shard) if grads else None
     workspace = alloc_workspace(N, H, 1, dev) if workspace is None else workspace
     vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
-    st = lib.flce_vp_backward(_ptr(X), _ptr(W_shard), _ptr(y), N, H, Vs, v0, V, ignore_index, all_lse.shape[0],
-                              _ptr(all_lse), _ptr(all_zy), vp(mean_count), _ptr(loss), _ptr(status), vp(dX), vp(dW),
-                              _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    with torch.cuda.device(dev):
+        st = lib.flce_vp_backward(_ptr(X), _ptr(W_shard), _ptr(y), N, H, Vs, v0, V, ignore_index, all_lse.shape[0],
+                                  _ptr(all_lse), _ptr(all_zy), vp(mean_count), _ptr(loss), _ptr(status), vp(dX),
+                                  vp(dW), _ptr(workspace), workspace.numel(), _stream_handle(stream, dev))
     _check(st, "flce_vp_backward")
     return loss, status, dX, dW
 
@@ -323,6 +376,9 @@ def cross_entropy(logits, y, ignore_index: int = -100, *, reduction: str = "mean
         raise ValueError("expected contiguous logits [N, V] and targets [N]")
     N, V = logits.shape
     dev = logits.device
+    if y.device != dev or (workspace is not None and workspace.device != dev):
+        raise ValueError("logits, targets and workspace must be on one device")
+    _check_aux(grad_row_scale, torch.float32, N, dev, "grad_row_scale")
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     status = torch.empty(1, dtype=torch.int32, device=dev)
     rl = torch.empty(N, dtype=torch.float32, device=dev) if row_loss else None
@@ -330,9 +386,10 @@ def cross_entropy(logits, y, ignore_index: int = -100, *, reduction: str = "mean
     if workspace is None:
         workspace = torch.empty(int(lib.flce_ce_workspace_size(N, V)), dtype=torch.uint8, device=dev)
     vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
-    st = lib.flce_cross_entropy(_ptr(logits), _ptr(y), N, V, ignore_index, REDUCTIONS[reduction], vp(grad_row_scale),
-                                _ptr(loss), vp(rl), _ptr(status), vp(dz), _ptr(workspace), workspace.numel(),
-                                _stream_handle(stream))
+    with torch.cuda.device(dev):
+        st = lib.flce_cross_entropy(_ptr(logits), _ptr(y), N, V, ignore_index, REDUCTIONS[reduction],
+                                    vp(grad_row_scale), _ptr(loss), vp(rl), _ptr(status), vp(dz), _ptr(workspace),
+                                    workspace.numel(), _stream_handle(stream, dev))
     _check(st, "flce_cross_entropy")
     return loss, status, rl, dz
 
@@ -348,10 +405,18 @@ def forward_backward_host(hX, hW, hy, dev_bufs, ignore_index: int = -100, *, h_o
     if h_out is None:
         h_out = (torch.empty_like(hX), torch.empty_like(hW))
     h_dX, h_dW = h_out
+    _check_tensors(hX, hW, hy, h_dX, h_dW, require_cuda=False)
+    if hX.device.type != "cpu":
+        raise ValueError("hX, hW, hy and the host outputs must be CPU tensors")
+    _check_tensors(d_X, d_W, d_y, d_dX, d_dW, ws)
+    if d_X.shape != hX.shape or d_W.shape != hW.shape:
+        raise ValueError("device buffers must have the host tensors' shapes")
     loss = ctypes.c_float(0.0)
-    st = lib.flce_forward_backward_host(_ptr(hX), _ptr(hW), _ptr(hy), N, H, V, ignore_index, ctypes.byref(loss),
-                                        _ptr(h_dX), _ptr(h_dW), _ptr(d_X), _ptr(d_W), _ptr(d_y), _ptr(d_dX),
-                                        _ptr(d_dW), _ptr(ws), ws.numel(), _stream_handle(stream))
+    with torch.cuda.device(d_X.device):
+        st = lib.flce_forward_backward_host(_ptr(hX), _ptr(hW), _ptr(hy), N, H, V, ignore_index,
+                                            ctypes.byref(loss), _ptr(h_dX), _ptr(h_dW), _ptr(d_X), _ptr(d_W),
+                                            _ptr(d_y), _ptr(d_dX), _ptr(d_dW), _ptr(ws), ws.numel(),
+                                            _stream_handle(stream, d_X.device))
     _check(st, "flce_forward_backward_host")
     return loss.value, h_dX, h_dW
 
@@ -378,17 +443,22 @@ def profile_read():
 def forward_backward_noalloc(X, W, y, ignore_index: int = -100, *, dX=None, dW=None, stream=None):
     """Like :func:`forward_backward` but with no workspace: the library uses its
     fixed device scratch array (NOALLOC_SCRATCH_BYTES), for callers that cannot
-    allocate device memory.  Larger problems raise FLCE_ERR_WORKSPACE_TOO_SMALL;
-    overlapping calls race on the shared array."""
+    allocate device memory.  Problems whose flce_workspace_size exceeds it raise
+    FLCE_ERR_WORKSPACE_TOO_SMALL; overlapping calls race on the shared array.
+    The call runs with X's device current, on that device's current stream
+    unless ``stream`` is given: the scratch array the library picks is that
+    device's."""
     lib = load_library()
-    _check_inputs(X, W, y)
+    _check_tensors(X, W, y, dX, dW)
     N, H = X.shape
     V = W.shape[0]
     dX = torch.empty_like(X) if dX is None else dX
     dW = torch.empty_like(W) if dW is None else dW
     loss = ctypes.c_float(0.0)
-    st = lib.flce_forward_backward_noalloc(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index,
-                                           ctypes.byref(loss), _ptr(dX), _ptr(dW), _stream_handle(stream))
+    with torch.cuda.device(X.device):
+        st = lib.flce_forward_backward_noalloc(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index,
+                                               ctypes.byref(loss), _ptr(dX), _ptr(dW),
+                                               _stream_handle(stream, X.device))
     _check(st, "flce_forward_backward_noalloc")
     return loss.value, dX, dW
 
@@ -399,22 +469,27 @@ def probe_pass2_timeout(X, W, y, ignore_index: int = -100, *, timeout_ns: int = 
     comes, every wait bounded by ``timeout_ns``; returns the device status
     tensor int32[1] (FLCE_ERR_TIMEOUT once the stream gets there)."""
     lib = load_library()
-    _check_inputs(X, W, y)
+    _check_tensors(X, W, y, workspace=workspace)
     N, H = X.shape
     V = W.shape[0]
     loss = torch.empty(1, dtype=torch.float32, device=X.device)
     status = torch.empty(1, dtype=torch.int32, device=X.device)
     dX, dW = torch.empty_like(X), torch.empty_like(W)
     workspace = alloc_workspace(N, H, V, X.device) if workspace is None else workspace
-    _check(lib.flce_probe_pass2_timeout(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, _ptr(loss), _ptr(status),
-                                        _ptr(dX), _ptr(dW), _ptr(workspace), workspace.numel(), timeout_ns,
-                                        _stream_handle(stream)), "flce_probe_pass2_timeout")
+    with torch.cuda.device(X.device):
+        _check(lib.flce_probe_pass2_timeout(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, _ptr(loss),
+                                            _ptr(status), _ptr(dX), _ptr(dW), _ptr(workspace), workspace.numel(),
+                                            timeout_ns, _stream_handle(stream, X.device)),
+               "flce_probe_pass2_timeout")
     return status
 
 
-def probe_bounded_wait(timeout_ns: int = 1_000_000, stream=None):
+def probe_bounded_wait(timeout_ns: int = 1_000_000, stream=None, device=None):
     """Runs the bounded-wait probe and returns its device status tensor int32[3]."""
     lib = load_library()
-    st = torch.empty(3, dtype=torch.int32, device="cuda")
-    _check(lib.flce_probe_bounded_wait(timeout_ns, _ptr(st), _stream_handle(stream)), "flce_probe_bounded_wait")
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    st = torch.empty(3, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib.flce_probe_bounded_wait(timeout_ns, _ptr(st), _stream_handle(stream, dev)),
+               "flce_probe_bounded_wait")
     return st

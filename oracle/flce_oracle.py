@@ -56,8 +56,9 @@ Each shard's columns of G then give its rows of dW in full and its share of dX.
 Inputs are converted exactly to fp64 (bf16 -> fp64 is exact).  A matrix product
 (numpy/BLAS in fp64) serves as a step; nothing is blocked, fused or reordered
 beyond what the definition states, except that the functions meant for full-size
-workloads evaluate the per-row definition for a block of rows at a time so that
-the fp64 logits of a block, not of the whole batch, are in memory.
+workloads (:func:`full_loss`, :func:`full_grads` and the row-subset functions)
+evaluate the per-row definition for a block of rows at a time so that the fp64
+logits of a block, not of the whole batch, are in memory.
 """
 from __future__ import annotations
 
@@ -217,6 +218,47 @@ def dw_rows(X, W, y, vocab_rows, lse, n: int, ignore_index: int = IGNORE_INDEX, 
     G *= valid[:, None]
     G *= (1.0 / n) if n else 0.0
     return G.T @ X64
+
+
+def full_grads(X, W, y, ignore_index: int = IGNORE_INDEX, block: int = 1024, W64=None, X64=None):
+    """Steps 1-5 over every row and every vocabulary entry, with the 'mean'
+    reduction: returns (loss, dX, dW, lse, n) like :func:`flce_reference`.
+
+    The rows are taken a block at a time.  For the rows b of a block the logits
+    Z_b = X_b W^T, their lse, their row losses and G_b follow the definition
+    exactly as for the whole matrix; dX_b = G_b W is final for those rows, and
+    dW = sum over blocks of G_b^T X_b (the same sum over rows as G^T X, grouped
+    by block).  Only the fp64 logits of one block are in memory at a time.
+    """
+    W64 = _f64(W) if W64 is None else W64
+    X64 = _f64(X) if X64 is None else X64
+    y = _i64(y)
+    N = X64.shape[0]
+    V = W64.shape[0]
+    valid = valid_mask(y, V, ignore_index)
+    n = int(valid.sum())
+    inv_n = (1.0 / n) if n else 0.0
+    dX = np.empty_like(X64)
+    dW = np.zeros_like(W64)
+    lse = np.empty(N, dtype=np.float64)
+    loss_sum = 0.0
+    for b0 in range(0, N, block):
+        b1 = min(N, b0 + block)
+        rows = np.arange(b1 - b0)
+        vb = valid[b0:b1]
+        yb = np.where(vb, y[b0:b1], 0)
+        Z = X64[b0:b1] @ W64.T                     # z_ij for the block's rows
+        lse_b = log_sum_exp(Z)
+        loss_sum += float(np.where(vb, lse_b - Z[rows, yb], 0.0).sum())
+        Z -= lse_b[:, None]                        # G_b, in place of the block's logits:
+        np.exp(Z, out=Z)                           #   softmax
+        Z[rows, yb] -= 1.0                         #   minus the one-hot target
+        Z *= (vb * inv_n)[:, None]                 #   1/n on valid rows, 0 on ignored rows
+        dX[b0:b1] = Z @ W64
+        dW += Z.T @ X64[b0:b1]
+        lse[b0:b1] = lse_b
+    loss = float(loss_sum / n) if n else 0.0
+    return loss, dX, dW, lse, n
 
 
 # ---------------------------------------------------------------------------

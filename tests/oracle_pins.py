@@ -242,6 +242,64 @@ def pin_row_functions(orc):
     _close(orc.row_lse(X, W, rows), lse[rows], 1e-14, what="row_lse subset")
 
 
+def pin_full_grads(orc):
+    """The blocked whole-tensor gradients used at full size equal the whole-matrix
+    definition, on a case whose last block is ragged, one of whose blocks holds
+    only ignored rows and whose targets include the first and last entries."""
+    X, W, y = _case(95, 300, 24, 530, n_ign=20)
+    y[64:128] = IGN          # block 1 (of 64-row blocks) is all ignored
+    y[3], y[200] = 0, 529
+    loss, dX, dW, lse, n = orc.flce_reference(X, W, y)
+    l2, dX2, dW2, lse2, n2 = orc.full_grads(X, W, y, block=64)
+    assert n2 == n and abs(l2 - loss) <= 1e-13 * abs(loss), (l2, loss)
+    _close(lse2, lse, 1e-14, what="blocked lse")
+    _close(dX2, dX, 1e-12, atol=1e-18, what="blocked dX")
+    _close(dW2, dW, 1e-12, atol=1e-18, what="blocked dW")
+    assert np.all(dX2[y == IGN] == 0.0)
+    # one block covering every row, and no valid row at all
+    l3, dX3, dW3, _, _ = orc.full_grads(X, W, y, block=1000)
+    assert abs(l3 - loss) <= 1e-13 * abs(loss)
+    _close(dW3, dW, 1e-12, atol=1e-18, what="single-block dW")
+    l4, dX4, dW4, _, n4 = orc.full_grads(X, W, np.full(300, IGN), block=64)
+    assert n4 == 0 and l4 == 0.0 and not dX4.any() and not dW4.any()
+
+
+def _bf16_value(bits: int) -> float:
+    """The number a bf16 bit pattern encodes (sign, 8-bit exponent, 7-bit
+    fraction, bias 127), decoded by hand."""
+    bits = int(bits)
+    sign = -1.0 if bits & 0x8000 else 1.0
+    e = (bits >> 7) & 0xFF
+    f = bits & 0x7F
+    if e == 0:
+        return sign * math.ldexp(f, -126 - 7)
+    return sign * math.ldexp(128 + f, e - 127 - 7)
+
+
+def pin_torch_inputs(orc):
+    """The tensors the GPU tests feed (torch bf16 on the CPU, int32 targets) reach
+    the oracle as the exact numbers their bit patterns encode, and the head gives
+    the same result for them as for those numbers given as fp64 arrays."""
+    bits = [0x3F80, 0xC000, 0x0001, 0x007F, 0x0080, 0x7F7F, 0x3F81, 0x8000, 0xBEAA, 0x4B80, 0x3C23]
+    t = torch.tensor(np.array(bits, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)
+    got = orc._f64(t)
+    assert got.dtype == np.float64
+    want = np.array([_bf16_value(b) for b in bits])
+    assert np.array_equal(got, want), (got, want)
+    r = _rng(97)
+    Xb = torch.tensor(r.integers(-2**15, 2**15, size=(5, 8)).astype(np.int16)).view(torch.bfloat16)
+    Wb = torch.tensor(r.integers(-2**15, 2**15, size=(9, 8)).astype(np.int16)).view(torch.bfloat16)
+    # keep finite, moderate values: clear the top exponent bits
+    Xb = (Xb.view(torch.int16) & 0x3FFF).view(torch.bfloat16)
+    Wb = (Wb.view(torch.int16) & 0x3FFF).view(torch.bfloat16)
+    yt = torch.tensor([0, 8, IGN, 4, 2], dtype=torch.int32)
+    dec = lambda a: np.vectorize(_bf16_value)(a.view(torch.int16).numpy().astype(np.uint16).astype(np.int64))  # noqa: E731
+    l1, dX1, dW1, _, _ = orc.flce_reference(Xb, Wb, yt)
+    l2, dX2, dW2, _, _ = orc.flce_reference(dec(Xb), dec(Wb), yt.numpy().astype(np.int64))
+    assert l1 == l2 and np.array_equal(dX1, dX2) and np.array_equal(dW1, dW2)
+    assert np.array_equal(orc._i64(yt), np.array([0, 8, IGN, 4, 2]))
+
+
 def pin_reductions(orc):
     """'sum' is n times 'mean' (loss and both gradients); 'none' with per-row
     upstream weights g equals torch autograd of sum_i g_i * CE_i (reduction
@@ -329,6 +387,6 @@ ALL_PINS = [
     pin_zero_weight, pin_zero_input, pin_two_class, pin_large_logits,
     pin_torch_autograd, pin_finite_difference, pin_rows_of_g_sum_to_zero,
     pin_shift_invariance, pin_ignored_rows, pin_no_valid_rows, pin_target_range,
-    pin_permutations, pin_equal_logits, pin_row_functions, pin_reductions, pin_ce_on_logits,
-    pin_vocab_shards,
+    pin_permutations, pin_equal_logits, pin_row_functions, pin_full_grads, pin_torch_inputs, pin_reductions,
+    pin_ce_on_logits, pin_vocab_shards,
 ]

@@ -53,18 +53,22 @@ def test_status_strings(lib):
 
 def test_workspace_size_by_vocab(lib):
     from lm_head_linear_03_b200 import flce
-    # the base size depends on N and H only; a vocabulary large enough that the
-    # packed-X area (N x H bf16) keeps the whole within 5% of the logits adds it
-    base = flce.workspace_size(8192, 4096, 1)
-    area = 8192 * 4096 * 2
-    for v in (1, 2, 4096, 32064, 128256, 256000, 1 << 24):
-        want = base + area if (base + area) <= 0.05 * 8192 * v * 2 else base
-        assert flce.workspace_size(8192, 4096, v) == want, v
-    assert flce.workspace_size(4096, 2304, 256000) == flce.workspace_size(4096, 2304, 1) + 4096 * 2304 * 2
+    # the size depends on N and H only: the same for every vocabulary
+    sizes = {flce.workspace_size(8192, 4096, v) for v in (1, 2, 4096, 32064, 128256, 256000, 1 << 24)}
+    assert len(sizes) == 1, sizes
+    base = sizes.pop()
+    # the workspace that lets a call reorder token rows adds the N x H bf16 area
+    assert flce.workspace_size_reorder(8192, 4096) == base + 8192 * 4096 * 2
+    assert flce.workspace_size_reorder(4096, 2304) == flce.workspace_size(4096, 2304, 256000) + 4096 * 2304 * 2
+    assert flce.workspace_size_reorder(300, 136) == flce.workspace_size(300, 136, 5) + (300 * 136 * 2 + 255) // 256 * 256
     # the Llama-3-8B head workload stays within 5% of its N x V x 2-byte logits
     assert flce.workspace_size(8192, 4096, 128256) <= 0.05 * 8192 * 128256 * 2
+    # the benchmark's choice: the reorder workspace where it stays within that 5%
+    assert not flce.reorder_fits(8192, 4096, 128256)
+    assert flce.reorder_fits(4096, 2304, 256000)
     assert flce.workspace_size(0, 4096, 10) == 0
     assert flce.workspace_size(16, 12, 10) == 0  # H % 8 != 0
+    assert flce.workspace_size_reorder(16, 12) == 0
 
 
 def test_plan_is_host_only(lib):
@@ -73,7 +77,8 @@ def test_plan_is_host_only(lib):
     assert p.vocab_chunk == 2048 and p.num_chunks == 63
     assert 1 <= p.lse_splits <= 64
     assert p.launches == 6  # prep, row order, pass 1, combine, pass 2, dX scatter
-    assert flce.plan(4096, 2304, 256000).launches == 7  # and the X pack (packed-X area fits)
+    assert p.workspace_bytes == flce.workspace_size(8192, 4096, 128256)
+    assert p.workspace_reorder_bytes == flce.workspace_size_reorder(8192, 4096)
 
 
 def test_argument_errors_before_any_launch(lib):
@@ -111,9 +116,10 @@ def _reorder_rule(valid):
 
 
 def test_row_order_rule_on_the_workloads(lib):
-    """Which of the named workloads take the reordered path with the default
-    workspace: the rule must say so and the packed-X area must fit the 5%
-    budget (host mirror of the device rule; the GPU tests check the device)."""
+    """Which of the named workloads take the reordered path with the workspace
+    the benchmark gives them: the rule must say so and the packed-X area must
+    fit the 5% budget (host mirror of the device rule; the GPU tests check the
+    device)."""
     import torch
     from lm_head_linear_03_b200 import flce
     from lm_head_linear_03_b200.inputs import WORKLOADS, make_targets
@@ -122,5 +128,48 @@ def test_row_order_rule_on_the_workloads(lib):
     for name, want in expect.items():
         w = WORKLOADS[name]
         y = make_targets(w, torch.Generator().manual_seed(w.seed))
-        has_area = flce.workspace_size(w.N, w.H, w.V) > flce.workspace_size(w.N, w.H, 1)
+        has_area = flce.reorder_fits(w.N, w.H, w.V)
         assert (_reorder_rule((y != -100).tolist()) and has_area) == want, name
+
+
+def test_binding_checks_outputs_before_any_call(lib):
+    """The binding rejects, on the host, output buffers of the wrong shape,
+    dtype or layout and tensors spread over several devices, before it hands
+    any pointer to the library."""
+    import torch
+    from lm_head_linear_03_b200 import flce
+    X = torch.zeros(16, 8, dtype=torch.bfloat16)
+    W = torch.zeros(32, 8, dtype=torch.bfloat16)
+    y = torch.zeros(16, dtype=torch.int32)
+    flce._check_tensors(X, W, y, torch.empty_like(X), torch.empty_like(W), require_cuda=False)
+    bad = [
+        dict(dX=torch.empty(15, 8, dtype=torch.bfloat16)),                 # too few rows
+        dict(dX=torch.empty(16, 8, dtype=torch.float32)),                  # wrong dtype
+        dict(dW=torch.empty(8, 32, dtype=torch.bfloat16).t()),             # not contiguous
+        dict(dW=torch.empty(33, 8, dtype=torch.bfloat16)),                 # wrong vocabulary size
+        dict(workspace=torch.empty(64, dtype=torch.int32)),                # workspace not bytes
+        dict(dX=torch.empty(16, 8, dtype=torch.bfloat16, device="meta")),  # another device
+    ]
+    for kw in bad:
+        with pytest.raises(ValueError):
+            flce._check_tensors(X, W, y, require_cuda=False, **kw)
+    with pytest.raises(ValueError, match="CUDA"):
+        flce.forward_backward(X, W, y)
+    with pytest.raises(ValueError, match="dX"):
+        flce.forward_backward(X, W, y, dX=torch.empty(15, 8, dtype=torch.bfloat16))
+
+
+def test_noalloc_limit_is_the_base_size(lib):
+    """The allocation-free entry takes any problem whose flce_workspace_size fits
+    its fixed scratch, even when the reorder workspace does not (it then keeps
+    the caller's row order); larger ones are rejected on the host."""
+    from lm_head_linear_03_b200 import flce
+    N, H, V = 1000, 4096, 256000
+    assert flce.workspace_size(N, H, V) <= flce.NOALLOC_SCRATCH_BYTES < flce.workspace_size_reorder(N, H)
+    assert flce.workspace_size(2000, 4096, V) > flce.NOALLOC_SCRATCH_BYTES
+    i64 = ctypes.c_int64
+    f = ctypes.c_float(0)
+    fake = ctypes.c_void_p(1 << 20)
+    # too large: rejected before the library looks at the device or the pointers
+    assert lib.flce_forward_backward_noalloc(fake, fake, fake, i64(2000), i64(4096), i64(V), -100, ctypes.byref(f),
+                                             fake, fake, None) == 3

@@ -52,6 +52,14 @@ MUTATIONS = [
      "G = np.exp(Z - np.asarray(lse_rows, dtype=np.float64)[::-1][:, None])"),
     ("dW rows keep ignored rows", "    G *= valid[:, None]\n    G *= (1.0 / n) if n else 0.0\n    return G.T @ X64",
      "    G *= (1.0 / n) if n else 0.0\n    return G.T @ X64"),
+    ("blocked gradients drop the ragged last block", "    for b0 in range(0, N, block):",
+     "    for b0 in range(0, N - N % block, block):"),
+    ("blocked G keeps ignored rows", "Z *= (vb * inv_n)[:, None]", "Z *= inv_n"),
+    ("blocked dW takes the first block's rows of X", "dW += Z.T @ X64[b0:b1]", "dW += Z.T @ X64[:b1 - b0]"),
+    ("blocked one-hot added", "Z[rows, yb] -= 1.0", "Z[rows, yb] += 1.0"),
+    ("blocked loss over all rows' count", "    loss = float(loss_sum / n) if n else 0.0",
+     "    loss = float(loss_sum / N) if n else 0.0"),
+    ("bf16 tensors converted through fp16", "            a = a.float()", "            a = a.half().float()"),
 ]
 
 

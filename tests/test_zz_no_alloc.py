@@ -63,7 +63,7 @@ def test_noalloc_reorders_rows_when_its_scratch_has_room():
     from lm_head_linear_03_b200 import flce
     from oracle import flce_oracle as O
     w = custom("noalloc_reorder", N=1100, H=256, V=5000, ignore_frac=0.5)
-    assert flce.workspace_size(w.N, w.H, 1) + flce.packed_x_bytes(w.N, w.H) <= flce.NOALLOC_SCRATCH_BYTES
+    assert flce.workspace_size_reorder(w.N, w.H) <= flce.NOALLOC_SCRATCH_BYTES
     X, W, y = make_inputs(w)
     loss, dX, dW = flce.forward_backward_noalloc(X.cuda(), W.cuda(), y.cuda())
     rl, rdX, rdW, _, _ = O.flce_reference(X, W, y)
@@ -71,3 +71,22 @@ def test_noalloc_reorders_rows_when_its_scratch_has_room():
     assert_grad_close(dX.float().cpu().numpy().astype("float64"), rdX, "dX")
     assert_grad_close(dW.float().cpu().numpy().astype("float64"), rdW, "dW")
     assert torch.count_nonzero(dX[(y == -100).cuda()]).item() == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_keeps_the_order_when_only_the_base_size_fits():
+    """A problem whose flce_workspace_size fits the fixed scratch but whose
+    reorder workspace does not is accepted; the call keeps the caller's row
+    order and still matches the oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from lm_head_linear_03_b200 import flce
+    from oracle import flce_oracle as O
+    w = custom("noalloc_base_only", N=1000, H=4096, V=3000, ignore_frac=0.5)
+    assert flce.workspace_size(w.N, w.H, w.V) <= flce.NOALLOC_SCRATCH_BYTES < flce.workspace_size_reorder(w.N, w.H)
+    X, W, y = make_inputs(w)
+    loss, dX, dW = flce.forward_backward_noalloc(X.cuda(), W.cuda(), y.cuda())
+    rl, rdX, rdW, _, _ = O.flce_reference(X, W, y)
+    assert_loss_close(loss, rl)
+    assert_grad_close(dX.float().cpu().numpy().astype("float64"), rdX, "dX")
+    assert_grad_close(dW.float().cpu().numpy().astype("float64"), rdW, "dW")
