@@ -651,15 +651,15 @@ def run_pref(args, world, rank, local):
     N, H, V = w.N, w.H, w.V
     seq_len = 1024 if N >= 2048 else max(2, N // 2)
     rows = torch.arange(N, device=dev)
-    seq = rows // seq_len
     y = torch.where(rows % seq_len < seq_len // 4, torch.full_like(y, -100), y).contiguous()
-    S = int(seq.max().item()) + 1
-    chosen = torch.arange(0, S - 1, 2, device=dev)
+    S = -(-N // seq_len)
+    seq_start = torch.tensor([min(N, s * seq_len) for s in range(S + 1)], dtype=torch.int32, device=dev)
+    chosen = torch.arange(0, S - 1, 2, dtype=torch.int32, device=dev)
     rejected = chosen + 1
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        preference_forward_backward(X, W, y, seq, chosen, rejected, beta=0.1)
+        preference_forward_backward(X, W, y, seq_start, chosen, rejected, beta=0.1)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -689,11 +689,11 @@ def run_pref(args, world, rank, local):
                    "seq_len": seq_len, "prompt_rows_per_sequence": seq_len // 4},
         "fused_mean_ce_ms": fused_ms,
         "pref_over_fused": ms / fused_ms,
-        "gpu_launches": 10 * args.steps,
+        "gpu_launches": 13 * args.steps,
         "clocks": clocks,
-        "note": "this library's launches per step: forward-only head call (prep, row order, pass 1, combine) and "
-                "full head call (prep, row order, pass 1, combine, pass 2, scatter); host syncs for the "
-                "sequence count and the status checks fall inside the step",
+        "note": "this library's launches per step: forward-only head call (prep, row order, pass 1, combine), "
+                "the pair loss (sequence sums, pairs, row weights) and the full head call (prep, row order, "
+                "pass 1, combine, pass 2, scatter); the status checks' host syncs fall inside the step",
     }
     print(json.dumps(line), flush=True)
 

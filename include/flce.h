@@ -153,6 +153,28 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
                                          void* workspace, size_t workspace_bytes,
                                          cudaStream_t stream);
 
+/* Data-parallel entry whose dW can be reduced while the call still runs.
+ * Enqueues the mean-reduced call of flce_forward_backward_ex (d_mean_count:
+ * DEVICE int32 or NULL, as there) with the gradient pass split into
+ * `sections` launches over consecutive ranges of vocabulary chunks (1 ..
+ * 8; at most one per 2048-entry chunk).  After section k the call records
+ * section_done[k] (caller-created CUDA events) on `stream`; from then on dW rows
+ * [section_rows[k], section_rows[k+1]) are final, so the caller can start
+ * reducing them over the data-parallel ranks on another stream (e.g. an NCCL
+ * all-reduce after cudaStreamWaitEvent) while the later sections compute.
+ * section_rows: HOST int64 [sections + 1], filled before the call returns;
+ * sections beyond the number of chunks are empty and complete with the last.
+ * Other arguments and results as flce_forward_backward_async; the results
+ * are those of an unsplit call (the same sums in the same order).  The split
+ * follows from the pages' method: the gradient is computed chunk by chunk
+ * over the vocabulary ("Liger Kernel explained", cross-entropy head section),
+ * so the dW rows of a chunk are complete when its chunk is. */
+flce_status_t flce_forward_backward_sections(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N,
+                                             int64_t H, int64_t V, int32_t ignore_index, const int32_t* d_mean_count,
+                                             float* d_loss, int32_t* d_status, uint16_t* dX, uint16_t* dW,
+                                             void* workspace, size_t workspace_bytes, int32_t sections,
+                                             cudaEvent_t* section_done, int64_t* section_rows, cudaStream_t stream);
+
 /* Reductions of flce_forward_backward_ex.  All three are one weighted sum over
  * the non-ignored rows, loss = sum_i s_i l_i with l_i = lse_i - z_{i,y_i}, and
  * dX, dW are the gradients of that loss (G_ij = s_i (softmax_ij - [j == y_i])):
@@ -233,6 +255,46 @@ flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64
                                  int32_t ignore_index, int32_t reduction, const float* grad_row_scale,
                                  float* d_loss, float* d_row_loss, int32_t* d_status, uint16_t* dlogits,
                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Number of targets y_i != ignore_index among y[0..N), written to the DEVICE
+ * int32 *d_count when the stream gets there (an exact integer count).  It is
+ * the denominator of the token mean; a data-parallel caller all-reduces it
+ * over the ranks and passes the sum as d_mean_count of
+ * flce_forward_backward_ex, so that every rank's loss and dW are shares of
+ * the whole batch's.  y: DEVICE int32 [N].  Asynchronous. */
+flce_status_t flce_count_valid(const int32_t* y, int64_t N, int32_t ignore_index, int32_t* d_count,
+                               cudaStream_t stream);
+
+/* Pairwise logistic (DPO-form) preference loss on the head's per-row losses.
+ * The post-training losses of the library the pages describe ("Liger-Kernel:
+ * Triton kernels that replace HF training ops", section "Installation and the
+ * one-line patch": ORPO, DPO, CPO, SimPO ... called with the LM-head weight,
+ * the hidden states and the targets, returning the loss) build on two things
+ * the fused head gives without the logits: each target's log-probability,
+ * -l_i (flce_forward_backward_ex with reduction NONE and d_row_loss), and the
+ * gradient of a loss of their per-sequence sums (the same entry with
+ * grad_row_scale).  This entry is the step between them:
+ *   sequence s = token rows [seq_start[s], seq_start[s+1]),
+ *   logp_s = -sum of their row losses,
+ *   m_k = beta ((logp_c - ref_c) - (logp_r - ref_r)) for pair k with
+ *         c = chosen[k], r = rejected[k] (ref_logp NULL: ref = 0),
+ *   loss = -(1/P) sum_k log sigmoid(m_k),
+ *   grad_logp[s] = d loss / d logp_s,
+ *   row_weight[i] = -grad_logp[s] for a row i of sequence s whose target is
+ *                   not ignore_index, 0 for every other row: the upstream
+ *                   gradient of l_i, to pass as grad_row_scale.
+ * Arguments (all DEVICE, caller-owned): d_row_loss fp32 [N], y int32 [N],
+ * d_seq_start int32 [S+1] (non-decreasing, within [0, N]), d_chosen and
+ * d_rejected int32 [P] (sequence ids in [0, S)), d_ref_logp fp64 [S] or NULL;
+ * outputs d_loss fp64 [1], d_logp and d_grad_logp fp64 [S], d_row_weight
+ * fp32 [N], d_status int32 [1].  Sums are fp64 in a fixed order, so the result
+ * is the same on every call.  Sequence bounds or pair ids out of range set
+ * FLCE_ERR_INVALID_ARGUMENT in d_status.  Asynchronous. */
+flce_status_t flce_pairwise_logistic(const float* d_row_loss, const int32_t* y, int64_t N, int32_t ignore_index,
+                                     const int32_t* d_seq_start, int32_t S, const int32_t* d_chosen,
+                                     const int32_t* d_rejected, int32_t P, double beta, const double* d_ref_logp,
+                                     double* d_loss, double* d_logp, double* d_grad_logp, float* d_row_weight,
+                                     int32_t* d_status, cudaStream_t stream);
 
 /* Allocation-free variant of flce_forward_backward, for callers that cannot
  * allocate device memory: a plug-in or custom operator that is handed only the

@@ -8,12 +8,15 @@ ABI is declared in ``include/flce.h``; ``flce.py`` is its ctypes binding.
 from .flce import (  # noqa: F401
     FlceError,
     alloc_workspace,
+    count_valid,
     cross_entropy,
     forward_backward,
     forward_backward_async,
     forward_backward_ex,
     forward_backward_host,
+    forward_backward_sections,
     load_library,
+    pairwise_logistic,
     plan,
     profile_enable,
     profile_read,

@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <climits>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -56,9 +57,9 @@ WsLayout ws_layout(int64_t N, int64_t H, bool packed = false) {
   const size_t n = static_cast<size_t>(N);
   const size_t nblk = (n + COMBINE_THREADS - 1) / COMBINE_THREADS;
   L.ctrl = take(256);
-  // pass-2 completion counters: g_row[TM], x_row[TM], g_col[VC/BN], w_col[VC/BN]
+  // pass-2 completion counters: g_row[TM], x_row[TM], g_col[VC/BN], w_col[VC/SUBN]
   const size_t tm = (n + CM - 1) / CM;
-  L.counters_bytes = (2 * tm + 2 * (VC / BN)) * 4;
+  L.counters_bytes = (2 * tm + 2 * (VC / SUBN)) * 4;
   L.counters = take(L.counters_bytes);
   L.tile_cnt = take(tm * 4);
   L.tile_valid = take(tm * 4);
@@ -200,6 +201,16 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
   return r == CUDA_SUCCESS;
 }
 
+// K-blocks of the stagger at each end of a tile (1 .. MAX_LAG).
+int stagger_lag() {
+  static const int lag = [] {
+    const char* e = getenv("FLCE_LAG");
+    const int v = e ? atoi(e) : 2;
+    return std::max(1, std::min(MAX_LAG, v));
+  }();
+  return lag;
+}
+
 // ------------------------------------------------------------------ plan --
 struct Plan {
   int tiles_m;        // 256-token tiles (one per SM pair)
@@ -311,7 +322,8 @@ struct PipeCtx {
   cudaEvent_t w_ready[MAX_PIECES] = {};  // recorded on `copy` after piece i's copy
   int groups = 0;                      // pass-2 launches
   cudaEvent_t p2_done[MAX_PIECES] = {};
-  uint16_t* h_dW = nullptr;            // host dW, filled group by group on `copy`
+  uint16_t* h_dW = nullptr;            // host dW, filled group by group on `copy` (null: no copies)
+  int64_t* section_rows = nullptr;     // if set: dW rows [section_rows[k], section_rows[k+1]) of section k
 };
 
 // Per-device copy stream and events of the host-buffer entry, made on first
@@ -396,13 +408,13 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
 
   CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn, mHi, mLo, mXc_k, mXc_mn;
   const uint64_t n = static_cast<uint64_t>(N), h = static_cast<uint64_t>(H), v = static_cast<uint64_t>(V);
-  bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BNH) &&
+  bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, SUBNH) &&
             make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
             make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK) &&
             // the packed copy of X (the caller's X stands in when there is none: never read then)
             make_map(&mXc_k, Xc ? Xc : X, h, n, h * 2, BK, BM) && make_map(&mXc_mn, Xc ? Xc : X, h, n, h * 2, 64, BK) &&
-            (dX == nullptr || (make_map(&mHi, dX, h, n, h * 2, BN, BM, Swz::none) &&
-                               make_map(&mLo, lo, h, n, h * 2, BN, BM, Swz::none)));
+            (dX == nullptr || (make_map(&mHi, dX, h, n, h * 2, SUBN, BM, Swz::none) &&
+                               make_map(&mLo, lo, h, n, h * 2, SUBN, BM, Swz::none)));
   // 32 x 32 output boxes of the epilogues (64-byte swizzle)
   CUtensorMap mGo, mDWo, mHio, mLoo;
   ok = ok && (dX == nullptr || (make_map(&mGo, G, VC, n, VC * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
@@ -440,6 +452,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   a.tile_valid = reinterpret_cast<const int*>(ws + L.tile_valid);
   a.perm = perm;
   a.reordered = &ctrl->reordered;
+  a.lag = stagger_lag();
 
   // Valid rows per 256-row token tile, then the token-row order of both passes.
   {
@@ -470,7 +483,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   // Pass 1: logits tile by tile, online log-sum-exp per (row, split); a call
   // given every vocabulary shard's statistics has its lse already.
   int total_splits = P.splits;
-  if (opt.combine != COMBINE_SHARDS_IN && opt.pipe == nullptr) {
+  if (opt.combine != COMBINE_SHARDS_IN && (opt.pipe == nullptr || opt.pipe->pieces == 0)) {
     GemmArgs p1 = a;
     p1.tiles_m = P.tiles_m;
     p1.tiles_n = P.vtiles;
@@ -489,7 +502,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     for (int i = 0; i < pp.pieces; ++i) {
       const int64_t v0 = pp.piece_v[i], vp = pp.piece_v[i + 1] - pp.piece_v[i];
       CUtensorMap mWp;
-      if (!make_map(&mWp, W + v0 * H, h, static_cast<uint64_t>(vp), h * 2, BK, BNH)) return FLCE_ERR_CUDA;
+      if (!make_map(&mWp, W + v0 * H, h, static_cast<uint64_t>(vp), h * 2, BK, SUBNH)) return FLCE_ERR_CUDA;
       GemmArgs p1 = a;
       p1.V = static_cast<int>(vp);
       p1.v_off = static_cast<int>(v0);
@@ -553,16 +566,23 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     b.TM = P.tiles_m;
     b.HN = static_cast<int>((H + BN - 1) / BN);
     b.C = P.num_chunks;
+    const int64_t v_last = V - static_cast<int64_t>(P.num_chunks - 1) * VC;  // vocabulary of the last chunk
     b.VTf = VC / BN;
-    b.VT_last = static_cast<int>((V - static_cast<int64_t>(P.num_chunks - 1) * VC + BN - 1) / BN);
-    if (b.C == 1) b.VTf = b.VT_last;
+    b.VT_last = static_cast<int>((v_last + BN - 1) / BN);
+    b.VMf = VC / SUBN;
+    b.VM_last = static_cast<int>((v_last + SUBN - 1) / SUBN);
+    if (b.C == 1) {
+      b.VTf = b.VT_last;
+      b.VMf = b.VM_last;
+    }
+    auto vt_of = [&](int c) { return static_cast<long long>(c == b.C - 1 ? b.VT_last : b.VTf); };
+    auto vm_of = [&](int c) { return static_cast<long long>(c == b.C - 1 ? b.VM_last : b.VMf); };
     // section_end[c]: end of the queue's section c (dX(c) dW(c) G(c+1)), after G(0)
     std::vector<long long> section_end(b.C);
-    long long total = static_cast<long long>(b.C == 1 ? b.VT_last : b.VTf) * b.TM;  // G(0)
+    long long total = vt_of(0) * b.TM;  // G(0)
     for (int c = 0; c < b.C; ++c) {
-      const long long vt = c == b.C - 1 ? b.VT_last : b.VTf;
-      total += static_cast<long long>(b.TM) * b.HN + vt * b.HN;
-      if (c + 1 < b.C) total += static_cast<long long>(c + 1 == b.C - 1 ? b.VT_last : b.VTf) * b.TM;
+      total += static_cast<long long>(b.TM) * b.HN + vm_of(c) * b.HN;
+      if (c + 1 < b.C) total += vt_of(c + 1) * b.TM;
       section_end[c] = total;
     }
     b.total_items = total;
@@ -573,7 +593,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     b.g_row = ctr;
     b.x_row = ctr + b.TM;
     b.g_col = ctr + 2 * b.TM;
-    b.w_col = ctr + 2 * b.TM + VC / BN;
+    b.w_col = ctr + 2 * b.TM + VC / BN;  // VC / SUBN entries
     Pass2Maps pm;
     pm.Xk = mX_k;
     pm.Wk = mW_k;
@@ -606,10 +626,14 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       if (opt.pipe) {  // dW rows of chunks c0 .. c1-1 are final
         const PipeCtx& pp = *opt.pipe;
         const int64_t r0 = static_cast<int64_t>(c0) * VC, r1 = std::min<int64_t>(V, static_cast<int64_t>(c1) * VC);
-        if (cudaEventRecord(pp.p2_done[k], stream) != cudaSuccess ||
-            cudaStreamWaitEvent(pp.copy, pp.p2_done[k], 0) != cudaSuccess ||
-            cudaMemcpyAsync(pp.h_dW + r0 * H, dW + r0 * H, static_cast<size_t>(r1 - r0) * H * 2,
-                            cudaMemcpyDeviceToHost, pp.copy) != cudaSuccess)
+        if (pp.section_rows) {
+          pp.section_rows[k] = r0;
+          pp.section_rows[k + 1] = r1;
+        }
+        if (cudaEventRecord(pp.p2_done[k], stream) != cudaSuccess) return FLCE_ERR_CUDA;
+        if (pp.h_dW && (cudaStreamWaitEvent(pp.copy, pp.p2_done[k], 0) != cudaSuccess ||
+                        cudaMemcpyAsync(pp.h_dW + r0 * H, dW + r0 * H, static_cast<size_t>(r1 - r0) * H * 2,
+                                        cudaMemcpyDeviceToHost, pp.copy) != cudaSuccess))
           return FLCE_ERR_CUDA;
       }
     }
@@ -755,11 +779,13 @@ flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64
   c.row_loss = d_row_loss;
   c.blk_sum = reinterpret_cast<double*>(ws + L.blk_sum);
   c.ticket = reinterpret_cast<unsigned int*>(ws + L.ctrl + 4);
+  c.n_valid = reinterpret_cast<const int*>(ws + L.ctrl + 8);
   c.loss = d_loss;
   c.status = d_status;
   size_t slot;
   prof_begin(stream, KIND_PREP, &slot);
-  flce_prep_kernel<<<TM, CM, 0, stream>>>(y, c.N, ignore_index, reinterpret_cast<int*>(ws + L.tile_valid));
+  flce_prep_kernel<<<TM, CM, 0, stream>>>(y, c.N, ignore_index, reinterpret_cast<int*>(ws + L.tile_valid),
+                                          reinterpret_cast<int*>(ws + L.ctrl + 8));
   prof_end(stream, slot);
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   const int grid = static_cast<int>(std::min<int64_t>(N, static_cast<int64_t>(di.num_sms) * 4 * 64));
@@ -772,6 +798,69 @@ flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64
   prof_end(stream, slot);
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   return FLCE_OK;
+}
+
+flce_status_t flce_count_valid(const int32_t* y, int64_t N, int32_t ignore_index, int32_t* d_count,
+                               cudaStream_t stream) {
+  if (!y || !d_count || N <= 0 || N > (1ll << 30)) return FLCE_ERR_INVALID_ARGUMENT;
+  if (!aligned(y, 4) || !aligned(d_count, 4)) return FLCE_ERR_UNSUPPORTED;
+  DevInfo di;
+  int dev;
+  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
+  if (cudaMemsetAsync(d_count, 0, sizeof(int32_t), stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  const int tiles = static_cast<int>((N + CM - 1) / CM);
+  size_t slot;
+  prof_begin(stream, KIND_PREP, &slot);
+  flce_prep_kernel<<<tiles, CM, 0, stream>>>(y, static_cast<int>(N), ignore_index, nullptr, d_count);
+  prof_end(stream, slot);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+flce_status_t flce_pairwise_logistic(const float* d_row_loss, const int32_t* y, int64_t N, int32_t ignore_index,
+                                     const int32_t* d_seq_start, int32_t S, const int32_t* d_chosen,
+                                     const int32_t* d_rejected, int32_t P, double beta, const double* d_ref_logp,
+                                     double* d_loss, double* d_logp, double* d_grad_logp, float* d_row_weight,
+                                     int32_t* d_status, cudaStream_t stream) {
+  if (!d_row_loss || !y || !d_seq_start || !d_chosen || !d_rejected || !d_loss || !d_logp || !d_grad_logp ||
+      !d_row_weight || !d_status)
+    return FLCE_ERR_INVALID_ARGUMENT;
+  if (N <= 0 || N > (1ll << 30) || S <= 0 || S > (1 << 24) || P <= 0 || P > (1 << 24) || !(beta == beta))
+    return FLCE_ERR_INVALID_ARGUMENT;
+  if (!aligned(d_row_loss, 4) || !aligned(y, 4) || !aligned(d_seq_start, 4) || !aligned(d_chosen, 4) ||
+      !aligned(d_rejected, 4) || !aligned(d_ref_logp, 8) || !aligned(d_loss, 8) || !aligned(d_logp, 8) ||
+      !aligned(d_grad_logp, 8) || !aligned(d_row_weight, 4) || !aligned(d_status, 4))
+    return FLCE_ERR_UNSUPPORTED;
+  DevInfo di;
+  int dev;
+  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
+  if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess ||
+      cudaMemsetAsync(d_row_weight, 0, static_cast<size_t>(N) * sizeof(float), stream) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  PrefArgs a{};
+  a.row_loss = d_row_loss;
+  a.y = y;
+  a.seq_start = d_seq_start;
+  a.chosen = d_chosen;
+  a.rejected = d_rejected;
+  a.ref_logp = d_ref_logp;
+  a.beta = beta;
+  a.N = static_cast<int>(N);
+  a.S = S;
+  a.P = P;
+  a.ignore_index = ignore_index;
+  a.logp = d_logp;
+  a.grad_logp = d_grad_logp;
+  a.loss = d_loss;
+  a.row_weight = d_row_weight;
+  a.status = d_status;
+  flce_pref_logp_kernel<<<S, PREF_THREADS, 0, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  flce_pref_pairs_kernel<<<1, PREF_THREADS, 0, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  flce_pref_weights_kernel<<<S, PREF_THREADS, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
 namespace {
@@ -910,6 +999,40 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
   if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
   *h_loss = host.loss;
   return static_cast<flce_status_t>(host.status);
+}
+
+flce_status_t flce_forward_backward_sections(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N,
+                                             int64_t H, int64_t V, int32_t ignore_index, const int32_t* d_mean_count,
+                                             float* d_loss, int32_t* d_status, uint16_t* dX, uint16_t* dW,
+                                             void* workspace, size_t workspace_bytes, int32_t sections,
+                                             cudaEvent_t* section_done, int64_t* section_rows, cudaStream_t stream) {
+  if (!d_loss || !d_status || !section_done || !section_rows || sections < 1 || sections > MAX_PIECES)
+    return FLCE_ERR_INVALID_ARGUMENT;
+  for (int k = 0; k < sections; ++k)
+    if (!section_done[k]) return FLCE_ERR_INVALID_ARGUMENT;
+  const flce_status_t s = check_args(X, W, y, N, H, V, dX, dW, workspace);
+  if (s != FLCE_OK) return s;
+  if (!aligned(d_status, 4) || !aligned(d_loss, 4) || !aligned(d_mean_count, 4)) return FLCE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  const int chunks = static_cast<int>((V + VC - 1) / VC);
+  const int used = std::min(sections, chunks);
+  PipeCtx pp;
+  pp.pieces = 0;  // pass 1 in one launch: W is on the device already
+  pp.groups = used;
+  pp.section_rows = section_rows;
+  for (int k = 0; k < used; ++k) pp.p2_done[k] = section_done[k];
+  Options opt;
+  opt.mean_count = d_mean_count;
+  opt.pipe = &pp;
+  const flce_status_t e = enqueue(X, W, y, N, H, V, ignore_index, d_loss, d_status, dX, dW, workspace,
+                                  workspace_bytes, stream, opt);
+  if (e != FLCE_OK) return e;
+  // sections beyond the chunks hold no rows and are done with the last one
+  for (int k = used; k < sections; ++k) {
+    section_rows[k + 1] = V;
+    if (cudaEventRecord(section_done[k], stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  return FLCE_OK;
 }
 
 flce_status_t flce_plan(int64_t N, int64_t H, int64_t V, flce_plan_t* out) {

@@ -47,6 +47,9 @@ EXPORTED = (
     "flce_row_order_info",
     "flce_vp_shard_stats",
     "flce_vp_backward",
+    "flce_count_valid",
+    "flce_pairwise_logistic",
+    "flce_forward_backward_sections",
 )
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -124,6 +127,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_vp_backward.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp,
                                      vp, sz, vp]
     lib.flce_vp_backward.restype = ctypes.c_int
+    lib.flce_forward_backward_sections.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, sz, i32,
+                                                   ctypes.POINTER(vp), ctypes.POINTER(i64), vp]
+    lib.flce_forward_backward_sections.restype = ctypes.c_int
+    lib.flce_count_valid.argtypes = [vp, i64, i32, vp, vp]
+    lib.flce_count_valid.restype = ctypes.c_int
+    lib.flce_pairwise_logistic.argtypes = [vp, vp, i64, i32, vp, i32, vp, vp, i32, ctypes.c_double, vp, vp, vp, vp,
+                                           vp, vp, vp]
+    lib.flce_pairwise_logistic.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -493,3 +504,85 @@ def probe_bounded_wait(timeout_ns: int = 1_000_000, stream=None, device=None):
         _check(lib.flce_probe_bounded_wait(timeout_ns, _ptr(st), _stream_handle(stream, dev)),
                "flce_probe_bounded_wait")
     return st
+
+
+def count_valid(y, ignore_index: int = -100, *, out=None, stream=None):
+    """flce_count_valid: the number of targets != ignore_index, as a device
+    int32[1] tensor (asynchronous)."""
+    lib = load_library()
+    if y.dtype != torch.int32 or y.dim() != 1 or not y.is_contiguous() or not y.is_cuda:
+        raise ValueError("y must be a contiguous CUDA int32 tensor [N]")
+    out = torch.empty(1, dtype=torch.int32, device=y.device) if out is None else out
+    _check_aux(out, torch.int32, 1, y.device, "out")
+    with torch.cuda.device(y.device):
+        _check(lib.flce_count_valid(_ptr(y), y.numel(), ignore_index, _ptr(out), _stream_handle(stream, y.device)),
+               "flce_count_valid")
+    return out
+
+
+def pairwise_logistic(row_loss, y, seq_start, chosen, rejected, beta: float, ref_logp=None,
+                      ignore_index: int = -100, *, stream=None):
+    """flce_pairwise_logistic on device tensors: row_loss fp32 [N], y int32 [N],
+    seq_start int32 [S+1], chosen / rejected int32 [P], ref_logp fp64 [S] or
+    None.  Returns device tensors (loss fp64[1], logp fp64[S], grad_logp
+    fp64[S], row_weight fp32[N], status int32[1]) without waiting."""
+    lib = load_library()
+    dev = row_loss.device
+    N = row_loss.numel()
+    S = seq_start.numel() - 1
+    P = chosen.numel()
+    _check_aux(row_loss, torch.float32, N, dev, "row_loss")
+    _check_aux(y, torch.int32, N, dev, "y")
+    _check_aux(seq_start, torch.int32, S + 1, dev, "seq_start")
+    _check_aux(chosen, torch.int32, P, dev, "chosen")
+    _check_aux(rejected, torch.int32, P, dev, "rejected")
+    _check_aux(ref_logp, torch.float64, S, dev, "ref_logp")
+    if not row_loss.is_cuda or rejected.numel() != P or y.numel() != N:
+        raise ValueError("expected CUDA tensors, y[N] beside row_loss[N] and as many rejected as chosen ids")
+    loss = torch.empty(1, dtype=torch.float64, device=dev)
+    logp = torch.empty(S, dtype=torch.float64, device=dev)
+    grad = torch.empty(S, dtype=torch.float64, device=dev)
+    weight = torch.empty(N, dtype=torch.float32, device=dev)
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
+    with torch.cuda.device(dev):
+        _check(lib.flce_pairwise_logistic(_ptr(row_loss), _ptr(y), N, ignore_index, _ptr(seq_start), S,
+                                          _ptr(chosen), _ptr(rejected), P, float(beta), vp(ref_logp), _ptr(loss),
+                                          _ptr(logp), _ptr(grad), _ptr(weight), _ptr(status),
+                                          _stream_handle(stream, dev)), "flce_pairwise_logistic")
+    return loss, logp, grad, weight, status
+
+
+def forward_backward_sections(X, W, y, ignore_index: int = -100, *, sections: int = 4, mean_count=None, out=None,
+                              workspace=None, stream=None):
+    """flce_forward_backward_sections: the mean-reduced call with the gradient
+    pass in ``sections`` launches.  Returns (loss[1], status[1], dX, dW, events,
+    rows): ``events[k]`` (torch.cuda.Event) completes when dW rows
+    ``rows[k]:rows[k+1]`` are final.  Asynchronous."""
+    lib = load_library()
+    N, H = X.shape
+    V = W.shape[0]
+    dev = X.device
+    if out is None:
+        out = (torch.empty(1, dtype=torch.float32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
+               torch.empty_like(X), torch.empty_like(W))
+    loss, status, dX, dW = out
+    _check_tensors(X, W, y, dX, dW, workspace)
+    _check_aux(loss, torch.float32, 1, dev, "loss")
+    _check_aux(status, torch.int32, 1, dev, "status")
+    _check_aux(mean_count, torch.int32, 1, dev, "mean_count")
+    workspace = alloc_workspace(N, H, V, dev) if workspace is None else workspace
+    strm = stream if stream is not None else torch.cuda.current_stream(dev)
+    events = [torch.cuda.Event() for _ in range(sections)]
+    for e in events:  # the handle exists once the event has been recorded
+        e.record(strm)
+    handles = (ctypes.c_void_p * sections)(*[e.cuda_event for e in events])
+    rows = (ctypes.c_int64 * (sections + 1))()
+    vp = lambda t: None if t is None else _ptr(t)  # noqa: E731
+    with torch.cuda.device(dev):
+        _check(lib.flce_forward_backward_sections(_ptr(X), _ptr(W), _ptr(y), N, H, V, ignore_index, vp(mean_count),
+                                                  _ptr(loss), _ptr(status), _ptr(dX), _ptr(dW), _ptr(workspace),
+                                                  workspace.numel(), sections, handles, rows,
+                                                  ctypes.c_void_p(strm.cuda_stream)),
+               "flce_forward_backward_sections")
+    return loss, status, dX, dW, events, [int(r) for r in rows]

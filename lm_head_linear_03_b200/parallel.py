@@ -8,7 +8,10 @@ the fused head on its own tokens with the mean taken over the valid targets of
 *every* rank; the ranks' losses then add up to the batch loss and their dW to
 the batch dW, while each rank's dX is already final for its rows.  The
 exchanges are one all-reduce of the count (before the call) and all-reduces of
-the loss and dW (after it), through torch.distributed (NCCL on GPUs).
+the loss and dW (after it), through torch.distributed (NCCL on GPUs).  With
+``overlap_sections`` the gradient pass runs in sections of whole vocabulary
+chunks and each section's finished dW rows are all-reduced on a second stream
+while the later sections compute (:func:`dp_forward_backward_overlapped`).
 
 Vocabulary-parallel (:func:`vp_forward_backward`): W rows sharded over ranks in
 contiguous ranges, X and y replicated.  The loss is computed chunk by chunk
@@ -29,15 +32,22 @@ def _device_call(X, W, y, ignore_index, mean_count):
     return loss, status, dX, dW
 
 
-def dp_forward_backward(X, W, y, ignore_index: int = -100, *, group=None, local_call=None):
+def _device_count(y, ignore_index):
+    from .flce import count_valid
+    return count_valid(y, ignore_index)
+
+
+def dp_forward_backward(X, W, y, ignore_index: int = -100, *, group=None, local_call=None, count_call=None):
     """Returns (batch loss, this rank's dX, batch dW) for this rank's shard.
 
-    ``local_call(X, W, y, ignore_index, mean_count) -> (loss[1], status[1], dX, dW)``
-    runs the head on the shard with the mean over ``mean_count`` valid targets;
-    it defaults to the CUDA library.
+    ``count_call(y, ignore_index) -> int32[1]`` counts the shard's valid
+    targets and ``local_call(X, W, y, ignore_index, mean_count) -> (loss[1],
+    status[1], dX, dW)`` runs the head on the shard with the mean over
+    ``mean_count`` valid targets; both default to the CUDA library.
     """
     call = local_call or _device_call
-    n = (y != ignore_index).sum().to(torch.int32).reshape(1)
+    count = count_call or _device_count
+    n = count(y, ignore_index)
     dist.all_reduce(n, op=dist.ReduceOp.SUM, group=group)
     loss, status, dX, dW = call(X, W, y, ignore_index, n)
     bad = status.to(torch.int32).reshape(1).clone()
@@ -47,6 +57,34 @@ def dp_forward_backward(X, W, y, ignore_index: int = -100, *, group=None, local_
         raise FlceError(int(bad.item()), "dp_forward_backward")
     dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=group)
     dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=group)
+    return loss, dX, dW
+
+
+def dp_forward_backward_overlapped(X, W, y, ignore_index: int = -100, *, sections: int = 4, group=None,
+                                  workspace=None, comm_stream=None):
+    """:func:`dp_forward_backward` with the dW all-reduce overlapped with the
+    gradient pass (CUDA library and NCCL only): the call's gradient pass runs
+    in ``sections`` launches; after each one, ``comm_stream`` waits for it and
+    all-reduces the dW rows it finished, while the next section computes.
+    Returns (batch loss, this rank's dX, batch dW) like the unsplit version."""
+    from .flce import FlceError, count_valid, forward_backward_sections
+    n = count_valid(y, ignore_index)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM, group=group)
+    loss, status, dX, dW, events, rows = forward_backward_sections(X, W, y, ignore_index, sections=sections,
+                                                                   mean_count=n, workspace=workspace)
+    main = torch.cuda.current_stream(X.device)
+    comm = comm_stream or torch.cuda.Stream(device=X.device)
+    with torch.cuda.stream(comm):
+        for k, ev in enumerate(events):
+            comm.wait_event(ev)
+            if rows[k + 1] > rows[k]:
+                dist.all_reduce(dW[rows[k]:rows[k + 1]], op=dist.ReduceOp.SUM, group=group)
+    main.wait_stream(comm)
+    bad = status.clone()
+    dist.all_reduce(bad, op=dist.ReduceOp.MAX, group=group)
+    if int(bad.item()) != 0:
+        raise FlceError(int(bad.item()), "dp_forward_backward_overlapped")
+    dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=group)
     return loss, dX, dW
 
 

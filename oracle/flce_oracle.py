@@ -21,6 +21,11 @@ cross-entropy" pipeline, only without keeping the logit tensor:
   shape ``(vocab_size, hidden_size)``.
 * The same guide, section LigerCrossEntropyLoss: cross-entropy computed from a
   given ``(batch*seq, vocab)`` logit tensor and labels (:func:`ce_reference`).
+* "Liger-Kernel: Triton kernels that replace HF training ops", section
+  "Installation and the one-line patch": the fused-linear post-training losses
+  (ORPO, DPO, ...) take the LM-head weight, the hidden states and the targets
+  and return the loss; :func:`pairwise_logistic` is the DPO-form loss on the
+  per-sequence log-probabilities that the head's row losses give.
 
 The oracle therefore *does* materialise the logits (that is the plain
 definition) and follows these steps, with ``n`` the number of non-ignored rows:
@@ -311,3 +316,40 @@ def merge_shard_stats(all_lse, all_zy):
     the target).  Returns ``(lse, zy)``."""
     L = _f64(all_lse)
     return log_sum_exp(L.T), _f64(all_zy).sum(axis=0)
+
+
+# ---------------------------------------------------------------------------
+# Pairwise logistic (DPO-form) preference loss on the head's row losses.
+# ---------------------------------------------------------------------------
+
+def pairwise_logistic(row_loss, y, seq_start, chosen, rejected, beta: float, ref_logp=None,
+                      ignore_index: int = IGNORE_INDEX):
+    """Sequence s holds the token rows ``seq_start[s] .. seq_start[s+1]-1``;
+    ``logp_s = -(sum of their row losses)`` (a row loss is -log p(y_i | x_i),
+    0 on ignored rows).  Pair k compares sequences ``chosen[k]`` and
+    ``rejected[k]``: ``m_k = beta ((logp_c - ref_c) - (logp_r - ref_r))`` and
+    ``L = -(1/P) sum_k log sigmoid(m_k)``.  Returns
+    ``(L, logp, dL/dlogp, row weights)`` where the weight of a valid row i of
+    sequence s is ``-dL/dlogp_s`` (the upstream gradient of its row loss) and
+    every other row's is 0."""
+    rl = _f64(row_loss)
+    y = _i64(y)
+    st = _i64(seq_start)
+    c = _i64(chosen)
+    r = _i64(rejected)
+    S = len(st) - 1
+    logp = np.array([-rl[st[s]:st[s + 1]].sum() for s in range(S)])
+    d = logp if ref_logp is None else logp - _f64(ref_logp)
+    m = beta * (d[c] - d[r])
+    P = len(c)
+    loss = float(np.logaddexp(0.0, -m).sum() / P)       # -log sigmoid(m) = log(1 + e^-m)
+    gm = -1.0 / (1.0 + np.exp(m)) / P                   # dL/dm_k = -sigmoid(-m_k) / P
+    grad = np.zeros(S)
+    for k in range(P):
+        grad[c[k]] += beta * gm[k]
+        grad[r[k]] -= beta * gm[k]
+    w = np.zeros(len(rl))
+    for s in range(S):
+        w[st[s]:st[s + 1]] = -grad[s]
+    w[y == ignore_index] = 0.0
+    return loss, logp, grad, w

@@ -383,10 +383,50 @@ def pin_vocab_shards(orc):
     _close(np.where(valid, lse - zy, 0.0), per, 1e-12, what="row losses from merged statistics")
 
 
+def pin_pairwise_logistic(orc):
+    """The DPO-form pair loss: torch's logsigmoid + autograd on the same
+    sequence log-probabilities (a pair sharing a sequence with another pair
+    included); one pair in closed form, log(1 + exp(-beta d)); swapping chosen
+    and rejected turns softplus(-m) into softplus(m), whose difference is m."""
+    r = _rng(120)
+    lens = [5, 3, 7, 1, 4, 6]
+    st = np.concatenate([[0], np.cumsum(lens)])
+    N = int(st[-1])
+    rl = np.abs(r.standard_normal(N)) * 3.0
+    y = r.integers(0, 50, size=N)
+    y[[0, 6, 9]] = IGN
+    rl[y == IGN] = 0.0
+    ch = np.array([0, 2, 4, 2])
+    rj = np.array([1, 3, 5, 0])
+    ref = r.standard_normal(6)
+    beta = 0.7
+    loss, logp, grad, w = orc.pairwise_logistic(rl, y, st, ch, rj, beta, ref)
+    tl = torch.tensor(rl, requires_grad=True)
+    tlogp = torch.stack([-tl[st[s]:st[s + 1]].sum() for s in range(6)])
+    d = tlogp - torch.tensor(ref)
+    tloss = -torch.nn.functional.logsigmoid(beta * (d[ch] - d[rj])).mean()
+    tloss.backward()
+    assert abs(loss - tloss.item()) <= 1e-13 * abs(tloss.item())
+    _close(logp, tlogp.detach().numpy(), 1e-14, what="sequence log-probs")
+    # the row weight is the upstream gradient of the row loss (valid rows only)
+    want_w = np.where(y != IGN, tl.grad.numpy(), 0.0)
+    _close(w, want_w, 1e-12, atol=1e-17, what="row weights vs autograd")
+    rows_of = np.repeat(np.arange(6), lens)
+    _close(-grad[rows_of][y != IGN], tl.grad.numpy()[y != IGN], 1e-12, what="dL/dlogp")
+    # one pair: closed form
+    one = np.array([0]), np.array([1])
+    l1, lp1, g1, _ = orc.pairwise_logistic(rl, y, st, one[0], one[1], beta)
+    dd = lp1[0] - lp1[1]
+    assert abs(l1 - math.log1p(math.exp(-beta * dd))) <= 1e-13 * max(1.0, l1)
+    assert abs(g1[0] + beta / (1.0 + math.exp(beta * dd))) <= 1e-13
+    l2, _, _, _ = orc.pairwise_logistic(rl, y, st, one[1], one[0], beta)
+    assert abs((l1 - l2) - (-beta * dd)) <= 1e-12 * max(1.0, abs(beta * dd))
+
+
 ALL_PINS = [
     pin_zero_weight, pin_zero_input, pin_two_class, pin_large_logits,
     pin_torch_autograd, pin_finite_difference, pin_rows_of_g_sum_to_zero,
     pin_shift_invariance, pin_ignored_rows, pin_no_valid_rows, pin_target_range,
     pin_permutations, pin_equal_logits, pin_row_functions, pin_full_grads, pin_torch_inputs, pin_reductions,
-    pin_ce_on_logits, pin_vocab_shards,
+    pin_ce_on_logits, pin_vocab_shards, pin_pairwise_logistic,
 ]

@@ -59,6 +59,12 @@ MUTATIONS = [
     ("blocked one-hot added", "Z[rows, yb] -= 1.0", "Z[rows, yb] += 1.0"),
     ("blocked loss over all rows' count", "    loss = float(loss_sum / n) if n else 0.0",
      "    loss = float(loss_sum / N) if n else 0.0"),
+    ("pair loss: sign of the margin", "    loss = float(np.logaddexp(0.0, -m).sum() / P)",
+     "    loss = float(np.logaddexp(0.0, m).sum() / P)"),
+    ("pair loss: rejected gradient added", "        grad[r[k]] -= beta * gm[k]", "        grad[r[k]] += beta * gm[k]"),
+    ("pair loss: ignored rows weighted", "    w[y == ignore_index] = 0.0\n", "    pass\n"),
+    ("pair loss: reference log-probs added", "d = logp if ref_logp is None else logp - _f64(ref_logp)",
+     "d = logp if ref_logp is None else logp + _f64(ref_logp)"),
     ("bf16 tensors converted through fp16", "            a = a.float()", "            a = a.half().float()"),
 ]
 

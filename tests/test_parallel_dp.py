@@ -42,6 +42,11 @@ def _oracle_call(X, W, y, ignore_index, mean_count):
             torch.tensor(dW))
 
 
+def _oracle_count(y, ignore_index):
+    from oracle import flce_oracle as O
+    return torch.tensor([int(O.valid_mask(y.numpy(), 1 << 30, ignore_index).sum())], dtype=torch.int32)
+
+
 def _rank(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
@@ -51,7 +56,7 @@ def _rank(rank, world, port, q):
     X, W, y = _batch()
     shard = slice(rank * 20, (rank + 1) * 20)
     loss, dX, dW = dp_forward_backward(torch.tensor(X[shard]), torch.tensor(W), torch.tensor(y[shard]),
-                                       local_call=_oracle_call)
+                                       local_call=_oracle_call, count_call=_oracle_count)
     q.put((rank, float(loss.item()), dX.numpy(), dW.numpy()))
     dist.destroy_process_group()
 
