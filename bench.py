@@ -51,11 +51,18 @@ def parse():
     ap.add_argument("--sustain-s", type=float, default=3.0,
                     help="after the timed region, run the step for at least this many seconds more and report "
                          "that run under 'sustained' (0: skip)")
-    ap.add_argument("--op", choices=["flce", "ce", "unfused", "vp", "pref"], default="flce",
+    ap.add_argument("--op", choices=["flce", "ce", "unfused", "vp", "pref", "dp-nccl", "vp-nccl"], default="flce",
                     help="flce: the fused head (default); ce: cross-entropy on given logits of the same workload; "
                          "unfused: PyTorch eager linear + cross_entropy + autograd, a context row (not this library); "
                          "vp: the vocabulary-parallel head's shards run one after another on this GPU; "
-                         "pref: the pairwise logistic preference loss on the head")
+                         "pref: the pairwise logistic preference loss on the head; "
+                         "dp-nccl: the data-parallel head over the ranks (each rank its own tokens, W replicated, "
+                         "count / dW / loss all-reduces over NCCL inside the step); "
+                         "vp-nccl: the vocabulary-parallel head over the ranks (W rows sharded, statistics "
+                         "all-gather and dX all-reduce over NCCL inside the step)")
+    ap.add_argument("--sections", type=int, default=4,
+                    help="dp-nccl: gradient-pass sections whose dW rows are all-reduced while later sections "
+                         "compute (0: one all-reduce after the call)")
     ap.add_argument("--shards", type=int, default=8, help="vocabulary shards of --op vp")
     return ap.parse_args()
 
@@ -239,6 +246,21 @@ def max_over_ranks(x: float, world: int) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def nccl_group(world):
+    """The process group of the multi-device ops: the torchrun group, or one of
+    a single rank (NCCL on this GPU) when the bench runs alone."""
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        import datetime
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120))
+    return dist
 
 
 def dist_teardown(world):
@@ -633,6 +655,103 @@ def run_vp(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_dp_nccl(args, world, rank, local):
+    """The data-parallel head as a program: every rank holds its own tokens
+    (the workload's N rows, drawn with the rank in the seed) and the whole W;
+    a step counts the valid targets and all-reduces the count, runs the head
+    with the mean over that count, and all-reduces dW (section by section on a
+    second stream while later sections compute, --sections > 0) and the loss,
+    all over NCCL inside the timed region.  Weak scaling: value = all ranks'
+    tokens over the slowest rank's time."""
+    import dataclasses
+
+    import lm_head_linear_03_b200 as F
+    from lm_head_linear_03_b200.inputs import make_inputs
+    from lm_head_linear_03_b200.parallel import dp_forward_backward, dp_forward_backward_overlapped
+    F.load_library()
+    dist = nccl_group(world)
+    w = workload(args)
+    dev = torch.device("cuda", local)
+    X, _, y = make_inputs(dataclasses.replace(w, seed=w.seed + 1000 * rank), dev)
+    _, W, _ = make_inputs(w, dev)
+    N, H, V = w.N, w.H, w.V
+    ws = F.alloc_workspace(N, H, V, dev)
+    comm = torch.cuda.Stream(device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if args.sections > 0:
+            dp_forward_backward_overlapped(X, W, y, sections=args.sections, workspace=ws, comm_stream=comm)
+        else:
+            dp_forward_backward(X, W, y)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    ms, clocks = timed_region(dev, stream, world, args.steps, step)
+    ms /= args.steps
+    if rank != 0:
+        return
+    line = {
+        "metric": "data-parallel fused linear-CE fwd+bwd tokens/s over NCCL (collectives inside the step)",
+        "value": world * N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "N_per_rank": N, "H": H, "V": V, "parallelism": f"dp{world}",
+                   "dW_allreduce": f"{args.sections} sections overlapped" if args.sections > 0 else "after the call"},
+        "gpu_launches": (8 if args.sections > 0 else 7) * args.steps,
+        "clocks": clocks,
+        "note": "this library's launches per step: the count, then prep, row order, pass 1, combine, pass 2 (one "
+                "launch per section), dX scatter; NCCL's kernels not counted",
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_vp_nccl(args, world, rank, local):
+    """The vocabulary-parallel head as a program: rank r holds W rows
+    vocab_shard_range(V, world, r) and the same X and y; a step runs the
+    shard's statistics, all-gathers them, runs the shard's backward and
+    all-reduces dX, all over NCCL inside the timed region.  Strong scaling:
+    the N tokens of one step are shared by all ranks."""
+    import lm_head_linear_03_b200 as F
+    from lm_head_linear_03_b200.inputs import make_inputs
+    from lm_head_linear_03_b200.parallel import vocab_shard_range, vp_forward_backward
+    F.load_library()
+    nccl_group(world)
+    w = workload(args)
+    dev = torch.device("cuda", local)
+    X, W, y = make_inputs(w, dev)
+    N, H, V = w.N, w.H, w.V
+    v0, v1 = vocab_shard_range(V, world, rank)
+    Ws = W[v0:v1].contiguous()
+    del W
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vp_forward_backward(X, Ws, y, v0, V)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    ms, clocks = timed_region(dev, stream, world, args.steps, step)
+    ms /= args.steps
+    if rank != 0:
+        return
+    line = {
+        "metric": "vocabulary-parallel fused linear-CE fwd+bwd tokens/s over NCCL (collectives inside the step)",
+        "value": N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "H": H, "V": V, "parallelism": f"vp{world}",
+                   "shard_rows": v1 - v0},
+        "gpu_launches": 9 * args.steps,
+        "clocks": clocks,
+        "note": "this library's launches per step: statistics (prep, row order, pass 1, combine) and backward "
+                "(prep, row order, combine, pass 2, scatter); NCCL's kernels not counted",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_pref(args, world, rank, local):
     """The pairwise logistic (DPO-form) preference loss on the head, measured:
     the workload's token rows packed as sequences of 1024 rows whose first
@@ -768,10 +887,17 @@ def main():
             run_vp(args, world, rank, local)
         elif args.op == "pref":
             run_pref(args, world, rank, local)
+        elif args.op == "dp-nccl":
+            run_dp_nccl(args, world, rank, local)
+        elif args.op == "vp-nccl":
+            run_vp_nccl(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
         dist_teardown(world)
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():  # the single-rank group of the multi-device ops
+            dist.destroy_process_group()
 
 
 if __name__ == "__main__":

@@ -82,6 +82,12 @@ typedef enum {
 /* Human-readable name of a status code (static storage). */
 const char* flce_status_string(int status);
 
+/* Where the last FLCE_ERR_CUDA returned on this host thread came from: the
+ * library's source line of the failing step, the CUDA runtime's error code
+ * and its text (static storage).  Any argument may be NULL.  Zero / "no error"
+ * when no call on this thread has failed. */
+void flce_last_cuda_error(int32_t* line, int32_t* cuda_error, const char** text);
+
 /* Bytes of device workspace one call needs.  The logits are processed one
  * vocabulary chunk of fixed width at a time, so the size depends on N and H
  * only: V is accepted for the caller's convenience and does not change the

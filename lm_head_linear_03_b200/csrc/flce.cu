@@ -7,7 +7,6 @@
 #include <algorithm>
 #include <climits>
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -26,6 +25,17 @@ constexpr int MAX_SPLITS = 64;
 constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per bounded wait
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// The last CUDA failure this library reported (FLCE_ERR_CUDA), per host thread:
+// the source line of the failing step and the CUDA runtime's error.
+thread_local int g_fail_line = 0;
+thread_local cudaError_t g_fail_code = cudaSuccess;
+
+flce_status_t cuda_fail(int line) {
+  g_fail_line = line;
+  g_fail_code = cudaPeekAtLastError();
+  return FLCE_ERR_CUDA;
+}
 
 struct WsLayout {
   size_t ctrl, counters, counters_bytes, tile_cnt, tile_valid, perm, y_perm, g_perm, lse2, zy, part_m, part_l,
@@ -57,9 +67,9 @@ WsLayout ws_layout(int64_t N, int64_t H, bool packed = false) {
   const size_t n = static_cast<size_t>(N);
   const size_t nblk = (n + COMBINE_THREADS - 1) / COMBINE_THREADS;
   L.ctrl = take(256);
-  // pass-2 completion counters: g_row[TM], x_row[TM], g_col[VC/BN], w_col[VC/SUBN]
+  // pass-2 completion counters: g_row[TM], x_row[TM], g_col[VC/BN], w_col[VC/BN]
   const size_t tm = (n + CM - 1) / CM;
-  L.counters_bytes = (2 * tm + 2 * (VC / SUBN)) * 4;
+  L.counters_bytes = (2 * tm + 2 * (VC / BN)) * 4;
   L.counters = take(L.counters_bytes);
   L.tile_cnt = take(tm * 4);
   L.tile_valid = take(tm * 4);
@@ -199,16 +209,6 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
                                                 : CU_TENSOR_MAP_SWIZZLE_NONE,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
-}
-
-// K-blocks of the stagger at each end of a tile (1 .. MAX_LAG).
-int stagger_lag() {
-  static const int lag = [] {
-    const char* e = getenv("FLCE_LAG");
-    const int v = e ? atoi(e) : 2;
-    return std::max(1, std::min(MAX_LAG, v));
-  }();
-  return lag;
 }
 
 // ------------------------------------------------------------------ plan --
@@ -382,12 +382,12 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
                       void* workspace, size_t ws_bytes, cudaStream_t stream, const Options& opt = Options()) {
   DevInfo di;
   int dev;
-  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (device_info(&di, &dev) != cudaSuccess) return cuda_fail(__LINE__);
   if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
-  if (set_kernel_attrs(dev) != cudaSuccess) return FLCE_ERR_CUDA;
-  if (!get_encode()) return FLCE_ERR_CUDA;
+  if (set_kernel_attrs(dev) != cudaSuccess) return cuda_fail(__LINE__);
+  if (!get_encode()) return cuda_fail(__LINE__);
 
-  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;  // now with max_clusters
+  if (device_info(&di, &dev) != cudaSuccess) return cuda_fail(__LINE__);  // now with max_clusters
   // reordered rows need the packed-X area: only a large enough workspace has it
   // (vocabulary shards keep the caller's order: their statistics are per row)
   const WsLayout L = ws_layout(N, H, opt.combine == COMBINE_FULL && ws_bytes >= ws_layout(N, H, true).total);
@@ -408,25 +408,25 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
 
   CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn, mHi, mLo, mXc_k, mXc_mn;
   const uint64_t n = static_cast<uint64_t>(N), h = static_cast<uint64_t>(H), v = static_cast<uint64_t>(V);
-  bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, SUBNH) &&
+  bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BNH) &&
             make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
             make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK) &&
             // the packed copy of X (the caller's X stands in when there is none: never read then)
             make_map(&mXc_k, Xc ? Xc : X, h, n, h * 2, BK, BM) && make_map(&mXc_mn, Xc ? Xc : X, h, n, h * 2, 64, BK) &&
-            (dX == nullptr || (make_map(&mHi, dX, h, n, h * 2, SUBN, BM, Swz::none) &&
-                               make_map(&mLo, lo, h, n, h * 2, SUBN, BM, Swz::none)));
+            (dX == nullptr || (make_map(&mHi, dX, h, n, h * 2, BN, BM, Swz::none) &&
+                               make_map(&mLo, lo, h, n, h * 2, BN, BM, Swz::none)));
   // 32 x 32 output boxes of the epilogues (64-byte swizzle)
   CUtensorMap mGo, mDWo, mHio, mLoo;
   ok = ok && (dX == nullptr || (make_map(&mGo, G, VC, n, VC * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
                                 make_map(&mDWo, dW, h, v, h * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
                                 make_map(&mHio, dX, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
                                 make_map(&mLoo, lo, h, n, h * 2, EPI_BOX, EPI_BOX, Swz::k64)));
-  if (!ok) return FLCE_ERR_CUDA;
+  if (!ok) return cuda_fail(__LINE__);
 
   // control words and pass-2 counters start at zero (they are contiguous)
-  if (cudaMemsetAsync(ctrl, 0, L.counters + L.counters_bytes - L.ctrl, stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaMemsetAsync(ctrl, 0, L.counters + L.counters_bytes - L.ctrl, stream) != cudaSuccess) return cuda_fail(__LINE__);
   if (d_status != &ctrl->status && cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess)
-    return FLCE_ERR_CUDA;
+    return cuda_fail(__LINE__);
 
   GemmArgs a{};
   a.N = static_cast<int>(N);
@@ -452,7 +452,6 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   a.tile_valid = reinterpret_cast<const int*>(ws + L.tile_valid);
   a.perm = perm;
   a.reordered = &ctrl->reordered;
-  a.lag = stagger_lag();
 
   // Valid rows per 256-row token tile, then the token-row order of both passes.
   {
@@ -461,7 +460,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     flce_prep_kernel<<<P.tiles_m, CM, 0, stream>>>(y, static_cast<int>(N), ignore_index,
                                                    reinterpret_cast<int*>(ws + L.tile_cnt));
     prof_end(stream, slot);
-    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
     prof_begin(stream, KIND_ORDER, &slot);
     flce_row_order_kernel<<<P.tiles_m, CM, 0, stream>>>(
         y, opt.grad_row_scale, static_cast<int>(N), P.tiles_m, ignore_index,
@@ -469,14 +468,14 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
         static_cast<int>(V), static_cast<int>(opt.V_total ? opt.V_total : V),
         reinterpret_cast<int*>(ws + L.tile_valid), perm, y_perm, g_perm, &ctrl->reordered, &ctrl->n_rows, d_status);
     prof_end(stream, slot);
-    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
     if (L.packed) {  // X rows in the new order (returns at once when the order was kept)
       const int pgrid = static_cast<int>(std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(di.num_sms) * 8));
       prof_begin(stream, KIND_PACK, &slot);
       flce_pack_rows_kernel<<<pgrid, 256, 0, stream>>>(X, Xc, perm, &ctrl->reordered, &ctrl->n_rows,
                                                         static_cast<int>(N), static_cast<int>(H));
       prof_end(stream, slot);
-      if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+      if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
     }
   }
 
@@ -494,7 +493,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     prof_begin(stream, KIND_LSE, &slot);
     flce_pass1_kernel<<<CLUSTER * P.lse_clusters, NUM_THREADS, P1_SMEM_BYTES, stream>>>(mX_k, mXc_k, mW_k, p1);
     prof_end(stream, slot);
-    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
   } else if (opt.combine != COMBINE_SHARDS_IN) {
     // one launch per W piece, after its copy; its splits fill the next partial slots
     const PipeCtx& pp = *opt.pipe;
@@ -502,7 +501,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     for (int i = 0; i < pp.pieces; ++i) {
       const int64_t v0 = pp.piece_v[i], vp = pp.piece_v[i + 1] - pp.piece_v[i];
       CUtensorMap mWp;
-      if (!make_map(&mWp, W + v0 * H, h, static_cast<uint64_t>(vp), h * 2, BK, SUBNH)) return FLCE_ERR_CUDA;
+      if (!make_map(&mWp, W + v0 * H, h, static_cast<uint64_t>(vp), h * 2, BK, BNH)) return cuda_fail(__LINE__);
       GemmArgs p1 = a;
       p1.V = static_cast<int>(vp);
       p1.v_off = static_cast<int>(v0);
@@ -514,12 +513,12 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       p1.num_units = P.tiles_m * p1.splits;
       total_splits += p1.splits;
       const int grid = static_cast<int>(std::min<long long>(p1.num_units, P.clusters));
-      if (cudaStreamWaitEvent(stream, pp.w_ready[i], 0) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (cudaStreamWaitEvent(stream, pp.w_ready[i], 0) != cudaSuccess) return cuda_fail(__LINE__);
       size_t slot;
       prof_begin(stream, KIND_LSE, &slot);
       flce_pass1_kernel<<<CLUSTER * grid, NUM_THREADS, P1_SMEM_BYTES, stream>>>(mX_k, mXc_k, mWp, p1);
       prof_end(stream, slot);
-      if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+      if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
     }
   }
   // Combine the splits: lse, loss, n_valid, 1/n.
@@ -557,7 +556,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     prof_begin(stream, KIND_COMBINE, &slot);
     flce_combine_kernel<<<grid, COMBINE_THREADS, 0, stream>>>(c);
     prof_end(stream, slot);
-    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
   }
   // Pass 2: every chunk's logit recompute, dW and dX tiles in one persistent launch
   // (skipped for a forward-only call and for a shard's statistics).
@@ -566,23 +565,16 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     b.TM = P.tiles_m;
     b.HN = static_cast<int>((H + BN - 1) / BN);
     b.C = P.num_chunks;
-    const int64_t v_last = V - static_cast<int64_t>(P.num_chunks - 1) * VC;  // vocabulary of the last chunk
     b.VTf = VC / BN;
-    b.VT_last = static_cast<int>((v_last + BN - 1) / BN);
-    b.VMf = VC / SUBN;
-    b.VM_last = static_cast<int>((v_last + SUBN - 1) / SUBN);
-    if (b.C == 1) {
-      b.VTf = b.VT_last;
-      b.VMf = b.VM_last;
-    }
-    auto vt_of = [&](int c) { return static_cast<long long>(c == b.C - 1 ? b.VT_last : b.VTf); };
-    auto vm_of = [&](int c) { return static_cast<long long>(c == b.C - 1 ? b.VM_last : b.VMf); };
+    b.VT_last = static_cast<int>((V - static_cast<int64_t>(P.num_chunks - 1) * VC + BN - 1) / BN);
+    if (b.C == 1) b.VTf = b.VT_last;
     // section_end[c]: end of the queue's section c (dX(c) dW(c) G(c+1)), after G(0)
     std::vector<long long> section_end(b.C);
-    long long total = vt_of(0) * b.TM;  // G(0)
+    long long total = static_cast<long long>(b.C == 1 ? b.VT_last : b.VTf) * b.TM;  // G(0)
     for (int c = 0; c < b.C; ++c) {
-      total += static_cast<long long>(b.TM) * b.HN + vm_of(c) * b.HN;
-      if (c + 1 < b.C) total += vt_of(c + 1) * b.TM;
+      const long long vt = c == b.C - 1 ? b.VT_last : b.VTf;
+      total += static_cast<long long>(b.TM) * b.HN + vt * b.HN;
+      if (c + 1 < b.C) total += static_cast<long long>(c + 1 == b.C - 1 ? b.VT_last : b.VTf) * b.TM;
       section_end[c] = total;
     }
     b.total_items = total;
@@ -593,7 +585,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     b.g_row = ctr;
     b.x_row = ctr + b.TM;
     b.g_col = ctr + 2 * b.TM;
-    b.w_col = ctr + 2 * b.TM + VC / BN;  // VC / SUBN entries
+    b.w_col = ctr + 2 * b.TM + VC / BN;
     Pass2Maps pm;
     pm.Xk = mX_k;
     pm.Wk = mW_k;
@@ -622,7 +614,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
       prof_begin(stream, KIND_PASS2, &slot);
       flce_pass2_kernel<<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, stream>>>(pm, b);
       prof_end(stream, slot);
-      if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+      if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
       if (opt.pipe) {  // dW rows of chunks c0 .. c1-1 are final
         const PipeCtx& pp = *opt.pipe;
         const int64_t r0 = static_cast<int64_t>(c0) * VC, r1 = std::min<int64_t>(V, static_cast<int64_t>(c1) * VC);
@@ -630,11 +622,11 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
           pp.section_rows[k] = r0;
           pp.section_rows[k + 1] = r1;
         }
-        if (cudaEventRecord(pp.p2_done[k], stream) != cudaSuccess) return FLCE_ERR_CUDA;
+        if (cudaEventRecord(pp.p2_done[k], stream) != cudaSuccess) return cuda_fail(__LINE__);
         if (pp.h_dW && (cudaStreamWaitEvent(pp.copy, pp.p2_done[k], 0) != cudaSuccess ||
                         cudaMemcpyAsync(pp.h_dW + r0 * H, dW + r0 * H, static_cast<size_t>(r1 - r0) * H * 2,
                                         cudaMemcpyDeviceToHost, pp.copy) != cudaSuccess))
-          return FLCE_ERR_CUDA;
+          return cuda_fail(__LINE__);
       }
     }
     // reordered rows: the final dX rows go back in place (no-op otherwise)
@@ -643,7 +635,7 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     flce_dx_scatter_kernel<<<sgrid, 256, 0, stream>>>(lo, dX, perm, &ctrl->reordered, &ctrl->n_rows,
                                                       static_cast<int>(N), static_cast<int>(H));
     prof_end(stream, slot);
-    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
   }
   return FLCE_OK;
 }
@@ -661,8 +653,8 @@ flce_status_t sync_call(const uint16_t* X, const uint16_t* W, const int32_t* y, 
   if (s != FLCE_OK) return s;
   Ctrl host{};
   if (cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-    return FLCE_ERR_CUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
+    return cuda_fail(__LINE__);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return cuda_fail(__LINE__);
   *loss = host.loss;
   return static_cast<flce_status_t>(host.status);
 }
@@ -671,6 +663,12 @@ flce_status_t sync_call(const uint16_t* X, const uint16_t* W, const int32_t* y, 
 
 // ================================================================== C ABI ==
 extern "C" {
+
+void flce_last_cuda_error(int32_t* line, int32_t* cuda_error, const char** text) {
+  if (line) *line = g_fail_line;
+  if (cuda_error) *cuda_error = static_cast<int32_t>(g_fail_code);
+  if (text) *text = cudaGetErrorString(g_fail_code);
+}
 
 const char* flce_status_string(int s) {
   switch (s) {
@@ -757,13 +755,13 @@ flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64
   if (workspace_bytes < L.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   DevInfo di;
   int dev;
-  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (device_info(&di, &dev) != cudaSuccess) return cuda_fail(__LINE__);
   if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int TM = static_cast<int>((N + CM - 1) / CM);
   if (cudaMemsetAsync(ws + L.ctrl, 0, 256, stream) != cudaSuccess ||
       cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess)
-    return FLCE_ERR_CUDA;
+    return cuda_fail(__LINE__);
   CeArgs c{};
   c.logits = logits;
   c.dlogits = dlogits;
@@ -787,16 +785,16 @@ flce_status_t flce_cross_entropy(const uint16_t* logits, const int32_t* y, int64
   flce_prep_kernel<<<TM, CM, 0, stream>>>(y, c.N, ignore_index, reinterpret_cast<int*>(ws + L.tile_valid),
                                           reinterpret_cast<int*>(ws + L.ctrl + 8));
   prof_end(stream, slot);
-  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
   const int grid = static_cast<int>(std::min<int64_t>(N, static_cast<int64_t>(di.num_sms) * 4 * 64));
   prof_begin(stream, KIND_CE, &slot);
   flce_ce_rows_kernel<<<grid, CE_THREADS, 0, stream>>>(c);
   prof_end(stream, slot);
-  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
   prof_begin(stream, KIND_COMBINE, &slot);
   flce_ce_reduce_kernel<<<static_cast<int>((N + COMBINE_THREADS - 1) / COMBINE_THREADS), COMBINE_THREADS, 0, stream>>>(c);
   prof_end(stream, slot);
-  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
   return FLCE_OK;
 }
 
@@ -806,15 +804,15 @@ flce_status_t flce_count_valid(const int32_t* y, int64_t N, int32_t ignore_index
   if (!aligned(y, 4) || !aligned(d_count, 4)) return FLCE_ERR_UNSUPPORTED;
   DevInfo di;
   int dev;
-  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (device_info(&di, &dev) != cudaSuccess) return cuda_fail(__LINE__);
   if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
-  if (cudaMemsetAsync(d_count, 0, sizeof(int32_t), stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaMemsetAsync(d_count, 0, sizeof(int32_t), stream) != cudaSuccess) return cuda_fail(__LINE__);
   const int tiles = static_cast<int>((N + CM - 1) / CM);
   size_t slot;
   prof_begin(stream, KIND_PREP, &slot);
   flce_prep_kernel<<<tiles, CM, 0, stream>>>(y, static_cast<int>(N), ignore_index, nullptr, d_count);
   prof_end(stream, slot);
-  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : cuda_fail(__LINE__);
 }
 
 flce_status_t flce_pairwise_logistic(const float* d_row_loss, const int32_t* y, int64_t N, int32_t ignore_index,
@@ -833,11 +831,11 @@ flce_status_t flce_pairwise_logistic(const float* d_row_loss, const int32_t* y, 
     return FLCE_ERR_UNSUPPORTED;
   DevInfo di;
   int dev;
-  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (device_info(&di, &dev) != cudaSuccess) return cuda_fail(__LINE__);
   if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
   if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream) != cudaSuccess ||
       cudaMemsetAsync(d_row_weight, 0, static_cast<size_t>(N) * sizeof(float), stream) != cudaSuccess)
-    return FLCE_ERR_CUDA;
+    return cuda_fail(__LINE__);
   PrefArgs a{};
   a.row_loss = d_row_loss;
   a.y = y;
@@ -856,11 +854,11 @@ flce_status_t flce_pairwise_logistic(const float* d_row_loss, const int32_t* y, 
   a.row_weight = d_row_weight;
   a.status = d_status;
   flce_pref_logp_kernel<<<S, PREF_THREADS, 0, stream>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
   flce_pref_pairs_kernel<<<1, PREF_THREADS, 0, stream>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
   flce_pref_weights_kernel<<<S, PREF_THREADS, 0, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : cuda_fail(__LINE__);
 }
 
 namespace {
@@ -921,12 +919,12 @@ flce_status_t flce_probe_bounded_wait(int64_t timeout_ns, int32_t* d_status, cud
   if (!aligned(d_status, 4)) return FLCE_ERR_UNSUPPORTED;
   DevInfo di;
   int dev;
-  if (device_info(&di, &dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (device_info(&di, &dev) != cudaSuccess) return cuda_fail(__LINE__);
   if (!di.sm100) return FLCE_ERR_UNSUPPORTED;
   // d_status[0], d_status[1]: the two waits' results; d_status[2]: the counter nobody sets
-  if (cudaMemsetAsync(d_status, 0, 3 * sizeof(int32_t), stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaMemsetAsync(d_status, 0, 3 * sizeof(int32_t), stream) != cudaSuccess) return cuda_fail(__LINE__);
   flce_wait_probe_kernel<<<1, 32, 0, stream>>>(d_status, d_status + 2, static_cast<unsigned long long>(timeout_ns));
-  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : cuda_fail(__LINE__);
 }
 
 flce_status_t flce_probe_pass2_timeout(const uint16_t* X, const uint16_t* W, const int32_t* y, int64_t N, int64_t H,
@@ -954,13 +952,13 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
   if (s != FLCE_OK) return s;
   if (workspace_bytes < ws_layout(N, H).total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   PipeRes* pr = nullptr;
-  if (pipe_resources(&pr) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (pipe_resources(&pr) != cudaSuccess) return cuda_fail(__LINE__);
   std::lock_guard<std::mutex> lk(pr->mu);  // one host-buffer call per device at a time: shared copy stream
   const size_t xb = static_cast<size_t>(N) * H * 2, yb = N * 4;
   // X and y first, on the caller's stream: every kernel needs them
   if (cudaMemcpyAsync(d_X, h_X, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
       cudaMemcpyAsync(d_y, h_y, yb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
-    return FLCE_ERR_CUDA;
+    return cuda_fail(__LINE__);
   // W in pieces on the copy stream, which starts after the caller's earlier work
   PipeCtx pp;
   pp.copy = pr->copy;
@@ -970,7 +968,7 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
   pp.groups = MAX_PIECES;
   pp.h_dW = h_dW;
   if (cudaEventRecord(pr->start, stream) != cudaSuccess || cudaStreamWaitEvent(pr->copy, pr->start, 0) != cudaSuccess)
-    return FLCE_ERR_CUDA;
+    return cuda_fail(__LINE__);
   for (int i = 0; i < pp.pieces; ++i) {
     const int64_t v0 = pp.piece_v[i], v1 = pp.piece_v[i + 1];
     pp.w_ready[i] = pr->ev[i];
@@ -978,7 +976,7 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
     if (cudaMemcpyAsync(d_W + v0 * H, h_W + v0 * H, static_cast<size_t>(v1 - v0) * H * 2, cudaMemcpyHostToDevice,
                         pr->copy) != cudaSuccess ||
         cudaEventRecord(pp.w_ready[i], pr->copy) != cudaSuccess)
-      return FLCE_ERR_CUDA;
+      return cuda_fail(__LINE__);
   }
   for (int i = pp.pieces; i < MAX_PIECES; ++i) pp.p2_done[i] = pr->ev[MAX_PIECES + i];
   Options opt;
@@ -995,8 +993,8 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
   if (cudaMemcpyAsync(h_dX, d_dX, xb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
       cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
       cudaEventRecord(pr->done, pr->copy) != cudaSuccess || cudaStreamWaitEvent(stream, pr->done, 0) != cudaSuccess)
-    return FLCE_ERR_CUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
+    return cuda_fail(__LINE__);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return cuda_fail(__LINE__);
   *h_loss = host.loss;
   return static_cast<flce_status_t>(host.status);
 }
@@ -1030,7 +1028,7 @@ flce_status_t flce_forward_backward_sections(const uint16_t* X, const uint16_t* 
   // sections beyond the chunks hold no rows and are done with the last one
   for (int k = used; k < sections; ++k) {
     section_rows[k + 1] = V;
-    if (cudaEventRecord(section_done[k], stream) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cudaEventRecord(section_done[k], stream) != cudaSuccess) return cuda_fail(__LINE__);
   }
   return FLCE_OK;
 }
@@ -1079,7 +1077,7 @@ flce_status_t flce_profile_enable(int on) {
     g_prof.ev.resize(2 * PROF_PAIRS);
     g_prof.kind.resize(PROF_PAIRS);
     for (auto& e : g_prof.ev)
-      if (cudaEventCreate(&e) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (cudaEventCreate(&e) != cudaSuccess) return cuda_fail(__LINE__);
   }
   g_prof.on = on != 0;
   g_prof.used = 0;
@@ -1092,7 +1090,7 @@ flce_status_t flce_row_order_info(const void* workspace, int32_t* reordered, int
   Ctrl host{};
   if (cudaMemcpyAsync(&host, workspace, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
       cudaStreamSynchronize(stream) != cudaSuccess)
-    return FLCE_ERR_CUDA;
+    return cuda_fail(__LINE__);
   *reordered = host.reordered;
   *n_valid = host.n_rows;
   return FLCE_OK;
@@ -1105,9 +1103,9 @@ flce_status_t flce_profile_read(int32_t* launches, double* total_ms) {
     total_ms[k] = 0.0;
   }
   for (size_t i = 0; i < g_prof.used; ++i) {
-    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return cuda_fail(__LINE__);
     float ms = 0.f;
-    if (cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) return cuda_fail(__LINE__);
     launches[g_prof.kind[i]] += 1;
     total_ms[g_prof.kind[i]] += ms;
   }
@@ -1154,6 +1152,6 @@ extern "C" flce_status_t flce_forward_backward_noalloc(const uint16_t* X, const 
   if (s != FLCE_OK) return s;
   if (ws_layout(N, H).total > static_cast<size_t>(FLCE_NOALLOC_SCRATCH_BYTES)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
-  if (noalloc_scratch(&scratch) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return cuda_fail(__LINE__);
   return sync_call(X, W, y, N, H, V, ignore_index, loss, dX, dW, scratch, FLCE_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -1,11 +1,11 @@
 // Device code of the fused linear + cross-entropy head.
 //
-// One persistent, warp-specialised tcgen05 GEMM structure serves all four
+// One persistent, warp-specialised tcgen05 GEMM template serves all four
 // tensor-core steps; they differ in which operands the TMA engine streams in,
 // in which of them are MN-major, and in the epilogue that turns the fp32
 // accumulator tile in tensor memory into the step's output:
 //
-//   KIND_LSE  (pass 1)  z = X W^T per [256 tokens x 512 vocab] tile; the
+//   KIND_LSE  (pass 1)  z = X W^T per [128 tokens x 256 vocab] tile; the
 //                       epilogue keeps an online row max and sum of
 //                       exponentials over the tiles of one vocabulary split and
 //                       picks out the target logit.  No logit leaves the chip.
@@ -22,19 +22,10 @@
 // actually gets replaced").
 //
 // The CTAs run in pairs (clusters of two on neighbouring SMs).  A pair owns one
-// 256 x 512 accumulator tile, held as two halves of 256 x 256, one per half of
-// each CTA's tensor memory (all 512 columns).  For every 64-wide k-block each
-// CTA loads 128 rows of A and, for each half, 128 columns of B into its own
-// shared memory; the leader CTA issues one cta_group::2 UMMA group per half,
-// both reading the same A.  Per SM that is 48 KB of operands per 2 x 512
-// tensor-core cycles, a quarter less than a 256 x 256 pair tile needs.
-//
-// With the whole tensor memory in one tile there is no second accumulator for
-// the epilogue to drain while the next tile accumulates.  Instead the two
-// halves are staggered at the ends of each tile: for its last LAG k-blocks the
-// leader issues half 0 first and commits it, then half 1, so the epilogue
-// drains half 0 while half 1 finishes; the next tile issues half 0 for its
-// first LAG k-blocks before half 1, while the epilogue drains half 1.
+// 256 x 256 accumulator tile: each CTA loads 128 rows of A and 128 columns of B
+// into its own shared memory, the leader CTA issues cta_group::2 UMMAs that read
+// both halves, and each CTA's tensor memory receives its 128 rows.  Per SM this
+// halves the B-operand traffic of a 128 x 256 single-CTA tile.
 //
 // Warp roles (192 threads per CTA): warp 0 issues TMA loads, warp 1 issues UMMAs
 // (leader CTA only) and owns the tensor-memory allocation, warps 2..5 run the
@@ -49,24 +40,22 @@
 
 namespace flce {
 
-constexpr int CLUSTER = 2;            // SM pair: the two CTAs of a cluster share one UMMA tile
-constexpr int BM = 128;               // accumulator rows per CTA (TMEM lanes)
-constexpr int CM = CLUSTER * BM;      // rows of the pair's tile (UMMA M = 256)
-constexpr int SUBN = 256;             // columns of one UMMA (N) = one accumulator half
-constexpr int NSUB = 2;               // halves per pair tile
-constexpr int BN = NSUB * SUBN;       // columns of the pair's tile
-constexpr int SUBNH = SUBN / CLUSTER; // B columns of one half that each CTA holds
-constexpr int BK = 64;                // K per pipeline stage: one 128-B swizzle row of bf16
-constexpr int UMMA_K = 16;            // K per tcgen05.mma kind::f16
-constexpr int STAGES = 4;
+constexpr int CLUSTER = 2;     // SM pair: the two CTAs of a cluster share one UMMA tile
+constexpr int BM = 128;        // accumulator rows per CTA (TMEM lanes)
+constexpr int CM = CLUSTER * BM;  // rows of the pair's tile (UMMA M = 256)
+constexpr int BN = 256;        // accumulator columns (UMMA N)
+constexpr int BNH = BN / CLUSTER; // B columns each CTA of the pair holds
+constexpr int BK = 64;         // K per pipeline stage: one 128-B swizzle row of bf16
+constexpr int UMMA_K = 16;     // K per tcgen05.mma kind::f16
+constexpr int STAGES = 6;
 constexpr int A_TILE_BYTES = BM * BK * 2;
-constexpr int B_SUB_BYTES = SUBNH * BK * 2;
-constexpr int STAGE_BYTES = A_TILE_BYTES + NSUB * B_SUB_BYTES;
+constexpr int B_TILE_BYTES = BNH * BK * 2;
+constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
 constexpr int MN_BOX_BYTES = 64 * BK * 2;  // one 64(MN) x 64(K) MN-major box
 constexpr int NUM_THREADS = 192;
 constexpr int EPI_WARPS = 4;
-constexpr int TMEM_COLS = NSUB * SUBN;     // the whole tensor memory of the SM
-constexpr int MAX_LAG = STAGES - 1;        // k-blocks a stagger may hold back
+constexpr int ACC_COLS = BN;
+constexpr int TMEM_COLS = 2 * ACC_COLS;    // double-buffered accumulator
 // Epilogue staging: each epilogue warp owns two 4 KB buffers, each holding a
 // 32-row x 32-column bf16 box of the output (and, for dX, of the low half of
 // the running sum), stored with the 64-byte TMA swizzle.
@@ -75,14 +64,18 @@ constexpr int EPI_BOX_BYTES = EPI_BOX * EPI_BOX * 2;
 constexpr int EPI_BUF_BYTES = 2 * EPI_BOX_BYTES;
 constexpr int EPI_WARP_BYTES = 2 * EPI_BUF_BYTES;
 constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP_BYTES;
-// barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin, epilogue loads[2 per warp]
-constexpr int BAR_TFULL = 2 * STAGES, BAR_TEMPTY = 2 * STAGES + 2, BAR_FIN = 2 * STAGES + 4,
-              BAR_EPI = 2 * STAGES + 5;
-constexpr int NUM_BARRIERS = BAR_EPI + 2 * EPI_WARPS;
+// barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin, epilogue loads[2 per warp], drain
+constexpr int BAR_DRAIN = 2 * STAGES + 5 + 2 * EPI_WARPS;
+constexpr int NUM_BARRIERS = BAR_DRAIN + 1;
+// words after the barriers: tensor-memory address, abort flag, ring positions
+// the producer filled and the issuer consumed
+constexpr int SLOT_WORDS = 4;
+static_assert(NUM_BARRIERS * 8 + SLOT_WORDS * 4 <= 256, "barrier area");
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
-// Pass 1 stages nothing through shared memory in its epilogue.
-constexpr int P1_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
-static_assert(NUM_BARRIERS * 8 + 8 <= 256, "barrier area");
+// Pass 1 stages nothing through shared memory in its epilogue and needs no
+// staging area (a seventh stage measured no faster).
+constexpr int P1_STAGES = STAGES;
+constexpr int P1_SMEM_BYTES = P1_STAGES * STAGE_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr double LN2 = 0.6931471805599453;
 
@@ -112,14 +105,13 @@ enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
 
 struct GemmArgs {
   int N, H, V, ignore_index;
-  int tiles_m, tiles_n;   // pass 1: 256-token tiles, 512-wide vocabulary tiles
+  int tiles_m, tiles_n;   // pass 1: 256-token tiles, 256-wide vocabulary tiles
   int k_blocks;           // pass 1: BK-wide steps along K = H
   int num_units;          // pass 1: tiles_m * splits
   int splits;             // pass 1: vocabulary splits
   int v_off;              // pass 1: vocabulary id of W's row 0 (a launch over a range of the vocabulary)
   int split_off;          // pass 1: first partial slot of this launch's splits
   int Vc;                 // pass 2: chunk width = row stride of the G buffer
-  int lag;                // k-blocks of the stagger at each end of a tile, 1 .. MAX_LAG
   const int32_t* y;
   float* part_m;          // [splits][N] running max, log2 units
   float* part_l;          // [splits][N] running sum of 2^(s - m)
@@ -145,16 +137,15 @@ struct GemmArgs {
   const int* perm;               // [ceil(N/256)*256] row of X behind each row
   const int* reordered;          // device word: 1 when the rows are reordered
   // pass 2 (one persistent launch over every chunk)
-  int TM, HN;             // 256-row token tiles, 512-column hidden tiles
+  int TM, HN;             // 256-row token tiles, 256-column hidden tiles
   int C;                  // vocabulary chunks
-  int VTf, VT_last;       // 512-wide vocabulary tiles (G items) in a full / the last chunk
-  int VMf, VM_last;       // 256-row vocabulary tiles (dW items) in a full / the last chunk
+  int VTf, VT_last;       // 256-wide vocabulary tiles in a full / the last chunk
   long long total_items;
   long long item_begin, item_end;  // the items of the queue this launch runs
-  int* g_row;             // [TM]  G tiles finished per token tile        (x EPI_WARPS*CLUSTER)
-  int* g_col;             // [VTf] G tiles finished per 512-wide column   (x EPI_WARPS*CLUSTER)
-  int* x_row;             // [TM]  dX tiles finished per token tile       (x EPI_WARPS*CLUSTER)
-  int* w_col;             // [VMf] dW tiles finished per 256-row vocab tile (x EPI_WARPS*CLUSTER)
+  int* g_row;             // [TM]  G tiles finished per token tile    (x EPI_WARPS*CLUSTER)
+  int* g_col;             // [VTf] G tiles finished per chunk column  (x EPI_WARPS*CLUSTER)
+  int* x_row;             // [TM]  dX tiles finished per token tile   (x EPI_WARPS*CLUSTER)
+  int* w_col;             // [VTf] dW tiles finished per chunk column (x EPI_WARPS*CLUSTER)
 };
 
 __device__ __forceinline__ void raise_status(int* status, int code) {
@@ -175,7 +166,7 @@ __device__ __forceinline__ void give_up_pair(volatile int* abort_flag, int rank,
 }
 
 // Pass-1 work unit u -> token tile mb, vocabulary split `split` and the range
-// [nb_begin, nb_end) of 512-wide vocabulary tiles it walks.  Units are ordered
+// [nb_begin, nb_end) of 256-wide vocabulary tiles it walks.  Units are ordered
 // split-major, so that SM pairs running at the same time share the same W
 // tiles through L2.
 __device__ __forceinline__ void unit_range(const GemmArgs& a, int u, int& mb, int& nb_begin, int& nb_end,
@@ -186,113 +177,23 @@ __device__ __forceinline__ void unit_range(const GemmArgs& a, int u, int& mb, in
   nb_end = static_cast<int>((static_cast<long long>(split + 1) * a.tiles_n) / a.splits);
 }
 
+// Pass-1 TMA loads of one pipeline stage for the CTA of rank `rank` in the pair:
+// its 128 rows of X and its 128 rows of W, both K-major.  X is read again by
+// every vocabulary tile (keep it in L2); W streams through once.
+__device__ __forceinline__ void load_stage_pass1(const CUtensorMap* mX, const CUtensorMap* mW, uint32_t sA,
+                                                 uint32_t sB, uint32_t bar, int mb, int nb, int kb, int rank,
+                                                 uint64_t keep, uint64_t stream) {
+  const int k0 = kb * BK;
+  tma_load_2d_pair(sA, mX, bar, k0, mb * CM + rank * BM, keep);
+  tma_load_2d_pair(sB, mW, bar, k0, nb * BN + rank * BNH, stream);
+}
+
 template <bool MN>
 __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
   if constexpr (MN)
     return sdesc_sw128(base + k * (UMMA_K * 128), MN_BOX_BYTES, 1024);
   else
     return sdesc_sw128(base + k * (UMMA_K * 2), 16, 1024);
-}
-
-// --------------------------------------------------------------- pipeline --
-
-// Shared-memory layout of a GEMM CTA and the ring of operand stages.
-struct Pipe {
-  uint32_t base;     // stage 0 (shared address, 1024-B aligned)
-  uint32_t bars;     // barrier slot 0
-  int stage;
-  uint32_t phase;
-  __device__ __forceinline__ uint32_t bar(int i) const { return bars + 8u * static_cast<uint32_t>(i); }
-  __device__ __forceinline__ uint32_t full(int s) const { return bar(s); }
-  __device__ __forceinline__ uint32_t empty(int s) const { return bar(STAGES + s); }
-  __device__ __forceinline__ uint32_t sA(int s) const { return base + static_cast<uint32_t>(s) * STAGE_BYTES; }
-  __device__ __forceinline__ uint32_t sB(int s, int half) const {
-    return sA(s) + A_TILE_BYTES + static_cast<uint32_t>(half) * B_SUB_BYTES;
-  }
-  __device__ __forceinline__ void advance() {
-    if (++stage == STAGES) {
-      stage = 0;
-      phase ^= 1u;
-    }
-  }
-};
-
-// Issues the UMMAs of one tile of the leader CTA: `nkb` k-blocks from the stage
-// ring, into half 0 and (when `two`) half 1 of the tensor memory.
-//   head (first h k-blocks):  half 0, then half 1 once the epilogue has freed it;
-//   body:                     both halves per k-block;
-//   tail (last t k-blocks):   half 0, commit tfull[0], then half 1, commit tfull[1].
-// tempty[j] is waited for before anything is written to half j (also when
-// `two` is false, so that each half's barriers advance one phase per tile).
-// Returns false when a wait gave up.
-__device__ __forceinline__ bool issue_tile(Pipe& p, int nkb, bool two, int lag, uint32_t tmem_base, uint32_t idesc,
-                                           bool a_mn, bool b_mn, uint32_t (&tph)[2], volatile int* abort,
-                                           unsigned long long timeout_ns) {
-  const int s0 = p.stage;
-  const uint32_t p0 = p.phase;
-  auto st = [&](int i) { return (s0 + i) % STAGES; };
-  auto ph = [&](int i) { return p0 ^ static_cast<uint32_t>(((s0 + i) / STAGES) & 1); };
-  auto mma = [&](int half, int i, bool first) {
-    const uint32_t sa = p.sA(st(i)), sb = p.sB(st(i), half);
-    const uint32_t d = tmem_base + static_cast<uint32_t>(half * SUBN);
-#pragma unroll
-    for (int k = 0; k < BK / UMMA_K; ++k) {
-      const uint64_t ad = a_mn ? operand_desc<true>(sa, k) : operand_desc<false>(sa, k);
-      const uint64_t bd = b_mn ? operand_desc<true>(sb, k) : operand_desc<false>(sb, k);
-      umma_bf16_pair(d, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
-    }
-  };
-  auto got_full = [&](int i) {
-    if (!mbar_wait(p.full(st(i)), ph(i), abort, timeout_ns)) return false;
-    tc_fence_after();
-    return true;
-  };
-  const int h = min(lag, nkb);
-  const int t = min(lag, nkb - h);
-  if (!mbar_wait<true>(p.bar(BAR_TEMPTY + 0), tph[0] ^ 1u, abort, timeout_ns)) return false;
-  tc_fence_after();
-  for (int i = 0; i < h; ++i) {
-    if (!got_full(i)) return false;
-    mma(0, i, i == 0);
-  }
-  if (!mbar_wait<true>(p.bar(BAR_TEMPTY + 1), tph[1] ^ 1u, abort, timeout_ns)) return false;
-  tc_fence_after();
-  for (int i = 0; i < h; ++i) {
-    if (two) mma(1, i, i == 0);
-    umma_commit_pair(p.empty(st(i)), 0x3);
-  }
-  for (int i = h; i < nkb - t; ++i) {
-    if (!got_full(i)) return false;
-    mma(0, i, false);
-    if (two) mma(1, i, false);
-    umma_commit_pair(p.empty(st(i)), 0x3);
-  }
-  for (int i = nkb - t; i < nkb; ++i) {
-    if (!got_full(i)) return false;
-    mma(0, i, false);
-  }
-  umma_commit_pair(p.bar(BAR_TFULL + 0), 0x3);
-  for (int i = nkb - t; i < nkb; ++i) {
-    if (two) mma(1, i, false);
-    umma_commit_pair(p.empty(st(i)), 0x3);
-  }
-  umma_commit_pair(p.bar(BAR_TFULL + 1), 0x3);
-  tph[0] ^= 1u;
-  tph[1] ^= 1u;
-  const int q = s0 + nkb;
-  p.stage = q % STAGES;
-  p.phase = p0 ^ static_cast<uint32_t>((q / STAGES) & 1);
-  return true;
-}
-
-// The producer's wait for a free stage, then the leader's expect-tx for the
-// bytes both CTAs will load into it.  Returns the leader's full barrier (a
-// cluster address) for the loads, or 0 when the wait gave up.
-__device__ __forceinline__ uint32_t claim_stage(const Pipe& p, bool leader, bool two, volatile int* abort,
-                                                unsigned long long timeout_ns) {
-  if (!mbar_wait(p.empty(p.stage), p.phase ^ 1u, abort, timeout_ns)) return 0;
-  if (leader) mbar_arrive_expect_tx(p.full(p.stage), CLUSTER * (A_TILE_BYTES + (two ? 2 : 1) * B_SUB_BYTES));
-  return mapa_shared(p.full(p.stage), 0);
 }
 
 // ------------------------------------------------------------- epilogues --
@@ -303,11 +204,11 @@ struct LseState {
   bool has_zy;
 };
 
-// Pass 1: fold one [128 x 256] half of a logit tile, vocabulary columns
-// col_base .., into the running (max, sum) of the row.
-__device__ __forceinline__ void epi_lse_half(const GemmArgs& a, uint32_t taddr, int col_base, LseState& st) {
+// Pass 1: fold one [128 x 256] logit tile into the running (max, sum) of the row.
+__device__ __forceinline__ void epi_lse_tile(const GemmArgs& a, uint32_t taddr, int nb, LseState& st) {
+  const int col_base = nb * BN;
 #pragma unroll 1
-  for (int c = 0; c < SUBN / 32; ++c) {
+  for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
@@ -390,9 +291,8 @@ __device__ __forceinline__ void stage_and_store(EpiStage& es, int lane, const CU
   ++es.k;
 }
 
-// Pass 2: G = valid * (softmax - onehot) / n for one half tile, stored as bf16
-// at G-buffer columns gcol .. gcol+255 (vocabulary vbase + gcol ..).
-__device__ __forceinline__ void epi_grad_half(const GemmArgs& a, int vbase, uint32_t taddr, int row0, int gcol,
+// Pass 2: G = valid * (softmax - onehot) / n for one tile, stored as bf16.
+__device__ __forceinline__ void epi_grad_tile(const GemmArgs& a, int vbase, uint32_t taddr, int row0, int nb,
                                               int row_local, EpiStage& es, const CUtensorMap* mapG) {
   const int row = row0 + row_local;
   const int lane = row_local & 31;
@@ -403,13 +303,13 @@ __device__ __forceinline__ void epi_grad_half(const GemmArgs& a, int vbase, uint
   const float scale = valid ? row_weight(a.reduction, a.inv_n, a.grad_row_scale, row) : 0.f;
   const int wrow0 = row0 + (row_local & ~31);
 #pragma unroll 1
-  for (int c = 0; c < SUBN / 32; ++c) {
+  for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
-    const int colg0 = vbase + gcol + c * 32;
+    const int colg0 = vbase + nb * BN + c * 32;
     const int lim = a.V - colg0;
-    stage_and_store(es, lane, mapG, gcol + c * 32, wrow0, l2_evict_normal(), [&](float (&g)[32]) {
+    stage_and_store(es, lane, mapG, nb * BN + c * 32, wrow0, l2_evict_normal(), [&](float (&g)[32]) {
 #pragma unroll
       for (int t = 0; t < 32; ++t)
         g[t] = (valid && t < lim) ? ex2_approx(fmaf(__uint_as_float(r[t]), LOG2E, -l2)) * scale : 0.f;
@@ -424,62 +324,62 @@ __device__ __forceinline__ void epi_grad_half(const GemmArgs& a, int vbase, uint
 }
 
 // dW rows of this chunk: the K = tokens contraction is complete, round to bf16.
-__device__ __forceinline__ void epi_dw_half(uint32_t taddr, int wrow_base, int col, int row_local, EpiStage& es,
-                                            const CUtensorMap* mapDW) {
+__device__ __forceinline__ void epi_dw_tile(int vbase, uint32_t taddr, int row0, int nb, int row_local,
+                                            EpiStage& es, const CUtensorMap* mapDW) {
   const int lane = row_local & 31;
-  const int wrow0 = wrow_base + (row_local & ~31);
+  const int wrow0 = vbase + row0 + (row_local & ~31);
 #pragma unroll 1
-  for (int c = 0; c < SUBN / 32; ++c) {
+  for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
-    stage_and_store(es, lane, mapDW, col + c * 32, wrow0, l2_evict_first(), [&](float (&v)[32]) {
+    stage_and_store(es, lane, mapDW, nb * BN + c * 32, wrow0, l2_evict_first(), [&](float (&v)[32]) {
 #pragma unroll
       for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
     });
   }
 }
 
-// Writes a half tile of zeros (rows row0.., columns col..) without reading the
+// Writes a tile of zeros (rows row0.., columns nb*BN..) without reading the
 // accumulator: outputs of rows that are all ignored, or a contraction with
 // no k-block left.
-__device__ __forceinline__ void epi_zero_half(int row0, int col, int row_local, EpiStage& es,
+__device__ __forceinline__ void epi_zero_tile(uint32_t taddr, int row0, int nb, int row_local, EpiStage& es,
                                               const CUtensorMap* map) {
+  (void)taddr;
   const int lane = row_local & 31;
   const int wrow0 = row0 + (row_local & ~31);
 #pragma unroll 1
-  for (int c = 0; c < SUBN / 32; ++c) {
-    stage_and_store(es, lane, map, col + c * 32, wrow0, l2_evict_first(), [&](float (&v)[32]) {
+  for (int c = 0; c < BN / 32; ++c) {
+    stage_and_store(es, lane, map, nb * BN + c * 32, wrow0, l2_evict_first(), [&](float (&v)[32]) {
 #pragma unroll
       for (int t = 0; t < 32; ++t) v[t] = 0.f;
     });
   }
 }
 
-// dX += G_c W_c for one half tile (columns col ..).  The running sum lives in
-// two bf16 words, hi (in dX itself) and lo (workspace), with value = hi + lo:
-// about 16 significant bits, enough for an fp32-grade sum over the chunks, at
-// the memory cost of one bf16 copy of dX.  Each 32-column slice of the warp's
-// rows is read back (hi and lo boxes by TMA, one slice ahead), combined with
-// the accumulator and written back by TMA.  The last chunk writes the rounded
-// sum through `mapFinal` (dX itself, or the workspace when the rows are
-// reordered and a scatter puts them in place).
-__device__ __forceinline__ void epi_dx_half(const GemmArgs& a, bool first_chunk, bool last_chunk, uint32_t taddr,
-                                            int row0, int col, int row_local, EpiStage& es, const CUtensorMap* mapHi,
+// dX += G_c W_c.  The running sum lives in two bf16 words, hi (in dX itself) and
+// lo (workspace), with value = hi + lo: about 16 significant bits, enough for an
+// fp32-grade sum over the chunks, at the memory cost of one bf16 copy of dX.
+// Each 32-column slice of the warp's rows is read back (hi and lo boxes by TMA,
+// one slice ahead), combined with the accumulator and written back by TMA.
+// The last chunk writes the rounded sum through `mapFinal` (dX itself, or the
+// workspace when the rows are reordered and a scatter puts them in place).
+__device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk, bool last_chunk, uint32_t taddr,
+                                            int row0, int nb, int row_local, EpiStage& es, const CUtensorMap* mapHi,
                                             const CUtensorMap* mapLo, const CUtensorMap* mapFinal,
                                             volatile int* abort_flag, bool& ok) {
   const int lane = row_local & 31;
   const int wrow0 = row0 + (row_local & ~31);
   const bool accumulate = !first_chunk;
-  constexpr int SLICES = SUBN / 32;
+  constexpr int SLICES = BN / 32;
   const uint64_t stream = l2_evict_first();  // the running sum is touched once per chunk
   auto fetch = [&](uint32_t b, int c) {  // lane 0: hi and lo boxes of slice c into buffer b
     bulk_wait_read<0>();                 // the buffer's previous store has read it
     fence_proxy_async_smem();
     const uint32_t bar = es.bar + 8u * b;
     mbar_arrive_expect_tx(bar, 2 * EPI_BOX_BYTES);
-    tma_load_2d(es.addr + b * EPI_BUF_BYTES, mapHi, bar, col + c * 32, wrow0, stream);
-    tma_load_2d(es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, mapLo, bar, col + c * 32, wrow0, stream);
+    tma_load_2d(es.addr + b * EPI_BUF_BYTES, mapHi, bar, nb * BN + c * 32, wrow0, stream);
+    tma_load_2d(es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, mapLo, bar, nb * BN + c * 32, wrow0, stream);
   };
   if (accumulate && lane == 0) fetch(es.k & 1u, 0);
 #pragma unroll 1
@@ -502,15 +402,23 @@ __device__ __forceinline__ void epi_dx_half(const GemmArgs& a, bool first_chunk,
     if (accumulate) {
       const bool got = mbar_wait(es.bar + 8u * b, (es.k >> 1) & 1u, abort_flag, a.timeout_ns);
       if (!__all_sync(0xffffffffu, got)) {
+        // let the boxes still in flight land in this warp's buffers before it
+        // leaves: this slice's, and the next slice's if it was fetched
+        if (lane == 0) {
+          volatile int never = 0;
+          mbar_wait(es.bar + 8u * b, (es.k >> 1) & 1u, &never, 1000000ull);
+          if (c + 1 < SLICES) mbar_wait(es.bar + 8u * (b ^ 1u), ((es.k + 1) >> 1) & 1u, &never, 1000000ull);
+        }
+        __syncwarp();
         ok = false;
         return;
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 hv = *reinterpret_cast<const uint4*>(hbox + sw64(lane, j));
-        const uint4 lv = *reinterpret_cast<const uint4*>(lbox + sw64(lane, j));
-        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-        const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
+        const uint4 h = *reinterpret_cast<const uint4*>(hbox + sw64(lane, j));
+        const uint4 l = *reinterpret_cast<const uint4*>(lbox + sw64(lane, j));
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+        const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           v[8 * j + 2 * e] += bf16lo_to_f32(hw[e]) + bf16lo_to_f32(lw[e]);
@@ -533,67 +441,58 @@ __device__ __forceinline__ void epi_dx_half(const GemmArgs& a, bool first_chunk,
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(last_chunk ? mapFinal : mapHi, es.addr + b * EPI_BUF_BYTES, col + c * 32, wrow0, stream);
+      tma_store_2d(last_chunk ? mapFinal : mapHi, es.addr + b * EPI_BUF_BYTES, nb * BN + c * 32, wrow0, stream);
       if (!last_chunk)
-        tma_store_2d(mapLo, es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, col + c * 32, wrow0, stream);
+        tma_store_2d(mapLo, es.addr + b * EPI_BUF_BYTES + EPI_BOX_BYTES, nb * BN + c * 32, wrow0, stream);
       bulk_commit();
     }
     ++es.k;
   }
 }
 
-// Waits (all lanes of an epilogue warp) for half `j` of the accumulator.
-__device__ __forceinline__ bool wait_half(const Pipe& p, int j, uint32_t (&eph)[2], volatile int* abort,
-                                          unsigned long long timeout_ns) {
-  const bool got = mbar_wait(p.bar(BAR_TFULL + j), eph[j], abort, timeout_ns);
-  if (!__all_sync(0xffffffffu, got)) return false;
-  tc_fence_after();
-  return true;
-}
-// Hands half `j` of the accumulator back to the leader's issuer.
-__device__ __forceinline__ void release_half(uint32_t tempty_leader, int lane, int j, uint32_t (&eph)[2]) {
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive_cluster(tempty_leader);
-  eph[j] ^= 1u;
-}
-
-// Common start of both GEMM kernels: barriers, tensor memory, cluster sync.
-__device__ __forceinline__ void gemm_setup(const Pipe& p, uint32_t* tmem_slot, volatile int* abort_flag, int warp) {
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(p.full(s), 1);   // leader: its producer's arrive + both CTAs' bytes
-      mbar_init(p.empty(s), 1);  // the leader's UMMA commit, multicast to both
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(p.bar(BAR_TFULL + b), 1);                     // UMMA commit, multicast to both
-      mbar_init(p.bar(BAR_TEMPTY + b), CLUSTER * EPI_WARPS);  // leader: epilogue warps of both CTAs
-    }
-    mbar_init(p.bar(BAR_FIN), 1);  // the peer's end-of-work signal
-    for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(p.bar(BAR_EPI + e), 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync_all();  // barriers of both CTAs initialised before any cross-CTA use
-  tc_fence_after();
-}
+// ------------------------------------------------------------- wind-down --
 
 // Wind-down of both GEMM kernels: this CTA's work is done; tell the peer, wait
 // (bounded) for the peer to say the same, then free the pair's tensor memory
-// together.
-__device__ __forceinline__ void gemm_teardown(const Pipe& p, uint32_t tmem_base, int rank, int warp, int* status,
-                                              unsigned long long timeout_ns) {
+// together.  What is known complete before the tensor memory is freed and the
+// CTA exits:
+//   - every UMMA: the leader's last commit (issued after all its UMMAs, also
+//     after a give-up) arrives on the drain barrier of both CTAs once they
+//     have all completed;
+//   - every TMA store, and every epilogue TMA load: the epilogue warps wait
+//     for them (bulk groups; the running-sum boxes' barriers);
+//   - the operand loads: after a give-up, the leader waits on the full barrier
+//     of every ring position its producer filled and its issuer did not
+//     consume; each completes once both CTAs' bytes have landed, and only then
+//     does the leader tell the peer it is done.  Only if the two producers
+//     stopped at different positions can a load be left that no barrier
+//     reports; a fixed 100 us grace period covers that case.
+// Every wait here ends by completion or by its own time limit, not by the
+// abort flag.
+__device__ __forceinline__ void pair_wind_down(uint32_t bars, const uint32_t* slots, int rank, int warp,
+                                               volatile int* abort_flag, int* status, unsigned long long timeout_ns) {
+  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
-    mbar_arrive_cluster(mapa_shared(p.bar(BAR_FIN), static_cast<uint32_t>(rank ^ 1)));
+    volatile int never = 0;
+    if (!mbar_wait(bar(BAR_DRAIN), 0u, &never, END_WAIT_LIMITS * timeout_ns)) raise_status(status, ST_TIMEOUT);
+    if (*abort_flag && rank == 0) {
+      const long long filled = slots[2], consumed = slots[3];
+      bool all = true;
+      for (long long q = consumed; q < filled; ++q)
+        all = mbar_wait(bar(static_cast<int>(q % STAGES)), static_cast<uint32_t>((q / STAGES) & 1), &never,
+                        1000000ull) && all;
+      if (!all) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 100000ull) {
+        }
+      }
+    }
+    const uint32_t fin = bar(2 * STAGES + 4);
+    mbar_arrive_cluster(mapa_shared(fin, static_cast<uint32_t>(rank ^ 1)));
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait_cluster(p.bar(BAR_FIN), 0)) {
+    while (!mbar_try_wait_cluster(fin, 0)) {
       if (globaltimer_ns() - t0 > END_WAIT_LIMITS * timeout_ns) {
         raise_status(status, ST_TIMEOUT);
         break;
@@ -603,23 +502,29 @@ __device__ __forceinline__ void gemm_teardown(const Pipe& p, uint32_t tmem_base,
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(slots[0], TMEM_COLS);
   }
 }
 
 // The producer's tail: wait for the UMMA commits still headed for this CTA's
-// empty barriers, so none lands after the CTA has gone; after a give-up, let
-// copies already in flight land before the CTA can exit.
-__device__ __forceinline__ void producer_tail(Pipe& p, volatile int* abort_flag, unsigned long long timeout_ns,
-                                              int rank, int* status) {
+// empty barriers, so none lands after the CTA has gone, and record how far it
+// filled the ring.  After a give-up the peer's producer (which cannot see the
+// leader's full barriers) lets copies in flight land for 100 us.
+__device__ __forceinline__ void producer_tail(uint32_t bars, uint32_t* slots, long long filled, int& stage,
+                                              uint32_t& phase, volatile int* abort_flag,
+                                              unsigned long long timeout_ns, int rank, int* status) {
+  slots[2] = static_cast<uint32_t>(filled);
   for (int i = 0; i < STAGES; ++i) {
-    if (!mbar_wait(p.empty(p.stage), p.phase ^ 1u, abort_flag, timeout_ns)) {
+    if (!mbar_wait(bars + 8u * static_cast<uint32_t>(STAGES + stage), phase ^ 1u, abort_flag, timeout_ns)) {
       give_up_pair(abort_flag, rank, status);
       break;
     }
-    p.advance();
+    if (++stage == STAGES) {
+      stage = 0;
+      phase ^= 1u;
+    }
   }
-  if (*abort_flag) {
+  if (*abort_flag && rank != 0) {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 100000ull) {
     }
@@ -639,7 +544,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;  // swizzle atoms need 1024-B alignment
   uint8_t* base_ptr = smem_raw + (base - raw_addr);
+  constexpr int STAGES = P1_STAGES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + STAGES * STAGE_BYTES);
+  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -649,79 +556,147 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   const bool leader = rank == 0;
   const int cid = blockIdx.x / CLUSTER;
   const int ncl = gridDim.x / CLUSTER;
-  Pipe p{base, smem_u32(bars), 0, 0u};
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 + b); };
+  const uint32_t fin_bar = smem_u32(bars + 2 * STAGES + 4);
+  auto sA = [&](int s) { return base + s * STAGE_BYTES; };
+  auto sB = [&](int s) { return base + s * STAGE_BYTES + A_TILE_BYTES; };
 
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);    // leader: its producer's arrive + both CTAs' bytes
+      mbar_init(empty_bar(s), 1);   // the leader's UMMA commit, multicast to both
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);                 // UMMA commit, multicast to both
+      mbar_init(tempty_bar(b), CLUSTER * EPI_WARPS);  // leader: epilogue warps of both CTAs
+    }
+    mbar_init(fin_bar, 1);  // the peer's end-of-work signal
+    mbar_init(smem_u32(bars + BAR_DRAIN), 1);  // the leader's last UMMA commit
+    *abort_flag = 0;
+    tmem_slot[2] = tmem_slot[3] = 0;
+    fence_mbar_init();
+  }
   // X rows in the token-row order: the caller's X, or its packed copy
   const CUtensorMap* mX = *a.reordered != 0 ? &mapXc : &mapX;
   if (warp == 0 && lane == 0) {
     prefetch_tmap(mX);
     prefetch_tmap(&mapW);
   }
-  gemm_setup(p, tmem_slot, abort_flag, warp);
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any cross-CTA use
+  tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+
   auto give_up = [&]() { give_up_pair(abort_flag, rank, a.status); };
-  // a vocabulary tile has a second half when any of its columns 256.. exist
-  auto two_halves = [&](int nb) { return nb * BN + SUBN < a.V; };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
       const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      long long filled = 0;
       bool ok = true;
       for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
         unit_range(a, u, mb, nb0, nb1, split);
         if (a.tile_valid[mb] == 0) continue;  // every row of the tile is ignored
         for (int nb = nb0; ok && nb < nb1; ++nb) {
-          const bool two = two_halves(nb);
           for (int kb = 0; kb < a.k_blocks; ++kb) {
-            const uint32_t bar = claim_stage(p, leader, two, abort_flag, a.timeout_ns);
-            if (bar == 0) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
               give_up();
               ok = false;
               break;
             }
-            const int k0 = kb * BK;
-            tma_load_2d_pair(p.sA(p.stage), mX, bar, k0, mb * CM + rank * BM, keep);
-            for (int j = 0; j < (two ? 2 : 1); ++j)
-              tma_load_2d_pair(p.sB(p.stage, j), &mapW, bar, k0, nb * BN + j * SUBN + rank * SUBNH, stream);
-            p.advance();
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * STAGE_BYTES);
+            load_stage_pass1(mX, &mapW, sA(stage), sB(stage), mapa_shared(full_bar(stage), 0), mb, nb, kb, rank,
+                             keep, stream);
+            ++filled;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
       }
-      producer_tail(p, abort_flag, a.timeout_ns, rank, a.status);
+      producer_tail(smem_u32(bars), tmem_slot, filled, stage, phase, abort_flag, a.timeout_ns, rank, a.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ UMMA issuer (leader) --
     if (leader && lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(CM, SUBN, false, false);
-      uint32_t tph[2] = {0u, 0u};
+      constexpr uint32_t IDESC = idesc_bf16_f32(CM, BN, false, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      long long consumed = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
       bool ok = true;
       for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
         unit_range(a, u, mb, nb0, nb1, split);
         if (a.tile_valid[mb] == 0) continue;  // every row of the tile is ignored
         for (int nb = nb0; ok && nb < nb1; ++nb) {
-          if (!issue_tile(p, a.k_blocks, two_halves(nb), a.lag, tmem_base, IDESC, false, false, tph, abort_flag,
-                          a.timeout_ns)) {
+          if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
             give_up();
             ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+          for (int kb = 0; kb < a.k_blocks; ++kb) {
+            if (!mbar_wait(full_bar(stage), phase, abort_flag, a.timeout_ns)) {
+              give_up();
+              ok = false;
+              break;
+            }
+            ++consumed;
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k)
+              umma_bf16_pair(d_tmem, operand_desc<false>(sA(stage), k), operand_desc<false>(sB(stage), k), IDESC,
+                             (kb | k) != 0);
+            umma_commit_pair(empty_bar(stage), 0x3);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit_pair(tfull_bar(acc), 0x3);
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
         }
       }
-      // Tail: both halves released by the epilogues of both CTAs, so all
+      // Tail: both accumulators released by the epilogues of both CTAs, so all
       // UMMAs are done and no remote arrive is still on its way here.
-      for (int j = 0; ok && j < 2; ++j) {
-        if (!mbar_wait<true>(p.bar(BAR_TEMPTY + j), tph[j] ^ 1u, abort_flag, a.timeout_ns)) give_up();
+      for (int i = 0; i < 2; ++i) {
+        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          break;
+        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
       }
+      // the positions consumed, and one last commit that completes when every UMMA has
+      tmem_slot[3] = static_cast<uint32_t>(consumed);
+      umma_commit_pair(smem_u32(bars + BAR_DRAIN), 0x3);
     }
   } else {
     // ---------------------------------------------------------- epilogue --
     const int q = warp & 3;
     const int row_local = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t tempty_leader[2] = {mapa_shared(p.bar(BAR_TEMPTY + 0), 0), mapa_shared(p.bar(BAR_TEMPTY + 1), 0)};
-    uint32_t eph[2] = {0u, 0u};
+    const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
+    const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
     bool ok = true;
     for (int u = cid; ok && u < a.num_units; u += ncl) {
       int mb, nb0, nb1, split;
@@ -736,17 +711,21 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       st.run_l = 0.f;
       st.zy_val = 0.f;
       st.has_zy = false;
-      for (int nb = nb0; ok && nb < nb1; ++nb) {
-        const bool two = two_halves(nb);
-        for (int j = 0; j < 2; ++j) {
-          if (!wait_half(p, j, eph, abort_flag, a.timeout_ns)) {
-            give_up();
-            ok = false;
-            break;
-          }
-          if (j == 0 || two) epi_lse_half(a, tmem_base + lane_addr + j * SUBN, nb * BN + j * SUBN, st);
-          release_half(tempty_leader[j], lane, j, eph);
+      for (int nb = nb0; nb < nb1; ++nb) {
+        const bool got = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.timeout_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+          give_up();
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
+        epi_lse_tile(a, taddr, nb, st);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
       }
       if (ok && st.row < a.N) {
         a.part_m[static_cast<size_t>(split + a.split_off) * a.N + st.row] = st.run_m;
@@ -755,7 +734,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       }
     }
   }
-  gemm_teardown(p, tmem_base, rank, warp, a.status, a.timeout_ns);
+
+  pair_wind_down(smem_u32(bars), tmem_slot, rank, warp, abort_flag, a.status, a.timeout_ns);
 }
 
 // ===================================================== pass 2, one launch ==
@@ -765,20 +745,19 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
 //
 //   G(0)  |  dX(0) dW(0) G(1)  |  dX(1) dW(1) G(2)  | ... |  dX(C-1) dW(C-1)
 //
-// where G(c) are the logit-recompute tiles of chunk c (256 tokens x 512
-// vocabulary entries), dX(c) the dX += G_c W_c tiles (256 tokens x 512 hidden)
-// and dW(c) the dW rows of chunk c (256 vocabulary rows x 512 hidden).  The G
-// tiles of a chunk go column by column (all token tiles of one vocabulary
-// tile, then the next) when a chunk holds more than three rounds of them for
-// the SM pairs: the dW(c) items that their epilogues wait for finish column by
-// column.  With fewer rounds they go row by row, so that each token tile's G
-// row is complete early and the dX(c) items that wait for it are not all held
-// up by the last column.  There is one G buffer, so items wait for what they
-// read and for the readers of what they overwrite:
+// where G(c) are the logit-recompute tiles of chunk c, dX(c) the
+// dX += G_c W_c tiles and dW(c) the dW rows of chunk c.  The G tiles of a
+// chunk go column by column (all token tiles of one vocabulary tile, then the
+// next) when a chunk holds more than three rounds of them for the SM pairs:
+// the dW(c) items that their epilogues wait for finish column by column.  With
+// fewer rounds they go row by row, so that each token tile's G row is complete
+// early and the dX(c) items that wait for it are not all held up by the last
+// column.  There is one G buffer,
+// so items wait for what they read and for the readers of what they overwrite:
 //   dX(c) mainloop  after G(c) of its token tile (all its columns),
 //   dX(c) epilogue  after dX(c-1) of its token tile (running sum),
-//   dW(c) mainloop  after G(c) of the 512-wide column holding its rows,
-//   G(c)  epilogue  after dX(c-1) of its token tile and dW(c-1) of its rows.
+//   dW(c) mainloop  after G(c) of its column (all token tiles),
+//   G(c)  epilogue  after dX(c-1) of its token tile and dW(c-1) of its column.
 // Every dependency points to an earlier item and all SM pairs are resident at
 // once, so the queue always drains.  Completion is counted per token tile /
 // column in monotonic counters: each epilogue warp adds one after its TMA
@@ -791,10 +770,9 @@ struct Item {
 };
 
 __device__ __forceinline__ int chunk_vtiles(const GemmArgs& p, int c) { return c == p.C - 1 ? p.VT_last : p.VTf; }
-__device__ __forceinline__ int chunk_vmtiles(const GemmArgs& p, int c) { return c == p.C - 1 ? p.VM_last : p.VMf; }
 
 __device__ __forceinline__ long long section_size(const GemmArgs& p, int c) {
-  long long n = static_cast<long long>(p.TM) * p.HN + static_cast<long long>(chunk_vmtiles(p, c)) * p.HN;
+  long long n = static_cast<long long>(p.TM) * p.HN + static_cast<long long>(chunk_vtiles(p, c)) * p.HN;
   if (c + 1 < p.C) n += static_cast<long long>(chunk_vtiles(p, c + 1)) * p.TM;
   return n;
 }
@@ -839,7 +817,7 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
     ++c;
   }
   const long long nx = static_cast<long long>(p.TM) * p.HN;
-  const long long nw = static_cast<long long>(chunk_vmtiles(p, c)) * p.HN;
+  const long long nw = static_cast<long long>(chunk_vtiles(p, c)) * p.HN;
   it.c = c;
   if (r < nx) {
     it.kind = ITEM_DX;
@@ -868,34 +846,9 @@ struct Pass2Maps {
   CUtensorMap Gk, Wmn;     // dX: G_c rows K-major, W_c MN-major
   CUtensorMap Go, DWo;     // epilogue output boxes of G and dW
   CUtensorMap Hio, Loo;    // epilogue boxes of the dX running sum (hi = dX, lo)
-  CUtensorMap Hipf, Lopf;  // whole-half L2 prefetch of the running sum
+  CUtensorMap Hipf, Lopf;  // whole-tile L2 prefetch of the running sum
   CUtensorMap Xck, Xcmn;   // the packed copy of X (reordered rows), K- and MN-major
 };
-
-// Geometry of one pass-2 item: its k-blocks and whether its tile has a second half.
-struct ItemShape {
-  int kblocks;  // k-blocks the mainloop walks (before the dW skip of ignored token tiles)
-  bool two;     // the tile's columns 256.. hold any output
-  bool skip;    // G or dX tile whose rows are all ignored: no mainloop
-};
-
-__device__ __forceinline__ ItemShape item_shape(const GemmArgs& a, const Item& it) {
-  ItemShape s;
-  const int vcount = min(a.Vc, a.V - it.c * a.Vc);
-  s.skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
-  if (it.kind == ITEM_GRAD) {
-    s.kblocks = (a.H + BK - 1) / BK;
-    s.two = it.b * BN + SUBN < vcount;
-  } else if (it.kind == ITEM_DW) {
-    s.kblocks = (a.N + BK - 1) / BK;
-    s.two = it.b * BN + SUBN < a.H;
-  } else {
-    s.kblocks = (vcount + BK - 1) / BK;
-    s.two = it.b * BN + SUBN < a.H;
-  }
-  if (s.skip) s.kblocks = 0;
-  return s;
-}
 
 __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     flce_pass2_kernel(const __grid_constant__ Pass2Maps m, const GemmArgs a) {
@@ -914,8 +867,30 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   const bool leader = rank == 0;
   const long long cid = blockIdx.x / CLUSTER;
   const long long ncl = gridDim.x / CLUSTER;
-  Pipe p{base, smem_u32(bars), 0, 0u};
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 + b); };
+  const uint32_t fin_bar = smem_u32(bars + 2 * STAGES + 4);
+  auto sA = [&](int s) { return base + s * STAGE_BYTES; };
+  auto sB = [&](int s) { return base + s * STAGE_BYTES + A_TILE_BYTES; };
 
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), CLUSTER * EPI_WARPS);
+    }
+    mbar_init(fin_bar, 1);
+    for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(smem_u32(bars + 2 * STAGES + 5 + e), 1);
+    mbar_init(smem_u32(bars + BAR_DRAIN), 1);
+    *abort_flag = 0;
+    tmem_slot[2] = tmem_slot[3] = 0;
+    fence_mbar_init();
+  }
   // X rows in the token-row order: the caller's X, or its packed copy
   const bool reordered = *a.reordered != 0;
   const CUtensorMap* mXk = reordered ? &m.Xck : &m.Xk;
@@ -928,7 +903,13 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     prefetch_tmap(&m.Gk);
     prefetch_tmap(&m.Wmn);
   }
-  gemm_setup(p, tmem_slot, abort_flag, warp);
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   auto give_up = [&]() { give_up_pair(abort_flag, rank, a.status); };
@@ -936,32 +917,38 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   auto g_row_target = [&](int c) {
     return SIGNALS_PER_ITEM * (c < a.C - 1 ? (c + 1) * a.VTf : (a.C - 1) * a.VTf + a.VT_last);
   };
-  // dW: K runs over tokens; k-blocks of all-ignored token tiles add nothing
-  auto dw_kb_valid = [&](int kb) { return a.tile_valid[kb / (CM / BK)] != 0; };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
       const uint64_t keep = l2_evict_last(), normal = l2_evict_normal(), stream = l2_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      long long filled = 0;
       bool ok = true;
       for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
         const Item it = decode_item(a, u);
-        const ItemShape sh = item_shape(a, it);
         const int vbase = it.c * a.Vc;
-        if (sh.skip) {
-          // nothing to load
+        const int vcount = min(a.Vc, a.V - vbase);
+        // G and dX tiles of a token tile whose rows are all ignored are skipped
+        const bool skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
+        int kblocks;
+        if (skip) {
+          kblocks = 0;
+        } else if (it.kind == ITEM_GRAD) {
+          kblocks = (a.H + BK - 1) / BK;
         } else if (it.kind == ITEM_DW) {
-          ok = wait_counter(a.g_col + it.a / (BN / SUBN), SIGNALS_PER_ITEM * a.TM * (it.c + 1) + a.starve_dw,
-                            abort_flag, a.timeout_ns);
-        } else if (it.kind == ITEM_DX) {
+          kblocks = (a.N + BK - 1) / BK;
+          ok = wait_counter(a.g_col + it.a, SIGNALS_PER_ITEM * a.TM * (it.c + 1) + a.starve_dw, abort_flag,
+                            a.timeout_ns);
+        } else {
+          kblocks = (vcount + BK - 1) / BK;
           ok = wait_counter(a.g_row + it.a, g_row_target(it.c), abort_flag, a.timeout_ns);
           // pull this CTA's rows of the running sum into L2 if they are final already
           if (ok && it.c > 0 && ld_acquire_gpu(a.x_row + it.a) >= SIGNALS_PER_ITEM * it.c * a.HN) {
             fence_proxy_async_global();
-            for (int j = 0; j < (sh.two ? 2 : 1); ++j) {
-              tma_prefetch_l2_2d(&m.Hipf, it.b * BN + j * SUBN, it.a * CM + rank * BM, stream);
-              tma_prefetch_l2_2d(&m.Lopf, it.b * BN + j * SUBN, it.a * CM + rank * BM, stream);
-            }
+            tma_prefetch_l2_2d(&m.Hipf, it.b * BN, it.a * CM + rank * BM, stream);
+            tma_prefetch_l2_2d(&m.Lopf, it.b * BN, it.a * CM + rank * BM, stream);
           }
         }
         if (!ok) {
@@ -972,99 +959,141 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         // acquire above before those reads (G tiles read only X and W)
         if (it.kind != ITEM_GRAD) fence_proxy_async_global();
         const int m0 = it.a * CM + rank * BM;
-        for (int kb = 0; kb < sh.kblocks; ++kb) {
-          if (it.kind == ITEM_DW && !dw_kb_valid(kb)) continue;
-          const uint32_t bar = claim_stage(p, leader, sh.two, abort_flag, a.timeout_ns);
-          if (bar == 0) {
+        const int n0 = it.b * BN + rank * BNH;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          // dW: K runs over tokens; k-blocks of all-ignored token tiles add nothing
+          if (it.kind == ITEM_DW && a.tile_valid[kb / (CM / BK)] == 0) continue;
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
             give_up();
             ok = false;
             break;
           }
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * STAGE_BYTES);
+          const uint32_t bar = mapa_shared(full_bar(stage), 0);
           const int k0 = kb * BK;
-          const uint32_t sa = p.sA(p.stage);
-          for (int j = 0; j < (sh.two ? 2 : 1); ++j) {
-            const uint32_t sb = p.sB(p.stage, j);
-            const int n0 = it.b * BN + j * SUBN + rank * SUBNH;
-            if (it.kind == ITEM_GRAD) {
-              if (j == 0) tma_load_2d_pair(sa, mXk, bar, k0, m0, keep);
-              tma_load_2d_pair(sb, &m.Wk, bar, k0, vbase + n0, normal);
-            } else if (it.kind == ITEM_DW) {
-              if (j == 0) {
+          if (it.kind == ITEM_GRAD) {
+            tma_load_2d_pair(sA(stage), mXk, bar, k0, m0, keep);
+            tma_load_2d_pair(sB(stage), &m.Wk, bar, k0, vbase + n0, normal);
+          } else if (it.kind == ITEM_DW) {
 #pragma unroll
-                for (int i = 0; i < BM / 64; ++i)
-                  tma_load_2d_pair(sa + i * MN_BOX_BYTES, &m.Gmn, bar, m0 + i * 64, k0, normal);
-              }
+            for (int i = 0; i < BM / 64; ++i)
+              tma_load_2d_pair(sA(stage) + i * MN_BOX_BYTES, &m.Gmn, bar, m0 + i * 64, k0, normal);
 #pragma unroll
-              for (int i = 0; i < SUBNH / 64; ++i)
-                tma_load_2d_pair(sb + i * MN_BOX_BYTES, mXmn, bar, n0 + i * 64, k0, keep);
-            } else {
-              if (j == 0) tma_load_2d_pair(sa, &m.Gk, bar, k0, m0, normal);
+            for (int i = 0; i < BNH / 64; ++i)
+              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, mXmn, bar, n0 + i * 64, k0, keep);
+          } else {
+            tma_load_2d_pair(sA(stage), &m.Gk, bar, k0, m0, normal);
 #pragma unroll
-              for (int i = 0; i < SUBNH / 64; ++i)
-                tma_load_2d_pair(sb + i * MN_BOX_BYTES, &m.Wmn, bar, n0 + i * 64, vbase + k0, normal);
-            }
+            for (int i = 0; i < BNH / 64; ++i)
+              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, &m.Wmn, bar, n0 + i * 64, vbase + k0, normal);
           }
-          p.advance();
+          ++filled;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
-      producer_tail(p, abort_flag, a.timeout_ns, rank, a.status);
+      producer_tail(smem_u32(bars), tmem_slot, filled, stage, phase, abort_flag, a.timeout_ns, rank, a.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ UMMA issuer (leader) --
     if (leader && lane == 0) {
-      constexpr uint32_t ID_GRAD = idesc_bf16_f32(CM, SUBN, false, false);
-      constexpr uint32_t ID_DW = idesc_bf16_f32(CM, SUBN, true, true);
-      constexpr uint32_t ID_DX = idesc_bf16_f32(CM, SUBN, false, true);
-      // k-blocks of a dW item: those of token tiles holding a valid row (the same for every dW item)
-      int dw_kb = 0;
-      for (int kb = 0; kb < (a.N + BK - 1) / BK; ++kb) dw_kb += dw_kb_valid(kb) ? 1 : 0;
-      uint32_t tph[2] = {0u, 0u};
+      constexpr uint32_t ID_GRAD = idesc_bf16_f32(CM, BN, false, false);
+      constexpr uint32_t ID_DW = idesc_bf16_f32(CM, BN, true, true);
+      constexpr uint32_t ID_DX = idesc_bf16_f32(CM, BN, false, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      long long consumed = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
       bool ok = true;
       for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
         const Item it = decode_item(a, u);
-        const ItemShape sh = item_shape(a, it);
-        const int nkb = it.kind == ITEM_DW ? dw_kb : sh.kblocks;
+        const int vcount = min(a.Vc, a.V - it.c * a.Vc);
+        const bool skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
+        const int kblocks = skip                  ? 0
+                            : it.kind == ITEM_GRAD ? (a.H + BK - 1) / BK
+                            : it.kind == ITEM_DW   ? (a.N + BK - 1) / BK
+                                                   : (vcount + BK - 1) / BK;
         const uint32_t idesc = it.kind == ITEM_GRAD ? ID_GRAD : it.kind == ITEM_DW ? ID_DW : ID_DX;
-        if (!issue_tile(p, nkb, sh.two, a.lag, tmem_base, idesc, it.kind == ITEM_DW, it.kind != ITEM_GRAD, tph,
-                        abort_flag, a.timeout_ns)) {
+        const bool a_mn = it.kind == ITEM_DW;
+        const bool b_mn = it.kind != ITEM_GRAD;
+        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
           give_up();
-          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        uint32_t accumulate = 0;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (it.kind == ITEM_DW && a.tile_valid[kb / (CM / BK)] == 0) continue;
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, a.timeout_ns)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          ++consumed;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            const uint64_t ad = a_mn ? operand_desc<true>(sA(stage), k) : operand_desc<false>(sA(stage), k);
+            const uint64_t bd = b_mn ? operand_desc<true>(sB(stage), k) : operand_desc<false>(sB(stage), k);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, accumulate);
+            accumulate = 1;
+          }
+          umma_commit_pair(empty_bar(stage), 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(tfull_bar(acc), 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
       }
-      for (int j = 0; ok && j < 2; ++j) {
-        if (!mbar_wait<true>(p.bar(BAR_TEMPTY + j), tph[j] ^ 1u, abort_flag, a.timeout_ns)) give_up();
+      for (int i = 0; i < 2; ++i) {
+        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          break;
+        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
       }
+      // the positions consumed, and one last commit that completes when every UMMA has
+      tmem_slot[3] = static_cast<uint32_t>(consumed);
+      umma_commit_pair(smem_u32(bars + BAR_DRAIN), 0x3);
     }
   } else {
     // ---------------------------------------------------------- epilogue --
     const int q = warp & 3;
     const int row_local = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t tempty_leader[2] = {mapa_shared(p.bar(BAR_TEMPTY + 0), 0), mapa_shared(p.bar(BAR_TEMPTY + 1), 0)};
+    const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
+    const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
     EpiStage es;
     es.ptr = epi_ptr + q * EPI_WARP_BYTES;
     es.addr = smem_u32(es.ptr);
-    es.bar = p.bar(BAR_EPI + 2 * q);
+    es.bar = smem_u32(bars + 2 * STAGES + 5 + 2 * q);
     es.k = 0;
     // the rounded dX goes to the workspace when the rows are reordered
     const CUtensorMap* dx_final = reordered ? &m.Loo : &m.Hio;
     // with every token ignored the dW contraction has no k-block at all
     bool any_valid = false;
     for (int t = 0; t < a.TM && !any_valid; ++t) any_valid = a.tile_valid[t] != 0;
-    uint32_t eph[2] = {0u, 0u};
+    int acc = 0;
+    uint32_t acc_phase = 0;
     bool ok = true;
     for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
       const Item it = decode_item(a, u);
-      const ItemShape sh = item_shape(a, it);
       const int vbase = it.c * a.Vc;
       const int row0 = it.a * CM + rank * BM;
       // wait for the previous readers (G) / writers (dX) of what this tile writes
       if (lane == 0) {
         if (it.kind == ITEM_GRAD && it.c > 0) {
-          const int target = SIGNALS_PER_ITEM * it.c * a.HN;
-          ok = wait_counter(a.x_row + it.a, target, abort_flag, a.timeout_ns) &&
-               wait_counter(a.w_col + 2 * it.b, target, abort_flag, a.timeout_ns) &&
-               wait_counter(a.w_col + 2 * it.b + 1, target, abort_flag, a.timeout_ns);
+          ok = wait_counter(a.x_row + it.a, SIGNALS_PER_ITEM * it.c * a.HN, abort_flag, a.timeout_ns) &&
+               wait_counter(a.w_col + it.b, SIGNALS_PER_ITEM * it.c * a.HN, abort_flag, a.timeout_ns);
         } else if (it.kind == ITEM_DX && it.c > 0) {
           ok = wait_counter(a.x_row + it.a, SIGNALS_PER_ITEM * it.c * a.HN, abort_flag, a.timeout_ns);
         }
@@ -1075,38 +1104,39 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         give_up();
         break;
       }
-      for (int j = 0; j < 2; ++j) {
-        if (!wait_half(p, j, eph, abort_flag, a.timeout_ns)) {
+      const bool got = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        give_up();
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
+      const bool skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
+      if (skip) {
+        // all rows ignored: nothing reads this tile's G rows; its dX rows are
+        // zero, written once by the first chunk
+        if (it.kind == ITEM_DX && it.c == 0) epi_zero_tile(taddr, row0, it.b, row_local, es, &m.Hio);
+      } else if (it.kind == ITEM_GRAD) {
+        epi_grad_tile(a, vbase, taddr, row0, it.b, row_local, es, &m.Go);
+      } else if (it.kind == ITEM_DW) {
+        if (any_valid)
+          epi_dw_tile(vbase, taddr, row0, it.b, row_local, es, &m.DWo);
+        else
+          epi_zero_tile(taddr, vbase + row0, it.b, row_local, es, &m.DWo);
+      } else {
+        epi_dx_tile(a, it.c == 0, it.c == a.C - 1, taddr, row0, it.b, row_local, es, &m.Hio, &m.Loo, dx_final,
+                    abort_flag, ok);
+        if (!ok) {
           give_up();
-          ok = false;
           break;
         }
-        const uint32_t taddr = tmem_base + lane_addr + j * SUBN;
-        const int col = it.b * BN + j * SUBN;
-        if (j == 0 || sh.two) {
-          if (sh.skip) {
-            // all rows ignored: nothing reads this tile's G rows; its dX rows are
-            // zero, written once by the first chunk
-            if (it.kind == ITEM_DX && it.c == 0) epi_zero_half(row0, col, row_local, es, &m.Hio);
-          } else if (it.kind == ITEM_GRAD) {
-            epi_grad_half(a, vbase, taddr, row0, col, row_local, es, &m.Go);
-          } else if (it.kind == ITEM_DW) {
-            if (any_valid)
-              epi_dw_half(taddr, vbase + row0, col, row_local, es, &m.DWo);
-            else
-              epi_zero_half(vbase + row0, col, row_local, es, &m.DWo);
-          } else {
-            epi_dx_half(a, it.c == 0, it.c == a.C - 1, taddr, row0, col, row_local, es, &m.Hio, &m.Loo, dx_final,
-                        abort_flag, ok);
-            if (!ok) {
-              give_up();
-              break;
-            }
-          }
-        }
-        release_half(tempty_leader[j], lane, j, eph);
       }
-      if (!ok) break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
       // this warp's boxes have landed: count the tile as done for its readers
       if (lane == 0) {
         bulk_wait<0>();
@@ -1123,7 +1153,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     }
     if (lane == 0) bulk_wait<0>();
   }
-  gemm_teardown(p, tmem_base, rank, warp, a.status, a.timeout_ns);
+
+  pair_wind_down(smem_u32(bars), tmem_slot, rank, warp, abort_flag, a.status, a.timeout_ns);
 }
 
 // ---------------------------------------------------------------- prep --

@@ -29,6 +29,7 @@ NUM_KERNEL_KINDS = 8
 
 EXPORTED = (
     "flce_status_string",
+    "flce_last_cuda_error",
     "flce_workspace_size",
     "flce_workspace_size_reorder",
     "flce_forward_backward",
@@ -58,7 +59,12 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 class FlceError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        msg = f"{where}: {STATUS_NAMES.get(status, status)}"
+        if status == 6 and _lib is not None:  # FLCE_ERR_CUDA: say which step failed and why
+            line, code, text = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_char_p()
+            _lib.flce_last_cuda_error(ctypes.byref(line), ctypes.byref(code), ctypes.byref(text))
+            msg += f" (library line {line.value}: CUDA error {code.value}, {(text.value or b'').decode()})"
+        super().__init__(msg)
 
 
 class PlanT(ctypes.Structure):
@@ -88,6 +94,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     fp = ctypes.POINTER(ctypes.c_float)
     lib.flce_status_string.argtypes = [ctypes.c_int]
     lib.flce_status_string.restype = ctypes.c_char_p
+    lib.flce_last_cuda_error.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_char_p)]
+    lib.flce_last_cuda_error.restype = None
     lib.flce_workspace_size.argtypes = [i64, i64, i64]
     lib.flce_workspace_size.restype = sz
     lib.flce_workspace_size_reorder.argtypes = [i64, i64]

@@ -12,11 +12,6 @@ points to an earlier item.  The dependencies:
 - a dW(c) mainloop waits for its G(c) column;
 - a G(c) epilogue waits for dX(c-1) of its token tile and dW(c-1) of its column.
 
-Tiles: a G tile is 256 token rows x 512 vocabulary entries, a dX tile 256
-token rows x 512 hidden columns and a dW tile 256 vocabulary rows x 512 hidden
-columns, so a dW tile reads half of one G column and a G tile overwrites what
-two dW tiles of the previous chunk read.
-
 This module restates the kernel's item decoder in Python (the G tiles of a
 chunk: the first `cols_first` vocabulary tiles column by column, the rest row
 by row) and checks both properties for the workload shapes, the small test
@@ -25,30 +20,23 @@ import itertools
 
 import pytest
 
-TM_ROWS = 256   # token rows of a G or dX tile, vocabulary rows of a dW tile
-WIDE = 512      # columns of every tile
-VC = 2048       # vocabulary entries per chunk
+TILE = 256
+VC = 2048  # vocabulary entries per chunk
 
 
 def layout(N, H, V):
-    TM, HN, C = -(-N // TM_ROWS), -(-H // WIDE), -(-V // VC)
-    v_last = V - (C - 1) * VC
-    VT_last, VM_last = -(-v_last // WIDE), -(-v_last // TM_ROWS)
-    VTf = VC // WIDE if C > 1 else VT_last
-    VMf = VC // TM_ROWS if C > 1 else VM_last
-    return dict(TM=TM, HN=HN, C=C, VTf=VTf, VT_last=VT_last, VMf=VMf, VM_last=VM_last)
+    TM, HN, C = -(-N // TILE), -(-H // TILE), -(-V // VC)
+    VT_last = -(-(V - (C - 1) * VC) // TILE)
+    VTf = VC // TILE if C > 1 else VT_last
+    return dict(TM=TM, HN=HN, C=C, VTf=VTf, VT_last=VT_last)
 
 
 def vtiles(p, c):
     return p["VT_last"] if c == p["C"] - 1 else p["VTf"]
 
 
-def vmtiles(p, c):
-    return p["VM_last"] if c == p["C"] - 1 else p["VMf"]
-
-
 def section_size(p, c):
-    n = p["TM"] * p["HN"] + vmtiles(p, c) * p["HN"]
+    n = p["TM"] * p["HN"] + vtiles(p, c) * p["HN"]
     if c + 1 < p["C"]:
         n += vtiles(p, c + 1) * p["TM"]
     return n
@@ -76,7 +64,7 @@ def decode(p, i, cols_first):
     while c + 1 < p["C"] and r >= section_size(p, c):
         r -= section_size(p, c)
         c += 1
-    nx, nw = p["TM"] * p["HN"], vmtiles(p, c) * p["HN"]
+    nx, nw = p["TM"] * p["HN"], vtiles(p, c) * p["HN"]
     if r < nx:
         return ("X", c, r // p["HN"], r % p["HN"])
     if r < nx + nw:
@@ -92,7 +80,7 @@ def every_tile(p):
             out.add(("G", c, t, v))
         for t, h in itertools.product(range(p["TM"]), range(p["HN"])):
             out.add(("X", c, t, h))
-        for v, h in itertools.product(range(vmtiles(p, c)), range(p["HN"])):
+        for v, h in itertools.product(range(vtiles(p, c)), range(p["HN"])):
             out.add(("W", c, v, h))
     return out
 
@@ -103,11 +91,10 @@ def dependencies(p, item):
         deps = [("G", c, a, v) for v in range(vtiles(p, c))]
         return deps + ([("X", c - 1, a, h) for h in range(p["HN"])] if c else [])
     if k == "W":
-        return [("G", c, t, a // 2) for t in range(p["TM"])]
+        return [("G", c, t, a) for t in range(p["TM"])]
     if c == 0:
         return []
-    return [("X", c - 1, a, h) for h in range(p["HN"])] + [
-        ("W", c - 1, v, h) for v in (2 * b, 2 * b + 1) if v < vmtiles(p, c - 1) for h in range(p["HN"])]
+    return [("X", c - 1, a, h) for h in range(p["HN"])] + [("W", c - 1, b, h) for h in range(p["HN"])]
 
 
 def rows_first(p, pairs=74):
@@ -137,24 +124,14 @@ def test_queue_holds_every_tile_once_and_dependencies_point_back(shape, cols_fir
 
 
 def test_row_order_of_the_workloads():
-    """Row by row up to three rounds of the 74 pairs: the Gemma-like workload
-    (16 token tiles x 4 vocabulary tiles = 64 G tiles a chunk), the Llama head
-    (32 x 4) and N up to 55 token tiles; long context and Phi-3 go column by
-    column."""
-    for shape in [(4096, 2304, 256000), (8192, 4096, 128256), (14080, 4096, 128256)]:
-        assert rows_first(layout(*shape)), shape
-    for shape in [(14336, 4096, 128256), (16384, 4096, 128256), (32768, 3072, 32064)]:
-        assert not rows_first(layout(*shape)), shape
-
-
-def test_gradient_tiles_cover_the_chunk_columns_dw_reads():
-    """Every dW tile's rows lie inside one G column, and the two dW tiles a G
-    column holds are the ones its next G tile waits for."""
-    for shape in SHAPES:
-        p = layout(*shape)
-        for c in range(p["C"]):
-            assert vmtiles(p, c) <= 2 * vtiles(p, c)
-            assert -(-vmtiles(p, c) // 2) == vtiles(p, c)
+    """Row by row below three rounds of the 74 pairs: the Gemma-like workload
+    (16 token tiles x 8 vocabulary tiles = 128 G tiles a chunk) and N up to
+    27 token tiles; the Llama head, long context and Phi-3 go column by column."""
+    assert rows_first(layout(4096, 2304, 256000))
+    assert rows_first(layout(6912, 4096, 128256))
+    assert not rows_first(layout(7168, 4096, 128256))
+    for shape in [(8192, 4096, 128256), (16384, 4096, 128256), (32768, 3072, 32064)]:
+        assert not rows_first(layout(*shape))
 
 
 def test_row_order_completes_token_rows_early():
