@@ -144,10 +144,10 @@ flce_status_t flce_forward_backward_async(const uint16_t* X, const uint16_t* W, 
  *   same shapes (workspace >= flce_workspace_size bytes)
  * Copies the inputs to the device, runs the computation, copies loss, dX and
  * dW back, and waits for the stream.  No allocation happens inside.  The
- * copies overlap the kernels: W goes over in pieces on an internal copy stream
- * and pass 1 runs piece by piece as they land; pass 2 runs in sections of
- * whole vocabulary chunks and each section's finished dW rows come back while
- * the next one computes.  Results agree with flce_forward_backward's to
+ * copies overlap the kernels: W goes over in up to 16 pieces on an internal
+ * copy stream and pass 1 runs piece by piece as they land; pass 2 runs in up
+ * to 16 sections of whole vocabulary chunks, the last one a single chunk, and
+ * each section's finished dW rows come back while the next one computes.  Results agree with flce_forward_backward's to
  * rounding (the log-sum-exp partials are merged in another order).  The copy
  * stream and its events are made on first use, one set per device, and kept;
  * host-buffer calls on one device run one at a time. */
@@ -163,7 +163,9 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
  * Enqueues the mean-reduced call of flce_forward_backward_ex (d_mean_count:
  * DEVICE int32 or NULL, as there) with the gradient pass split into
  * `sections` launches over consecutive ranges of vocabulary chunks (1 ..
- * 8; at most one per 2048-entry chunk).  After section k the call records
+ * 16; at most one per 2048-entry chunk; with several, the last section is
+ * the last chunk alone, so that little is left to reduce after the last
+ * launch).  After section k the call records
  * section_done[k] (caller-created CUDA events) on `stream`; from then on dW rows
  * [section_rows[k], section_rows[k+1]) are final, so the caller can start
  * reducing them over the data-parallel ranks on another stream (e.g. an NCCL

@@ -314,7 +314,7 @@ flce_status_t check_args(const void* X, const void* W, const void* y, int64_t N,
 // runs as a few launches over consecutive chunk sections of its item queue,
 // and each section's finished dW rows go back on the copy stream while the
 // next section computes.
-constexpr int MAX_PIECES = 8;
+constexpr int MAX_PIECES = 16;
 struct PipeCtx {
   cudaStream_t copy = nullptr;
   int pieces = 0;                      // W pieces = pass-1 launches
@@ -604,17 +604,25 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     // one launch over the whole queue; a host-buffer call splits it into
     // sections of whole chunks and sends each section's dW rows back
     const int groups = opt.pipe ? std::max(1, std::min(opt.pipe->groups, b.C)) : 1;
+    // Sections of whole chunks; with several, the last one is a single chunk,
+    // so that little of dW is left to copy or reduce after the last launch.
+    auto section_chunk = [&](int k) {  // first chunk of section k (k = groups: the end)
+      if (groups == 1 || k == groups) return k == groups ? b.C : 0;
+      return static_cast<int>(static_cast<long long>(k) * (b.C - 1) / (groups - 1));
+    };
     size_t slot;
     for (int k = 0; k < groups; ++k) {
-      const int c0 = static_cast<int>(static_cast<long long>(k) * b.C / groups);
-      const int c1 = static_cast<int>(static_cast<long long>(k + 1) * b.C / groups);
+      const int c0 = section_chunk(k);
+      const int c1 = section_chunk(k + 1);
       b.item_begin = k == 0 ? 0 : section_end[c0 - 1];
       b.item_end = section_end[c1 - 1];
       const int grid = static_cast<int>(std::min<long long>(b.item_end - b.item_begin, P.clusters));
-      prof_begin(stream, KIND_PASS2, &slot);
-      flce_pass2_kernel<<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, stream>>>(pm, b);
-      prof_end(stream, slot);
-      if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
+      if (grid > 0) {
+        prof_begin(stream, KIND_PASS2, &slot);
+        flce_pass2_kernel<<<CLUSTER * grid, NUM_THREADS, SMEM_BYTES, stream>>>(pm, b);
+        prof_end(stream, slot);
+        if (cudaGetLastError() != cudaSuccess) return cuda_fail(__LINE__);
+      }
       if (opt.pipe) {  // dW rows of chunks c0 .. c1-1 are final
         const PipeCtx& pp = *opt.pipe;
         const int64_t r0 = static_cast<int64_t>(c0) * VC, r1 = std::min<int64_t>(V, static_cast<int64_t>(c1) * VC);
