@@ -21,6 +21,9 @@ using namespace flce;
 // Vocabulary entries per pass-2 chunk.  The G chunk buffer is N x VC bf16, so
 // the workspace stays independent of V.
 constexpr int VC = 2048;
+// Active k-blocks a paired dW item runs on its first half before it needs the
+// second buffer: about one dX epilogue's time on the previous item.
+constexpr int DW_LEAD = 16;
 constexpr int MAX_SPLITS = 64;
 constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per bounded wait
 
@@ -564,23 +567,28 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     GemmArgs b = a;
     b.TM = P.tiles_m;
     b.HN = static_cast<int>((H + BN - 1) / BN);
+    b.dw_lead = DW_LEAD;
     b.C = P.num_chunks;
     b.VTf = VC / BN;
     b.VT_last = static_cast<int>((V - static_cast<int64_t>(P.num_chunks - 1) * VC + BN - 1) / BN);
     if (b.C == 1) b.VTf = b.VT_last;
+    // G tiles column by column when a chunk holds more than three rounds of
+    // them for the SM pairs, else row by row (see the queue's description)
+    b.g_cols_first = static_cast<long long>(b.TM) * b.VTf > 3ll * P.clusters ? b.VTf : 0;
+    // dW items pair adjacent hidden tiles (256 x 512 in both accumulator
+    // buffers) in the same regime; with fewer rounds a chunk's items are on the
+    // critical path of the next chunk's G epilogues, and longer items only delay it
+    b.HW = b.g_cols_first ? (b.HN + 1) / 2 : b.HN;
     // section_end[c]: end of the queue's section c (dX(c) dW(c) G(c+1)), after G(0)
     std::vector<long long> section_end(b.C);
     long long total = static_cast<long long>(b.C == 1 ? b.VT_last : b.VTf) * b.TM;  // G(0)
     for (int c = 0; c < b.C; ++c) {
       const long long vt = c == b.C - 1 ? b.VT_last : b.VTf;
-      total += static_cast<long long>(b.TM) * b.HN + vt * b.HN;
+      total += static_cast<long long>(b.TM) * b.HN + vt * b.HW;
       if (c + 1 < b.C) total += static_cast<long long>(c + 1 == b.C - 1 ? b.VT_last : b.VTf) * b.TM;
       section_end[c] = total;
     }
     b.total_items = total;
-    // G tiles column by column when a chunk holds more than three rounds of
-    // them for the SM pairs, else row by row (see the queue's description)
-    b.g_cols_first = static_cast<long long>(b.TM) * b.VTf > 3ll * P.clusters ? b.VTf : 0;
     int* ctr = reinterpret_cast<int*>(ws + L.counters);
     b.g_row = ctr;
     b.x_row = ctr + b.TM;

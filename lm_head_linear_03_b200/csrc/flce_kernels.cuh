@@ -138,6 +138,8 @@ struct GemmArgs {
   const int* reordered;          // device word: 1 when the rows are reordered
   // pass 2 (one persistent launch over every chunk)
   int TM, HN;             // 256-row token tiles, 256-column hidden tiles
+  int HW;                 // dW items per vocabulary tile: hidden tiles in pairs, the last alone when HN is odd
+  int dw_lead;            // active k-blocks a paired dW item runs on its first half alone (see the issuer)
   int C;                  // vocabulary chunks
   int VTf, VT_last;       // 256-wide vocabulary tiles in a full / the last chunk
   long long total_items;
@@ -760,19 +762,30 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
 //   G(c)  epilogue  after dX(c-1) of its token tile and dW(c-1) of its column.
 // Every dependency points to an earlier item and all SM pairs are resident at
 // once, so the queue always drains.  Completion is counted per token tile /
-// column in monotonic counters: each epilogue warp adds one after its TMA
-// stores have landed, so a finished item adds EPI_WARPS * CLUSTER.
+// column in monotonic counters: each epilogue warp adds one per 256x256 tile
+// after its TMA stores have landed, so a finished tile adds EPI_WARPS * CLUSTER.
+//
+// A dW item covers two adjacent 256-column hidden tiles (the last one alone
+// when the hidden tiles are odd in number): a 256 x 512 tile in both halves of
+// the tensor memory, which reads its G^T operand once for both halves.  Its
+// K = tokens contraction is long and its epilogue short, so the loss of the
+// accumulator double buffer is confined to its two ends (see the issuer).
 
 enum : int { ITEM_GRAD = 0, ITEM_DW = 1, ITEM_DX = 2 };
 
 struct Item {
-  int kind, c, a, b;  // G: (tm, vb)  dW: (vm, hn)  dX: (tm, hn)
+  int kind, c, a, b;  // G: (tm, vb)  dW: (vm, hidden tile pair)  dX: (tm, hn)
 };
+
+// A dW item with two hidden tiles (2b and 2b+1)?
+__device__ __forceinline__ bool dw_paired(const GemmArgs& p, const Item& it) {
+  return p.HW < p.HN && 2 * it.b + 1 < p.HN;
+}
 
 __device__ __forceinline__ int chunk_vtiles(const GemmArgs& p, int c) { return c == p.C - 1 ? p.VT_last : p.VTf; }
 
 __device__ __forceinline__ long long section_size(const GemmArgs& p, int c) {
-  long long n = static_cast<long long>(p.TM) * p.HN + static_cast<long long>(chunk_vtiles(p, c)) * p.HN;
+  long long n = static_cast<long long>(p.TM) * p.HN + static_cast<long long>(chunk_vtiles(p, c)) * p.HW;
   if (c + 1 < p.C) n += static_cast<long long>(chunk_vtiles(p, c + 1)) * p.TM;
   return n;
 }
@@ -817,7 +830,7 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
     ++c;
   }
   const long long nx = static_cast<long long>(p.TM) * p.HN;
-  const long long nw = static_cast<long long>(chunk_vtiles(p, c)) * p.HN;
+  const long long nw = static_cast<long long>(chunk_vtiles(p, c)) * p.HW;
   it.c = c;
   if (r < nx) {
     it.kind = ITEM_DX;
@@ -826,8 +839,8 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
   } else if (r < nx + nw) {
     r -= nx;
     it.kind = ITEM_DW;
-    it.a = static_cast<int>(r / p.HN);
-    it.b = static_cast<int>(r - static_cast<long long>(it.a) * p.HN);
+    it.a = static_cast<int>(r / p.HW);
+    it.b = static_cast<int>(r - static_cast<long long>(it.a) * p.HW);
   } else {
     r -= nx + nw;
     it.kind = ITEM_GRAD;
@@ -835,6 +848,26 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& p, long long i) {
     grad_tile(p, c + 1, r, it);
   }
   return it;
+}
+
+// First 256-column hidden tile of a dW item.
+__device__ __forceinline__ int dw_first_tile(const GemmArgs& p, const Item& it) {
+  return p.HW < p.HN ? 2 * it.b : it.b;
+}
+
+// A paired dW item runs its first `lead` active k-blocks on the first half
+// alone and the same k-blocks on the second half last (see the issuer).  The
+// k-blocks over token tiles whose rows are all ignored are not active.  Returns
+// the raw k-block index just past the lead, with lead = min(dw_lead, active/2).
+__device__ __forceinline__ int dw_lead_end(const GemmArgs& a) {
+  const int kblocks = (a.N + BK - 1) / BK;
+  int active = 0;
+  for (int kb = 0; kb < kblocks; ++kb) active += a.tile_valid[kb / (CM / BK)] != 0 ? 1 : 0;
+  const int lead = min(a.dw_lead, active / 2);
+  int cnt = 0;
+  for (int kb = 0; kb < kblocks && cnt < lead; ++kb)
+    if (a.tile_valid[kb / (CM / BK)] != 0 && ++cnt == lead) return kb + 1;
+  return 0;
 }
 
 constexpr int SIGNALS_PER_ITEM = EPI_WARPS * CLUSTER;
@@ -926,6 +959,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       uint32_t phase = 0;
       long long filled = 0;
       bool ok = true;
+      const int dw_lead = dw_lead_end(a);
       for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
         const Item it = decode_item(a, u);
         const int vbase = it.c * a.Vc;
@@ -959,7 +993,42 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         // acquire above before those reads (G tiles read only X and W)
         if (it.kind != ITEM_GRAD) fence_proxy_async_global();
         const int m0 = it.a * CM + rank * BM;
-        const int n0 = it.b * BN + rank * BNH;
+        const int n0 = (it.kind == ITEM_DW ? dw_first_tile(a, it) : it.b) * BN + rank * BNH;
+        if (it.kind == ITEM_DW && dw_paired(a, it)) {
+          // one ring position: G^T (unless with_a is false) and the X columns from n
+          auto fill_dw = [&](int kb, bool with_a, int n) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
+              give_up();
+              return false;
+            }
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * (with_a ? STAGE_BYTES : B_TILE_BYTES));
+            const uint32_t bar = mapa_shared(full_bar(stage), 0);
+            const int k0 = kb * BK;
+            if (with_a) {
+#pragma unroll
+              for (int i = 0; i < BM / 64; ++i)
+                tma_load_2d_pair(sA(stage) + i * MN_BOX_BYTES, &m.Gmn, bar, m0 + i * 64, k0, normal);
+            }
+#pragma unroll
+            for (int i = 0; i < BNH / 64; ++i)
+              tma_load_2d_pair(sB(stage) + i * MN_BOX_BYTES, mXmn, bar, n + i * 64, k0, keep);
+            ++filled;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            return true;
+          };
+          // lead: first half alone; middle: both halves (two positions, G^T
+          // once); tail: second half alone over the lead's k-blocks
+          for (int kb = 0; ok && kb < dw_lead; ++kb)
+            if (a.tile_valid[kb / (CM / BK)] != 0) ok = fill_dw(kb, true, n0);
+          for (int kb = dw_lead; ok && kb < kblocks; ++kb)
+            if (a.tile_valid[kb / (CM / BK)] != 0) ok = fill_dw(kb, true, n0) && fill_dw(kb, false, n0 + BN);
+          for (int kb = 0; ok && kb < dw_lead; ++kb)
+            if (a.tile_valid[kb / (CM / BK)] != 0) ok = fill_dw(kb, true, n0 + BN);
+          continue;
+        }
         for (int kb = 0; kb < kblocks; ++kb) {
           // dW: K runs over tokens; k-blocks of all-ignored token tiles add nothing
           if (it.kind == ITEM_DW && a.tile_valid[kb / (CM / BK)] == 0) continue;
@@ -1005,11 +1074,96 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       int stage = 0;
       uint32_t phase = 0;
       long long consumed = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
+      int acc = 0;          // accumulator buffer of the next item
+      uint32_t tph = 0;     // bit b: phase of buffer b's tempty barrier (one flip per use)
       bool ok = true;
+      const int dw_lead = dw_lead_end(a);
+      auto take = [&]() {  // wait for the next ring position to fill
+        if (!mbar_wait(full_bar(stage), phase, abort_flag, a.timeout_ns)) {
+          give_up();
+          return -1;
+        }
+        ++consumed;
+        tc_fence_after();
+        const int s = stage;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return s;
+      };
+      auto mma_dw = [&](uint32_t d, int sa, int sb, uint32_t& accumulate) {
+#pragma unroll
+        for (int k = 0; k < BK / UMMA_K; ++k) {
+          umma_bf16_pair(d, operand_desc<true>(sA(sa), k), operand_desc<true>(sB(sb), k), ID_DW, accumulate);
+          accumulate = 1;
+        }
+      };
       for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
         const Item it = decode_item(a, u);
+        if (it.kind == ITEM_DW && dw_paired(a, it)) {
+          // 256 x 512: the first half in buffer p (the next in turn), the
+          // second in q, which the previous item's epilogue may still be
+          // reading.  The lead's k-blocks run on p alone meanwhile, and the
+          // same k-blocks run on q alone at the end, after p is committed, so
+          // that the epilogue drains p while q finishes; the next item then
+          // takes p again.
+          const int p = acc, q = acc ^ 1;
+          const int kblocks = (a.N + BK - 1) / BK;
+          uint32_t acc_p = 0, acc_q = 0;
+          if (!mbar_wait<true>(tempty_bar(p), ((tph >> p) & 1u) ^ 1u, abort_flag, a.timeout_ns)) {
+            give_up();
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dp = tmem_base + p * ACC_COLS, dq = tmem_base + q * ACC_COLS;
+          for (int kb = 0; ok && kb < dw_lead; ++kb) {
+            if (a.tile_valid[kb / (CM / BK)] == 0) continue;
+            const int s1 = take();
+            if (s1 < 0) {
+              ok = false;
+              break;
+            }
+            mma_dw(dp, s1, s1, acc_p);
+            umma_commit_pair(empty_bar(s1), 0x3);
+          }
+          if (!ok) break;
+          if (!mbar_wait<true>(tempty_bar(q), ((tph >> q) & 1u) ^ 1u, abort_flag, a.timeout_ns)) {
+            give_up();
+            break;
+          }
+          tc_fence_after();
+          for (int kb = dw_lead; ok && kb < kblocks; ++kb) {
+            if (a.tile_valid[kb / (CM / BK)] == 0) continue;
+            const int s1 = take();
+            const int s2 = s1 < 0 ? -1 : take();
+            if (s2 < 0) {
+              ok = false;
+              break;
+            }
+            mma_dw(dp, s1, s1, acc_p);
+            mma_dw(dq, s1, s2, acc_q);
+            umma_commit_pair(empty_bar(s1), 0x3);
+            umma_commit_pair(empty_bar(s2), 0x3);
+          }
+          if (!ok) break;
+          umma_commit_pair(tfull_bar(p), 0x3);
+          tph ^= 1u << p;
+          for (int kb = 0; ok && kb < dw_lead; ++kb) {
+            if (a.tile_valid[kb / (CM / BK)] == 0) continue;
+            const int s1 = take();
+            if (s1 < 0) {
+              ok = false;
+              break;
+            }
+            mma_dw(dq, s1, s1, acc_q);
+            umma_commit_pair(empty_bar(s1), 0x3);
+          }
+          if (!ok) break;
+          umma_commit_pair(tfull_bar(q), 0x3);
+          tph ^= 1u << q;
+          continue;
+        }
         const int vcount = min(a.Vc, a.V - it.c * a.Vc);
         const bool skip = it.kind != ITEM_DW && a.tile_valid[it.a] == 0;
         const int kblocks = skip                  ? 0
@@ -1019,7 +1173,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         const uint32_t idesc = it.kind == ITEM_GRAD ? ID_GRAD : it.kind == ITEM_DW ? ID_DW : ID_DX;
         const bool a_mn = it.kind == ITEM_DW;
         const bool b_mn = it.kind != ITEM_GRAD;
-        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+        if (!mbar_wait<true>(tempty_bar(acc), ((tph >> acc) & 1u) ^ 1u, abort_flag, a.timeout_ns)) {
           give_up();
           break;
         }
@@ -1050,16 +1204,14 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         }
         if (!ok) break;
         umma_commit_pair(tfull_bar(acc), 0x3);
+        tph ^= 1u << acc;
         acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
       }
-      for (int i = 0; i < 2; ++i) {
-        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+      for (int b = 0; b < 2; ++b) {
+        if (!mbar_wait<true>(tempty_bar(b), ((tph >> b) & 1u) ^ 1u, abort_flag, a.timeout_ns)) {
           give_up();
           break;
         }
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
       }
       // the positions consumed, and one last commit that completes when every UMMA has
       tmem_slot[3] = static_cast<uint32_t>(consumed);
@@ -1082,8 +1234,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     // with every token ignored the dW contraction has no k-block at all
     bool any_valid = false;
     for (int t = 0; t < a.TM && !any_valid; ++t) any_valid = a.tile_valid[t] != 0;
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    int acc = 0;       // accumulator buffer of the next item (the issuer's sequence)
+    uint32_t eph = 0;  // bit b: phase of buffer b's tfull barrier (one flip per use)
     bool ok = true;
     for (long long u = a.item_begin + cid; ok && u < a.item_end; u += ncl) {
       const Item it = decode_item(a, u);
@@ -1104,7 +1256,38 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         give_up();
         break;
       }
-      const bool got = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.timeout_ns);
+      if (it.kind == ITEM_DW && dw_paired(a, it)) {
+        // a paired dW item: its first half in buffer acc, its second in acc ^ 1;
+        // the next item takes acc again, the buffer freed first
+        for (int h = 0; h < 2; ++h) {
+          const int buf = acc ^ h;
+          const bool got = mbar_wait(tfull_bar(buf), (eph >> buf) & 1u, abort_flag, a.timeout_ns);
+          if (!__all_sync(0xffffffffu, got)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + lane_addr + buf * ACC_COLS;
+          const int nt = dw_first_tile(a, it) + h;
+          if (any_valid)
+            epi_dw_tile(vbase, taddr, row0, nt, row_local, es, &m.DWo);
+          else
+            epi_zero_tile(taddr, vbase + row0, nt, row_local, es, &m.DWo);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(buf == 0 ? tempty_leader0 : tempty_leader1);
+          eph ^= 1u << buf;
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          bulk_wait<0>();
+          fence_proxy_async_global();
+          red_release_gpu_add(a.w_col + it.a, 2);
+        }
+        continue;
+      }
+      const bool got = mbar_wait(tfull_bar(acc), (eph >> acc) & 1u, abort_flag, a.timeout_ns);
       if (!__all_sync(0xffffffffu, got)) {
         give_up();
         ok = false;
@@ -1120,10 +1303,11 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       } else if (it.kind == ITEM_GRAD) {
         epi_grad_tile(a, vbase, taddr, row0, it.b, row_local, es, &m.Go);
       } else if (it.kind == ITEM_DW) {
+        const int nt = dw_first_tile(a, it);
         if (any_valid)
-          epi_dw_tile(vbase, taddr, row0, it.b, row_local, es, &m.DWo);
+          epi_dw_tile(vbase, taddr, row0, nt, row_local, es, &m.DWo);
         else
-          epi_zero_tile(taddr, vbase + row0, it.b, row_local, es, &m.DWo);
+          epi_zero_tile(taddr, vbase + row0, nt, row_local, es, &m.DWo);
       } else {
         epi_dx_tile(a, it.c == 0, it.c == a.C - 1, taddr, row0, it.b, row_local, es, &m.Hio, &m.Loo, dx_final,
                     abort_flag, ok);
@@ -1135,8 +1319,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+      eph ^= 1u << acc;
       acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
       // this warp's boxes have landed: count the tile as done for its readers
       if (lane == 0) {
         bulk_wait<0>();

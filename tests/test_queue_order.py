@@ -5,8 +5,10 @@ to the SM pairs:
 
     G(0) | dX(0) dW(0) G(1) | dX(1) dW(1) G(2) | ... | dX(C-1) dW(C-1)
 
-It drains only if every tile appears exactly once and every dependency
-points to an earlier item.  The dependencies:
+A dW item covers two adjacent 256-column hidden tiles (the last one alone
+when their number is odd).  The queue drains only if every tile appears
+exactly once and every dependency points to an earlier item.  The
+dependencies:
 - a dX(c) mainloop waits for its token tile's G(c) row;
 - a dX(c) epilogue waits for dX(c-1) of its token tile;
 - a dW(c) mainloop waits for its G(c) column;
@@ -28,7 +30,14 @@ def layout(N, H, V):
     TM, HN, C = -(-N // TILE), -(-H // TILE), -(-V // VC)
     VT_last = -(-(V - (C - 1) * VC) // TILE)
     VTf = VC // TILE if C > 1 else VT_last
-    return dict(TM=TM, HN=HN, C=C, VTf=VTf, VT_last=VT_last)
+    return dict(TM=TM, HN=HN, HW=(HN + 1) // 2, C=C, VTf=VTf, VT_last=VT_last)
+
+
+def dw_tiles(p, b):
+    """Hidden tiles of dW item b: a pair, or the last tile alone."""
+    if p["HW"] == p["HN"]:
+        return (b,)
+    return (2 * b, 2 * b + 1) if 2 * b + 1 < p["HN"] else (2 * b,)
 
 
 def vtiles(p, c):
@@ -36,7 +45,7 @@ def vtiles(p, c):
 
 
 def section_size(p, c):
-    n = p["TM"] * p["HN"] + vtiles(p, c) * p["HN"]
+    n = p["TM"] * p["HN"] + vtiles(p, c) * p["HW"]
     if c + 1 < p["C"]:
         n += vtiles(p, c + 1) * p["TM"]
     return n
@@ -64,12 +73,12 @@ def decode(p, i, cols_first):
     while c + 1 < p["C"] and r >= section_size(p, c):
         r -= section_size(p, c)
         c += 1
-    nx, nw = p["TM"] * p["HN"], vtiles(p, c) * p["HN"]
+    nx, nw = p["TM"] * p["HN"], vtiles(p, c) * p["HW"]
     if r < nx:
         return ("X", c, r // p["HN"], r % p["HN"])
     if r < nx + nw:
         r -= nx
-        return ("W", c, r // p["HN"], r % p["HN"])
+        return ("W", c, r // p["HW"], r % p["HW"])
     return ("G", c + 1) + grad_tile(p, c + 1, r - nx - nw, cols_first)
 
 
@@ -80,8 +89,8 @@ def every_tile(p):
             out.add(("G", c, t, v))
         for t, h in itertools.product(range(p["TM"]), range(p["HN"])):
             out.add(("X", c, t, h))
-        for v, h in itertools.product(range(vtiles(p, c)), range(p["HN"])):
-            out.add(("W", c, v, h))
+        for v, w in itertools.product(range(vtiles(p, c)), range(p["HW"])):
+            out.add(("W", c, v, w))
     return out
 
 
@@ -94,7 +103,7 @@ def dependencies(p, item):
         return [("G", c, t, a) for t in range(p["TM"])]
     if c == 0:
         return []
-    return [("X", c - 1, a, h) for h in range(p["HN"])] + [("W", c - 1, b, h) for h in range(p["HN"])]
+    return [("X", c - 1, a, h) for h in range(p["HN"])] + [("W", c - 1, b, w) for w in range(p["HW"])]
 
 
 def rows_first(p, pairs=74):
@@ -149,3 +158,13 @@ def test_row_order_completes_token_rows_early():
         t, _ = grad_tile(p, 1, r, 1 << 20)
         last[t] = r
     assert min(last.values()) == (p["VTf"] - 1) * p["TM"]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_dw_items_cover_every_hidden_tile_once(shape):
+    """The dW items of a vocabulary tile pair the hidden tiles 2b and 2b+1; an
+    odd last tile goes alone, and one hidden tile means no pair."""
+    p = layout(*shape)
+    tiles = [t for b in range(p["HW"]) for t in dw_tiles(p, b)]
+    assert tiles == list(range(p["HN"]))
+    assert sum(len(dw_tiles(p, b)) == 2 for b in range(p["HW"])) == p["HN"] // 2
