@@ -226,7 +226,9 @@ struct Plan {
 };
 
 // Pass 1: pick the number of vocabulary splits whose units, dealt round-robin
-// to the persistent SM pairs, give the smallest largest per-pair tile count.
+// to the persistent SM pairs, give the smallest largest per-pair load.  A unit
+// walks its tiles in pairs (256 x 512), a pair costing about 1.6 lone tiles,
+// plus one tile's worth for its pipeline fill and partial write.
 int choose_splits(int tiles_m, int vtiles, int sms) {
   int best = 1;
   long long best_cost = LLONG_MAX;
@@ -239,7 +241,7 @@ int choose_splits(int tiles_m, int vtiles, int sms) {
     for (long long u = 0; u < units; ++u) {
       const long long s = u / tiles_m;
       const long long n = ((s + 1) * vtiles) / S - (s * vtiles) / S;
-      load[u % grid] += n + 1;  // +1: per-unit pipeline fill and partial write
+      load[u % grid] += 16 * (n / 2) + 10 * (n % 2) + 10;
     }
     const long long cost = *std::max_element(load.begin(), load.end());
     if (cost < best_cost) {

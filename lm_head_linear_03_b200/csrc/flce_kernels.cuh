@@ -72,10 +72,18 @@ constexpr int NUM_BARRIERS = BAR_DRAIN + 1;
 constexpr int SLOT_WORDS = 4;
 static_assert(NUM_BARRIERS * 8 + SLOT_WORDS * 4 <= 256, "barrier area");
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
-// Pass 1 stages nothing through shared memory in its epilogue and needs no
-// staging area (a seventh stage measured no faster).
-constexpr int P1_STAGES = STAGES;
-constexpr int P1_SMEM_BYTES = P1_STAGES * STAGE_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
+// Pass 1 takes adjacent vocabulary tiles in pairs, as one 256 x 512 tile in
+// both accumulator buffers: its stages hold this CTA's X tile and the W tiles
+// of both halves (48 KB), four of them in the same bytes as pass 2's six.  A
+// stage thus holds 1024 tensor-core cycles of work instead of 512, and the
+// loads in flight cover their latency.  Pass 1 stages nothing through shared
+// memory in its epilogue and needs no staging area.
+constexpr int P1_STAGES = 4;
+constexpr int P1_STAGE_BYTES = A_TILE_BYTES + 2 * B_TILE_BYTES;
+constexpr int P1_SMEM_BYTES = P1_STAGES * P1_STAGE_BYTES + 1024 /*alignment*/ + 256 /*barriers*/;
+static_assert(P1_STAGES <= STAGES, "pass 1 uses the first barriers of pass 2's layout");
+// k-blocks a tile pair runs on its first half alone (see the pass-1 issuer)
+constexpr int P1_LEAD = 8;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr double LN2 = 0.6931471805599453;
 
@@ -177,17 +185,6 @@ __device__ __forceinline__ void unit_range(const GemmArgs& a, int u, int& mb, in
   mb = u - split * a.tiles_m;
   nb_begin = static_cast<int>((static_cast<long long>(split) * a.tiles_n) / a.splits);
   nb_end = static_cast<int>((static_cast<long long>(split + 1) * a.tiles_n) / a.splits);
-}
-
-// Pass-1 TMA loads of one pipeline stage for the CTA of rank `rank` in the pair:
-// its 128 rows of X and its 128 rows of W, both K-major.  X is read again by
-// every vocabulary tile (keep it in L2); W streams through once.
-__device__ __forceinline__ void load_stage_pass1(const CUtensorMap* mX, const CUtensorMap* mW, uint32_t sA,
-                                                 uint32_t sB, uint32_t bar, int mb, int nb, int kb, int rank,
-                                                 uint64_t keep, uint64_t stream) {
-  const int k0 = kb * BK;
-  tma_load_2d_pair(sA, mX, bar, k0, mb * CM + rank * BM, keep);
-  tma_load_2d_pair(sB, mW, bar, k0, nb * BN + rank * BNH, stream);
 }
 
 template <bool MN>
@@ -471,6 +468,7 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk,
 //     reports; a fixed 100 us grace period covers that case.
 // Every wait here ends by completion or by its own time limit, not by the
 // abort flag.
+template <int NST>
 __device__ __forceinline__ void pair_wind_down(uint32_t bars, const uint32_t* slots, int rank, int warp,
                                                volatile int* abort_flag, int* status, unsigned long long timeout_ns) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -483,7 +481,7 @@ __device__ __forceinline__ void pair_wind_down(uint32_t bars, const uint32_t* sl
       const long long filled = slots[2], consumed = slots[3];
       bool all = true;
       for (long long q = consumed; q < filled; ++q)
-        all = mbar_wait(bar(static_cast<int>(q % STAGES)), static_cast<uint32_t>((q / STAGES) & 1), &never,
+        all = mbar_wait(bar(static_cast<int>(q % NST)), static_cast<uint32_t>((q / NST) & 1), &never,
                         1000000ull) && all;
       if (!all) {
         const uint64_t t0 = globaltimer_ns();
@@ -512,16 +510,17 @@ __device__ __forceinline__ void pair_wind_down(uint32_t bars, const uint32_t* sl
 // empty barriers, so none lands after the CTA has gone, and record how far it
 // filled the ring.  After a give-up the peer's producer (which cannot see the
 // leader's full barriers) lets copies in flight land for 100 us.
+template <int NST>
 __device__ __forceinline__ void producer_tail(uint32_t bars, uint32_t* slots, long long filled, int& stage,
                                               uint32_t& phase, volatile int* abort_flag,
                                               unsigned long long timeout_ns, int rank, int* status) {
   slots[2] = static_cast<uint32_t>(filled);
-  for (int i = 0; i < STAGES; ++i) {
+  for (int i = 0; i < NST; ++i) {
     if (!mbar_wait(bars + 8u * static_cast<uint32_t>(STAGES + stage), phase ^ 1u, abort_flag, timeout_ns)) {
       give_up_pair(abort_flag, rank, status);
       break;
     }
-    if (++stage == STAGES) {
+    if (++stage == NST) {
       stage = 0;
       phase ^= 1u;
     }
@@ -546,9 +545,9 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;  // swizzle atoms need 1024-B alignment
   uint8_t* base_ptr = smem_raw + (base - raw_addr);
-  constexpr int STAGES = P1_STAGES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + STAGES * STAGE_BYTES);
-  // barrier slots: full[STAGES], empty[STAGES], tfull[2], tempty[2], fin
+  // the ring of P1_STAGES stages, then the barriers (pass 2's layout; pass 1
+  // uses the first P1_STAGES full and empty barriers)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + P1_STAGES * P1_STAGE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -563,11 +562,12 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 + b); };
   const uint32_t fin_bar = smem_u32(bars + 2 * STAGES + 4);
-  auto sA = [&](int s) { return base + s * STAGE_BYTES; };
-  auto sB = [&](int s) { return base + s * STAGE_BYTES + A_TILE_BYTES; };
+  // stage s: this CTA's X tile, then the W tiles of the pair's halves 0 and 1
+  auto sA = [&](int s) { return base + s * P1_STAGE_BYTES; };
+  auto sB = [&](int s, int h) { return base + s * P1_STAGE_BYTES + A_TILE_BYTES + h * B_TILE_BYTES; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < P1_STAGES; ++s) {
       mbar_init(full_bar(s), 1);    // leader: its producer's arrive + both CTAs' bytes
       mbar_init(empty_bar(s), 1);   // the leader's UMMA commit, multicast to both
     }
@@ -606,29 +606,47 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       uint32_t phase = 0;
       long long filled = 0;
       bool ok = true;
+      // One stage: this CTA's X rows at k-block kb (read again by every
+      // vocabulary tile: kept in L2) and its W rows of tile nb + h for each
+      // half h in `halves` (bit h; W streams through once), all K-major.
+      auto fill = [&](int mb, int nb, int kb, int halves) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          return false;
+        }
+        const int nh = (halves & 1) + (halves >> 1);
+        if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * (A_TILE_BYTES + nh * B_TILE_BYTES));
+        const uint32_t bar = mapa_shared(full_bar(stage), 0);
+        tma_load_2d_pair(sA(stage), mX, bar, kb * BK, mb * CM + rank * BM, keep);
+        for (int h = 0; h < 2; ++h)
+          if ((halves >> h) & 1)
+            tma_load_2d_pair(sB(stage, h), &mapW, bar, kb * BK, (nb + h) * BN + rank * BNH, stream);
+        ++filled;
+        if (++stage == P1_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
+      const int le = min(P1_LEAD, a.k_blocks / 2);
       for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
         unit_range(a, u, mb, nb0, nb1, split);
         if (a.tile_valid[mb] == 0) continue;  // every row of the tile is ignored
-        for (int nb = nb0; ok && nb < nb1; ++nb) {
-          for (int kb = 0; kb < a.k_blocks; ++kb) {
-            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.timeout_ns)) {
-              give_up();
-              ok = false;
-              break;
-            }
-            if (leader) mbar_arrive_expect_tx(full_bar(stage), CLUSTER * STAGE_BYTES);
-            load_stage_pass1(mX, &mapW, sA(stage), sB(stage), mapa_shared(full_bar(stage), 0), mb, nb, kb, rank,
-                             keep, stream);
-            ++filled;
-            if (++stage == STAGES) {
-              stage = 0;
-              phase ^= 1u;
-            }
+        for (int nb = nb0; ok && nb < nb1;) {
+          if (nb + 1 < nb1) {  // tiles nb and nb + 1 as one 256 x 512 tile (see the issuer)
+            for (int kb = 0; ok && kb < le; ++kb) ok = fill(mb, nb, kb, 1);
+            for (int kb = le; ok && kb < a.k_blocks; ++kb) ok = fill(mb, nb, kb, 3);
+            for (int kb = 0; ok && kb < le; ++kb) ok = fill(mb, nb, kb, 2);
+            nb += 2;
+          } else {
+            for (int kb = 0; ok && kb < a.k_blocks; ++kb) ok = fill(mb, nb, kb, 1);
+            nb += 1;
           }
         }
       }
-      producer_tail(smem_u32(bars), tmem_slot, filled, stage, phase, abort_flag, a.timeout_ns, rank, a.status);
+      producer_tail<P1_STAGES>(smem_u32(bars), tmem_slot, filled, stage, phase, abort_flag, a.timeout_ns, rank,
+                               a.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ UMMA issuer (leader) --
@@ -637,55 +655,93 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       int stage = 0;
       uint32_t phase = 0;
       long long consumed = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
+      int acc = 0;       // accumulator buffer of the next tile
+      uint32_t tph = 0;  // bit b: phase of buffer b's tempty barrier (one flip per use)
       bool ok = true;
+      // One stage: the X tile times the W tile of each half h in `halves`
+      // into d[h]; f[h] says whether d[h] accumulates.
+      auto step = [&](int halves, uint32_t d0, uint32_t& f0, uint32_t d1, uint32_t& f1) {
+        if (!mbar_wait(full_bar(stage), phase, abort_flag, a.timeout_ns)) {
+          give_up();
+          return false;
+        }
+        ++consumed;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < BK / UMMA_K; ++k) {
+          const uint64_t ad = operand_desc<false>(sA(stage), k);
+          if (halves & 1) {
+            umma_bf16_pair(d0, ad, operand_desc<false>(sB(stage, 0), k), IDESC, f0);
+            f0 = 1;
+          }
+          if (halves & 2) {
+            umma_bf16_pair(d1, ad, operand_desc<false>(sB(stage, 1), k), IDESC, f1);
+            f1 = 1;
+          }
+        }
+        umma_commit_pair(empty_bar(stage), 0x3);
+        if (++stage == P1_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
+      auto acquire = [&](int b) {  // the epilogue has released buffer b
+        if (!mbar_wait<true>(tempty_bar(b), ((tph >> b) & 1u) ^ 1u, abort_flag, a.timeout_ns)) {
+          give_up();
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      const int le = min(P1_LEAD, a.k_blocks / 2);
       for (int u = cid; ok && u < a.num_units; u += ncl) {
         int mb, nb0, nb1, split;
         unit_range(a, u, mb, nb0, nb1, split);
         if (a.tile_valid[mb] == 0) continue;  // every row of the tile is ignored
-        for (int nb = nb0; ok && nb < nb1; ++nb) {
-          if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
-            give_up();
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-          for (int kb = 0; kb < a.k_blocks; ++kb) {
-            if (!mbar_wait(full_bar(stage), phase, abort_flag, a.timeout_ns)) {
-              give_up();
-              ok = false;
-              break;
+        for (int nb = nb0; ok && nb < nb1;) {
+          const int p = acc, q = acc ^ 1;
+          const uint32_t dp = tmem_base + p * ACC_COLS, dq = tmem_base + q * ACC_COLS;
+          uint32_t fp = 0, fq = 0;
+          ok = acquire(p);
+          if (ok && nb + 1 < nb1) {
+            // Tiles nb (buffer p) and nb + 1 (buffer q) share each X tile.
+            // q may still be in the epilogue of the previous tile: the lead's
+            // k-blocks run on p alone meanwhile, and the same k-blocks run on
+            // q alone at the end, after p is committed, so that the epilogue
+            // folds tile nb while tile nb + 1 finishes.  The next tile takes
+            // p again.
+            for (int kb = 0; ok && kb < le; ++kb) ok = step(1, dp, fp, dq, fq);
+            ok = ok && acquire(q);
+            for (int kb = le; ok && kb < a.k_blocks; ++kb) ok = step(3, dp, fp, dq, fq);
+            if (ok) {
+              umma_commit_pair(tfull_bar(p), 0x3);
+              tph ^= 1u << p;
             }
-            ++consumed;
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < BK / UMMA_K; ++k)
-              umma_bf16_pair(d_tmem, operand_desc<false>(sA(stage), k), operand_desc<false>(sB(stage), k), IDESC,
-                             (kb | k) != 0);
-            umma_commit_pair(empty_bar(stage), 0x3);
-            if (++stage == STAGES) {
-              stage = 0;
-              phase ^= 1u;
+            for (int kb = 0; ok && kb < le; ++kb) ok = step(2, dp, fp, dq, fq);
+            if (ok) {
+              umma_commit_pair(tfull_bar(q), 0x3);
+              tph ^= 1u << q;
             }
+            nb += 2;
+          } else if (ok) {
+            for (int kb = 0; ok && kb < a.k_blocks; ++kb) ok = step(1, dp, fp, dq, fq);
+            if (ok) {
+              umma_commit_pair(tfull_bar(p), 0x3);
+              tph ^= 1u << p;
+            }
+            acc ^= 1;
+            nb += 1;
           }
-          if (!ok) break;
-          umma_commit_pair(tfull_bar(acc), 0x3);
-          acc ^= 1;
-          if (acc == 0) acc_phase ^= 1u;
         }
       }
       // Tail: both accumulators released by the epilogues of both CTAs, so all
       // UMMAs are done and no remote arrive is still on its way here.
-      for (int i = 0; i < 2; ++i) {
-        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+      for (int b = 0; b < 2; ++b)
+        if (!mbar_wait<true>(tempty_bar(b), ((tph >> b) & 1u) ^ 1u, abort_flag, a.timeout_ns)) {
           give_up();
           break;
         }
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      }
       // the positions consumed, and one last commit that completes when every UMMA has
       tmem_slot[3] = static_cast<uint32_t>(consumed);
       umma_commit_pair(smem_u32(bars + BAR_DRAIN), 0x3);
@@ -697,8 +753,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
     const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    int acc = 0;       // accumulator buffer of the next tile (the issuer's sequence)
+    uint32_t eph = 0;  // bit b: phase of buffer b's tfull barrier (one flip per use)
     bool ok = true;
     for (int u = cid; ok && u < a.num_units; u += ncl) {
       int mb, nb0, nb1, split;
@@ -714,20 +770,24 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
       st.zy_val = 0.f;
       st.has_zy = false;
       for (int nb = nb0; nb < nb1; ++nb) {
-        const bool got = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.timeout_ns);
+        // a pair of tiles (nb, nb + 1) sits in buffers acc and acc ^ 1, and the
+        // tile after it in acc again (the issuer's sequence)
+        const bool second = ((nb - nb0) & 1) != 0;
+        const int buf = second ? acc ^ 1 : acc;
+        const bool got = mbar_wait(tfull_bar(buf), (eph >> buf) & 1u, abort_flag, a.timeout_ns);
         if (!__all_sync(0xffffffffu, got)) {
           give_up();
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t taddr = tmem_base + lane_addr + acc * ACC_COLS;
+        const uint32_t taddr = tmem_base + lane_addr + buf * ACC_COLS;
         epi_lse_tile(a, taddr, nb, st);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (lane == 0) mbar_arrive_cluster(buf == 0 ? tempty_leader0 : tempty_leader1);
+        eph ^= 1u << buf;
+        if (!second && nb + 1 == nb1) acc ^= 1;  // a lone last tile
       }
       if (ok && st.row < a.N) {
         a.part_m[static_cast<size_t>(split + a.split_off) * a.N + st.row] = st.run_m;
@@ -737,7 +797,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     }
   }
 
-  pair_wind_down(smem_u32(bars), tmem_slot, rank, warp, abort_flag, a.status, a.timeout_ns);
+  pair_wind_down<P1_STAGES>(smem_u32(bars), tmem_slot, rank, warp, abort_flag, a.status, a.timeout_ns);
 }
 
 // ===================================================== pass 2, one launch ==
@@ -1063,7 +1123,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
           }
         }
       }
-      producer_tail(smem_u32(bars), tmem_slot, filled, stage, phase, abort_flag, a.timeout_ns, rank, a.status);
+      producer_tail<STAGES>(smem_u32(bars), tmem_slot, filled, stage, phase, abort_flag, a.timeout_ns, rank,
+                            a.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ UMMA issuer (leader) --
@@ -1338,7 +1399,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
     if (lane == 0) bulk_wait<0>();
   }
 
-  pair_wind_down(smem_u32(bars), tmem_slot, rank, warp, abort_flag, a.status, a.timeout_ns);
+  pair_wind_down<STAGES>(smem_u32(bars), tmem_slot, rank, warp, abort_flag, a.status, a.timeout_ns);
 }
 
 // ---------------------------------------------------------------- prep --
