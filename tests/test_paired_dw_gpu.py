@@ -59,3 +59,35 @@ def test_paired_dw_items_repeat_bit_identically():
     _, dX1, dW1 = F.forward_backward(X, W, y)
     _, dX2, dW2 = F.forward_backward(X, W, y)
     assert torch.equal(dX1, dX2) and torch.equal(dW1, dW2)
+
+
+@pytest.mark.parametrize("w", PAIRED[1:3], ids=lambda w: w.name)
+def test_paired_dw_items_through_the_host_entry(w):
+    """The host-buffer entry: W in pieces (pass 1 per piece), pass 2 in
+    sections with dW copied back per section, on shapes that pair dW items."""
+    F = _lib()
+    X, W, y = make_inputs(w)
+    hX, hW, hy = X.pin_memory(), W.pin_memory(), y.pin_memory()
+    dev = (torch.empty_like(X, device="cuda"), torch.empty_like(W, device="cuda"),
+           torch.empty_like(y, device="cuda"), torch.empty_like(X, device="cuda"),
+           torch.empty_like(W, device="cuda"), F.alloc_workspace(w.N, w.H, w.V))
+    loss, hdX, hdW = F.forward_backward_host(hX, hW, hy, dev)
+    check_against_full_oracle(X, W, y, loss, hdX, hdW, w.name + " host", n_expected=w.N - w.n_ignored)
+
+
+@pytest.mark.parametrize("sections", [1, 3, 8])
+def test_paired_dw_items_in_sections_match_one_launch(sections):
+    """Pass 2 split into launches over whole chunks runs the same items in
+    the same order: bit-identical to the single launch."""
+    F = _lib()
+    w = PAIRED[2]
+    X, W, y = (t.cuda() for t in make_inputs(w))
+    ws = F.alloc_workspace(w.N, w.H, w.V)
+    l1, s1, dX1, dW1 = F.forward_backward_async(X, W, y, workspace=ws)
+    torch.cuda.synchronize()
+    dX1, dW1, l1 = dX1.clone(), dW1.clone(), l1.item()
+    l2, s2, dX2, dW2, events, rows = F.forward_backward_sections(X, W, y, sections=sections, workspace=ws)
+    torch.cuda.synchronize()
+    assert s1.item() == 0 and s2.item() == 0
+    assert rows[0] == 0 and rows[-1] == w.V
+    assert l2.item() == l1 and torch.equal(dX2, dX1) and torch.equal(dW2, dW1)
