@@ -105,6 +105,28 @@ def recorded_traffic(kernel: str, workload: str):
         return None
 
 
+def timeline_summary(tl):
+    """Spans of one host-buffer call from its recorded intervals [(kind name,
+    begin ms, end ms)]: the X/y copy, the W pieces, pass 1 per piece, pass 2
+    per section, the dW copies per section, then dX and the loss."""
+    def span(items):
+        return [round(min(b for _, b, _ in items), 3), round(max(e for _, _, e in items), 3)] if items else None
+    h2d = [t for t in tl if t[0] == "copy_host_to_device"]
+    d2h = [t for t in tl if t[0] == "copy_device_to_host"]
+    p1 = [t for t in tl if t[0] == "pass1_logits_lse"]
+    p2 = [t for t in tl if t[0] == "pass2_grad_dw_dx"]
+    out = {"x_y_to_device": span(h2d[:1]), "w_pieces_to_device": span(h2d[1:]), "pass1_pieces": span(p1),
+           "pass2_sections": span(p2), "dw_sections_to_host": span(d2h[:-1]), "dx_loss_to_host": span(d2h[-1:]),
+           "end": round(max(e for _, _, e in tl), 3) if tl else None,
+           "counts": {"w_pieces": len(h2d) - 1, "pass1_launches": len(p1), "pass2_launches": len(p2)}}
+    if p2 and len(h2d) > 1:
+        out["critical_path"] = {"w_copy": round(out["w_pieces_to_device"][1], 3),
+                                "w_landed_to_pass2": round(out["pass2_sections"][0] - out["w_pieces_to_device"][1], 3),
+                                "pass2": round(out["pass2_sections"][1] - out["pass2_sections"][0], 3),
+                                "after_pass2": round(out["end"] - out["pass2_sections"][1], 3)}
+    return out
+
+
 # ----------------------------------------------------------------- clocks --
 class ClockSampler:
     """nvidia-smi sampled every 200 ms while the timed region runs."""
@@ -434,6 +456,12 @@ def run_ours(args, world, rank, local):
         e2e = {"value": world * N / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "path": "flce_forward_backward_host: pinned host X,W,y -> device, compute, dX,dW,loss -> pinned host"}
+        # one more call, untimed, with its copies and launches on the library's
+        # record: where the time goes (CUDA events, ms after the first copy)
+        F.profile_enable(True)
+        F.forward_backward_host(hX, hW, hy, dbufs, h_out=h_out, stream=stream)
+        e2e["timeline_ms"] = timeline_summary(F.profile_timeline())
+        F.profile_enable(False)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -396,6 +396,23 @@ const char* flce_kernel_name(int kind);
 flce_status_t flce_profile_enable(int on);
 flce_status_t flce_profile_read(int32_t* launches, double* total_ms);
 
+/* Timeline of what the record holds, in the order it was recorded: the
+ * launches (kinds as above) and, for the host-buffer entry
+ * (flce_forward_backward_host), its copies: kind 8 host to device (X and y
+ * on the caller's stream, each W piece on the copy stream), kind 9 device to
+ * host (each section's dW rows on the copy stream, then dX and the loss on
+ * the caller's stream); flce_kernel_name names them too.  Waits for the
+ * recorded events and writes, for the first `capacity` intervals, kinds[i]
+ * and their begin and end in milliseconds after the begin of the first
+ * interval (HOST arrays of `capacity` entries); *count receives the number
+ * recorded, which may exceed capacity.  Clears the record, as
+ * flce_profile_read does.  FLCE_ERR_INVALID_ARGUMENT for a NULL pointer or a
+ * negative capacity. */
+#define FLCE_PROFILE_KIND_H2D 8
+#define FLCE_PROFILE_KIND_D2H 9
+flce_status_t flce_profile_timeline(int32_t* kinds, double* begin_ms, double* end_ms, int32_t capacity,
+                                    int32_t* count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,6 +20,7 @@ from .flce import (  # noqa: F401
     plan,
     profile_enable,
     profile_read,
+    profile_timeline,
     reorder_fits,
     row_order_info,
     vp_backward,

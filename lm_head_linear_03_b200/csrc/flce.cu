@@ -641,10 +641,14 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
           pp.section_rows[k + 1] = r1;
         }
         if (cudaEventRecord(pp.p2_done[k], stream) != cudaSuccess) return cuda_fail(__LINE__);
-        if (pp.h_dW && (cudaStreamWaitEvent(pp.copy, pp.p2_done[k], 0) != cudaSuccess ||
-                        cudaMemcpyAsync(pp.h_dW + r0 * H, dW + r0 * H, static_cast<size_t>(r1 - r0) * H * 2,
-                                        cudaMemcpyDeviceToHost, pp.copy) != cudaSuccess))
-          return cuda_fail(__LINE__);
+        if (pp.h_dW) {
+          if (cudaStreamWaitEvent(pp.copy, pp.p2_done[k], 0) != cudaSuccess) return cuda_fail(__LINE__);
+          prof_begin(pp.copy, KIND_D2H, &slot);
+          if (cudaMemcpyAsync(pp.h_dW + r0 * H, dW + r0 * H, static_cast<size_t>(r1 - r0) * H * 2,
+                              cudaMemcpyDeviceToHost, pp.copy) != cudaSuccess)
+            return cuda_fail(__LINE__);
+          prof_end(pp.copy, slot);
+        }
       }
     }
     // reordered rows: the final dX rows go back in place (no-op otherwise)
@@ -974,9 +978,12 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
   std::lock_guard<std::mutex> lk(pr->mu);  // one host-buffer call per device at a time: shared copy stream
   const size_t xb = static_cast<size_t>(N) * H * 2, yb = N * 4;
   // X and y first, on the caller's stream: every kernel needs them
+  size_t slot;
+  prof_begin(stream, KIND_H2D, &slot);
   if (cudaMemcpyAsync(d_X, h_X, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
       cudaMemcpyAsync(d_y, h_y, yb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return cuda_fail(__LINE__);
+  prof_end(stream, slot);
   // W in pieces on the copy stream, which starts after the caller's earlier work
   PipeCtx pp;
   pp.copy = pr->copy;
@@ -991,10 +998,12 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
     const int64_t v0 = pp.piece_v[i], v1 = pp.piece_v[i + 1];
     pp.w_ready[i] = pr->ev[i];
     pp.p2_done[i] = pr->ev[MAX_PIECES + i];
+    prof_begin(pr->copy, KIND_H2D, &slot);
     if (cudaMemcpyAsync(d_W + v0 * H, h_W + v0 * H, static_cast<size_t>(v1 - v0) * H * 2, cudaMemcpyHostToDevice,
-                        pr->copy) != cudaSuccess ||
-        cudaEventRecord(pp.w_ready[i], pr->copy) != cudaSuccess)
+                        pr->copy) != cudaSuccess)
       return cuda_fail(__LINE__);
+    prof_end(pr->copy, slot);
+    if (cudaEventRecord(pp.w_ready[i], pr->copy) != cudaSuccess) return cuda_fail(__LINE__);
   }
   for (int i = pp.pieces; i < MAX_PIECES; ++i) pp.p2_done[i] = pr->ev[MAX_PIECES + i];
   Options opt;
@@ -1008,9 +1017,12 @@ flce_status_t flce_forward_backward_host(const uint16_t* h_X, const uint16_t* h_
   }
   // dX and the control block on the caller's stream; dW went back section by section
   Ctrl host{};
+  prof_begin(stream, KIND_D2H, &slot);
   if (cudaMemcpyAsync(h_dX, d_dX, xb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-      cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-      cudaEventRecord(pr->done, pr->copy) != cudaSuccess || cudaStreamWaitEvent(stream, pr->done, 0) != cudaSuccess)
+      cudaMemcpyAsync(&host, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return cuda_fail(__LINE__);
+  prof_end(stream, slot);
+  if (cudaEventRecord(pr->done, pr->copy) != cudaSuccess || cudaStreamWaitEvent(stream, pr->done, 0) != cudaSuccess)
     return cuda_fail(__LINE__);
   if (cudaStreamSynchronize(stream) != cudaSuccess) return cuda_fail(__LINE__);
   *h_loss = host.loss;
@@ -1086,6 +1098,8 @@ const char* flce_kernel_name(int kind) {
     case KIND_ORDER: return "prep_row_order";
     case KIND_SCATTER: return "dx_row_scatter";
     case KIND_PACK: return "prep_pack_rows";
+    case KIND_H2D: return "copy_host_to_device";
+    case KIND_D2H: return "copy_device_to_host";
     default: return "unknown";
   }
 }
@@ -1121,11 +1135,31 @@ flce_status_t flce_profile_read(int32_t* launches, double* total_ms) {
     total_ms[k] = 0.0;
   }
   for (size_t i = 0; i < g_prof.used; ++i) {
+    if (g_prof.kind[i] >= FLCE_NUM_KERNEL_KINDS) continue;  // copies: see flce_profile_timeline
     if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return cuda_fail(__LINE__);
     float ms = 0.f;
     if (cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) return cuda_fail(__LINE__);
     launches[g_prof.kind[i]] += 1;
     total_ms[g_prof.kind[i]] += ms;
+  }
+  g_prof.used = 0;
+  return FLCE_OK;
+}
+
+flce_status_t flce_profile_timeline(int32_t* kinds, double* begin_ms, double* end_ms, int32_t capacity,
+                                    int32_t* count) {
+  if (!kinds || !begin_ms || !end_ms || !count || capacity < 0) return FLCE_ERR_INVALID_ARGUMENT;
+  *count = static_cast<int32_t>(g_prof.used);
+  for (size_t i = 0; i < g_prof.used; ++i) {
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return cuda_fail(__LINE__);
+    if (static_cast<int64_t>(i) >= capacity) continue;
+    float b = 0.f, e = 0.f;
+    if (cudaEventElapsedTime(&b, g_prof.ev[0], g_prof.ev[2 * i]) != cudaSuccess ||
+        cudaEventElapsedTime(&e, g_prof.ev[0], g_prof.ev[2 * i + 1]) != cudaSuccess)
+      return cuda_fail(__LINE__);
+    kinds[i] = g_prof.kind[i];
+    begin_ms[i] = b;
+    end_ms[i] = e;
   }
   g_prof.used = 0;
   return FLCE_OK;

@@ -107,7 +107,7 @@ __host__ __device__ __forceinline__ int target_elsewhere(int ignore_index) {
 // Kinds of launch, as the profiler reports them.
 enum : int {
   KIND_LSE = 0, KIND_COMBINE = 1, KIND_PASS2 = 2, KIND_PREP = 3, KIND_CE = 4, KIND_ORDER = 5, KIND_SCATTER = 6,
-  KIND_PACK = 7
+  KIND_PACK = 7, KIND_H2D = 8, KIND_D2H = 9  // the last two: copies of the host-buffer entry (profiling only)
 };
 enum : int { ST_TARGET_OUT_OF_RANGE = 4, ST_TIMEOUT = 5 };
 

@@ -39,6 +39,7 @@ EXPORTED = (
     "flce_kernel_name",
     "flce_profile_enable",
     "flce_profile_read",
+    "flce_profile_timeline",
     "flce_forward_backward_noalloc",
     "flce_forward_backward_ex",
     "flce_ce_workspace_size",
@@ -115,6 +116,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flce_profile_enable.restype = ctypes.c_int
     lib.flce_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)]
     lib.flce_profile_read.restype = ctypes.c_int
+    lib.flce_profile_timeline.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double),
+                                          ctypes.POINTER(ctypes.c_double), ctypes.c_int32,
+                                          ctypes.POINTER(ctypes.c_int32)]
+    lib.flce_profile_timeline.restype = ctypes.c_int
     lib.flce_forward_backward_ex.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                              vp]
     lib.flce_forward_backward_ex.restype = ctypes.c_int
@@ -457,6 +462,18 @@ def profile_read():
     _check(lib.flce_profile_read(n, ms), "flce_profile_read")
     names = kernel_names()
     return {names[k]: (int(n[k]), float(ms[k])) for k in range(NUM_KERNEL_KINDS)}
+
+
+def profile_timeline(capacity: int = 4096):
+    """[(name, begin ms, end ms)] of every recorded launch and host-buffer
+    copy since the last read, in record order, relative to the first begin."""
+    lib = load_library()
+    kinds = (ctypes.c_int32 * capacity)()
+    b = (ctypes.c_double * capacity)()
+    e = (ctypes.c_double * capacity)()
+    n = ctypes.c_int32()
+    _check(lib.flce_profile_timeline(kinds, b, e, capacity, ctypes.byref(n)), "flce_profile_timeline")
+    return [(lib.flce_kernel_name(kinds[i]).decode(), float(b[i]), float(e[i])) for i in range(min(n.value, capacity))]
 
 
 def forward_backward_noalloc(X, W, y, ignore_index: int = -100, *, dX=None, dW=None, stream=None):

@@ -120,3 +120,22 @@ def test_clock_records_rejected_or_kept():
               {"sm_mhz": 1100.0, "sm_max_mhz": 1965.0, "reasons": []}]   # held low with no reason: a clock lock
     assert not any(bench.clocks_rejected(c) for c in keep)
     assert all(bench.clocks_rejected(c) for c in reject)
+
+
+def test_timeline_summary_spans():
+    """bench.timeline_summary on a made-up record: spans by kind, and the
+    critical path W copy -> pass 2 -> what follows it."""
+    import bench
+    tl = [("copy_host_to_device", 0.0, 1.0)] + \
+         [("copy_host_to_device", 1.0 + i, 2.0 + i) for i in range(4)] + \
+         [("pass1_logits_lse", 2.0 + i, 2.5 + i) for i in range(4)] + \
+         [("combine_lse_loss", 5.5, 5.6)] + \
+         [("pass2_grad_dw_dx", 6.0 + i, 7.0 + i) for i in range(3)] + \
+         [("copy_device_to_host", 7.0 + i, 7.5 + i) for i in range(3)] + \
+         [("copy_device_to_host", 9.5, 10.0)]
+    s = bench.timeline_summary(tl)
+    assert s["x_y_to_device"] == [0.0, 1.0] and s["w_pieces_to_device"] == [1.0, 5.0]
+    assert s["pass1_pieces"] == [2.0, 5.5] and s["pass2_sections"] == [6.0, 9.0]
+    assert s["dw_sections_to_host"] == [7.0, 9.5] and s["dx_loss_to_host"] == [9.5, 10.0] and s["end"] == 10.0
+    assert s["counts"] == {"w_pieces": 4, "pass1_launches": 4, "pass2_launches": 3}
+    assert s["critical_path"] == {"w_copy": 5.0, "w_landed_to_pass2": 1.0, "pass2": 3.0, "after_pass2": 1.0}
