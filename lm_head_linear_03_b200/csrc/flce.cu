@@ -197,7 +197,7 @@ bool get_encode() {
 
 // 2-D bf16 row-major tensor [outer][inner], 128-B swizzled boxes of
 // box_inner x box_outer elements; out-of-range elements read as zero.
-enum class Swz { k128, k64, none };
+enum class Swz { k128, k64 };
 
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
               uint32_t box_inner, uint32_t box_outer, Swz swz = Swz::k128) {
@@ -207,9 +207,7 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              swz == Swz::k128  ? CU_TENSOR_MAP_SWIZZLE_128B
-                              : swz == Swz::k64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                : CU_TENSOR_MAP_SWIZZLE_NONE,
+                              swz == Swz::k128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -411,15 +409,13 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
   const float* g_rows = opt.grad_row_scale ? g_perm : nullptr;  // upstream weights in the rows' order
   uint16_t* Xc = L.packed ? reinterpret_cast<uint16_t*>(ws + L.xc) : nullptr;
 
-  CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn, mHi, mLo, mXc_k, mXc_mn;
+  CUtensorMap mX_k, mW_k, mG_mn, mX_mn, mG_k, mW_mn, mXc_k, mXc_mn;
   const uint64_t n = static_cast<uint64_t>(N), h = static_cast<uint64_t>(H), v = static_cast<uint64_t>(V);
   bool ok = make_map(&mX_k, X, h, n, h * 2, BK, BM) && make_map(&mW_k, W, h, v, h * 2, BK, BNH) &&
             make_map(&mG_mn, G, VC, n, VC * 2, 64, BK) && make_map(&mX_mn, X, h, n, h * 2, 64, BK) &&
             make_map(&mG_k, G, VC, n, VC * 2, BK, BM) && make_map(&mW_mn, W, h, v, h * 2, 64, BK) &&
             // the packed copy of X (the caller's X stands in when there is none: never read then)
-            make_map(&mXc_k, Xc ? Xc : X, h, n, h * 2, BK, BM) && make_map(&mXc_mn, Xc ? Xc : X, h, n, h * 2, 64, BK) &&
-            (dX == nullptr || (make_map(&mHi, dX, h, n, h * 2, BN, BM, Swz::none) &&
-                               make_map(&mLo, lo, h, n, h * 2, BN, BM, Swz::none)));
+            make_map(&mXc_k, Xc ? Xc : X, h, n, h * 2, BK, BM) && make_map(&mXc_mn, Xc ? Xc : X, h, n, h * 2, 64, BK);
   // 32 x 32 output boxes of the epilogues (64-byte swizzle)
   CUtensorMap mGo, mDWo, mHio, mLoo;
   ok = ok && (dX == nullptr || (make_map(&mGo, G, VC, n, VC * 2, EPI_BOX, EPI_BOX, Swz::k64) &&
@@ -607,8 +603,6 @@ flce_status_t enqueue(const uint16_t* X, const uint16_t* W, const int32_t* y, in
     pm.DWo = mDWo;
     pm.Hio = mHio;
     pm.Loo = mLoo;
-    pm.Hipf = mHi;
-    pm.Lopf = mLo;
     pm.Xck = mXc_k;
     pm.Xcmn = mXc_mn;
     // one launch over the whole queue; a host-buffer call splits it into

@@ -939,7 +939,6 @@ struct Pass2Maps {
   CUtensorMap Gk, Wmn;     // dX: G_c rows K-major, W_c MN-major
   CUtensorMap Go, DWo;     // epilogue output boxes of G and dW
   CUtensorMap Hio, Loo;    // epilogue boxes of the dX running sum (hi = dX, lo)
-  CUtensorMap Hipf, Lopf;  // whole-tile L2 prefetch of the running sum
   CUtensorMap Xck, Xcmn;   // the packed copy of X (reordered rows), K- and MN-major
 };
 
@@ -1014,7 +1013,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
-      const uint64_t keep = l2_evict_last(), normal = l2_evict_normal(), stream = l2_evict_first();
+      const uint64_t keep = l2_evict_last(), normal = l2_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       long long filled = 0;
@@ -1038,12 +1037,6 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NUM_THREADS, 1
         } else {
           kblocks = (vcount + BK - 1) / BK;
           ok = wait_counter(a.g_row + it.a, g_row_target(it.c), abort_flag, a.timeout_ns);
-          // pull this CTA's rows of the running sum into L2 if they are final already
-          if (ok && it.c > 0 && ld_acquire_gpu(a.x_row + it.a) >= SIGNALS_PER_ITEM * it.c * a.HN) {
-            fence_proxy_async_global();
-            tma_prefetch_l2_2d(&m.Hipf, it.b * BN, it.a * CM + rank * BM, stream);
-            tma_prefetch_l2_2d(&m.Lopf, it.b * BN, it.a * CM + rank * BM, stream);
-          }
         }
         if (!ok) {
           give_up();
