@@ -225,8 +225,9 @@ struct Plan {
 
 // Pass 1: pick the number of vocabulary splits whose units, dealt round-robin
 // to the persistent SM pairs, give the smallest largest per-pair load.  A unit
-// walks its tiles in pairs (256 x 512), a pair costing about 1.6 lone tiles,
-// plus one tile's worth for its pipeline fill and partial write.
+// walks its tiles in pairs (256 x 512), a pair costing about 1.6 lone tiles
+// (an estimate from the tiles' k-block rates; counting one per tile measured
+// the same), plus one tile's worth for its pipeline fill and partial write.
 int choose_splits(int tiles_m, int vtiles, int sms) {
   int best = 1;
   long long best_cost = LLONG_MAX;
