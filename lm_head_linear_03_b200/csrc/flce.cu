@@ -195,8 +195,9 @@ bool get_encode() {
   return true;
 }
 
-// 2-D bf16 row-major tensor [outer][inner], 128-B swizzled boxes of
-// box_inner x box_outer elements; out-of-range elements read as zero.
+// 2-D bf16 row-major tensor [outer][inner], boxes of box_inner x box_outer
+// elements with the 128-B swizzle (operands) or the 64-B one (the epilogues'
+// 32 x 32 boxes); out-of-range elements read as zero.
 enum class Swz { k128, k64 };
 
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,

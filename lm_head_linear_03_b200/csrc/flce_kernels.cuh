@@ -25,7 +25,11 @@
 // 256 x 256 accumulator tile: each CTA loads 128 rows of A and 128 columns of B
 // into its own shared memory, the leader CTA issues cta_group::2 UMMAs that read
 // both halves, and each CTA's tensor memory receives its 128 rows.  Per SM this
-// halves the B-operand traffic of a 128 x 256 single-CTA tile.
+// halves the B-operand traffic of a 128 x 256 single-CTA tile.  Pass 1, and
+// pass 2's dW items where its queue pairs them, take two adjacent 256-column
+// tiles as one 256 x 512 tile in both accumulator buffers: two UMMAs per
+// k-block share the A tile, so a k-block reads 48 KB of operands for twice
+// the work of a 32 KB one (see the pass-1 issuer and the pass-2 queue).
 //
 // Warp roles (192 threads per CTA): warp 0 issues TMA loads, warp 1 issues UMMAs
 // (leader CTA only) and owns the tensor-memory allocation, warps 2..5 run the
