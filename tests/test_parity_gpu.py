@@ -312,15 +312,18 @@ def test_bounded_waits_give_up_and_report_timeout():
     run_full_oracle_case(*make_inputs(WORKLOADS["tiny"]))
 
 
-def test_pass2_starved_waits_give_up_and_report_timeout():
+@pytest.mark.parametrize("shape", [(700, 256, 5000), (7424, 1024, 4100)], ids=["single_dw", "paired_dw"])
+def test_pass2_starved_waits_give_up_and_report_timeout(shape):
     """The GEMM kernels' own waits: a call whose dW items wait for one more
     G tile than the queue produces ends with FLCE_ERR_TIMEOUT within seconds
     (each SM pair winds down, both CTAs together), and the next call on the
-    device matches the oracle."""
+    device matches the oracle.  The second shape runs its dW items as paired
+    256 x 512 tiles (a chunk holds more than three rounds of G tiles)."""
     _lib()
     from lm_head_linear_03_b200 import flce
     import time
-    w = custom("starved_dw", N=700, H=256, V=5000, ignore_frac=0.1)
+    N, H, V = shape
+    w = custom(f"starved_dw_{N}", N=N, H=H, V=V, ignore_frac=0.1)
     X, W, y = make_inputs(w)
     Xd, Wd, yd = X.cuda(), W.cuda(), y.cuda()
     torch.cuda.synchronize()
