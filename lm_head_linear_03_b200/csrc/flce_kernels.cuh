@@ -471,7 +471,10 @@ __device__ __forceinline__ void epi_dx_tile(const GemmArgs& a, bool first_chunk,
 //     stopped at different positions can a load be left that no barrier
 //     reports; a fixed 100 us grace period covers that case.
 // Every wait here ends by completion or by its own time limit, not by the
-// abort flag.
+// abort flag.  NST is the kernel's ring length (pass 1: P1_STAGES, pass 2:
+// STAGES); both kernels lay their barriers out as pass 2 does, so the full
+// barrier of ring position q is barrier q % NST and its empty barrier
+// STAGES + q % NST.
 template <int NST>
 __device__ __forceinline__ void pair_wind_down(uint32_t bars, const uint32_t* slots, int rank, int warp,
                                                volatile int* abort_flag, int* status, unsigned long long timeout_ns) {
@@ -513,7 +516,8 @@ __device__ __forceinline__ void pair_wind_down(uint32_t bars, const uint32_t* sl
 // The producer's tail: wait for the UMMA commits still headed for this CTA's
 // empty barriers, so none lands after the CTA has gone, and record how far it
 // filled the ring.  After a give-up the peer's producer (which cannot see the
-// leader's full barriers) lets copies in flight land for 100 us.
+// leader's full barriers) lets copies in flight land for 100 us.  NST: the
+// ring length, as for pair_wind_down (empty barriers at STAGES + stage).
 template <int NST>
 __device__ __forceinline__ void producer_tail(uint32_t bars, uint32_t* slots, long long filled, int& stage,
                                               uint32_t& phase, volatile int* abort_flag,
